@@ -1,0 +1,335 @@
+"""Checks that pin the CPU oracle to facts outside itself: hand-worked
+fixtures (tests/golden), brute-force enumeration on tiny inputs with scores
+computed by explicit loops, closed forms, special cases that reduce to a
+library routine, and invariants of the method.
+
+Each check is a plain function that raises AssertionError; the pytest module
+test_oracle_pins.py runs them, and test_oracle_mutations.py plants mistakes in
+the oracle and verifies that some check catches each one.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import os
+
+import numpy as np
+import torch
+
+from oracle import hisa_oracle as ho
+from oracle import ofp8
+from oracle.run import Sequence
+from hierarchical_top_key_b200 import synthetic
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- golden
+
+
+def pin_golden_flat():
+    g = _load("flat_relu_weights.json")
+    q, w, keys = (np.array(g[k], np.float64) for k in ("q", "w", "keys"))
+    np.testing.assert_array_equal(ho.indexer_scores(q, w, keys), np.array(g["scores"], np.float64))
+    for c in g["cases"]:
+        idx, _ = ho.flat_query(q, w, keys, c["n_visible"], c["top_k"])
+        assert list(idx) == c["indices"], (c, list(idx))
+
+
+def _golden_hisa(name):
+    g = _load(name)
+    B = g["block_size"]
+    q, w, keys = (np.array(g[k], np.float64) for k in ("q", "w", "keys"))
+    kp = ho.pool_blocks(keys, B, "f32")
+    np.testing.assert_array_equal(kp[:, 0], np.array(g["pooled"], np.float64))
+    for c in g["cases"]:
+        blocks, idx, _ = ho.hisa_query(q, w, keys, kp, c["n_visible"], B, c["top_m"], c["top_k"])
+        assert list(blocks) == c["blocks"], (name, c, list(blocks))
+        assert list(idx) == c["indices"], (name, c, list(idx))
+    for c in g.get("flat_cases", []):
+        idx, _ = ho.flat_query(q, w, keys, c["n_visible"], c["top_k"])
+        assert list(idx) == c["indices"], (name, c, list(idx))
+
+
+def pin_golden_hisa_blocks():
+    _golden_hisa("hisa_blocks_1d.json")
+
+
+def pin_golden_relu_of_mean():
+    _golden_hisa("hisa_relu_of_mean.json")
+
+
+def pin_golden_e4m3():
+    g = _load("ofp8_e4m3.json")
+    xs = np.array([e["x"] for e in g["encode"]])
+    codes = np.array([e["code"] for e in g["encode"]], np.uint8)
+    np.testing.assert_array_equal(ofp8.e4m3_encode(xs), codes)
+    dc = np.array([e["code"] for e in g["decode"]], np.uint8)
+    np.testing.assert_array_equal(ofp8.e4m3_decode(dc), np.array([e["x"] for e in g["decode"]]))
+    assert np.all(np.isnan(ofp8.e4m3_decode(np.array(g["nan_codes"], np.uint8))))
+
+
+def pin_golden_bf16():
+    g = _load("bf16_round.json")
+    xs = np.array([c["x"] for c in g["cases"]], np.float64)
+    np.testing.assert_array_equal(ofp8.bf16_round(xs), np.array([c["bf16"] for c in g["cases"]]))
+
+
+# ---------------------------------------------------------------- library special cases
+
+
+def pin_e4m3_matches_torch_in_range():
+    """Inside +-448 saturation plays no part, and E4M3 round-to-nearest-even
+    is what torch's float8_e4m3fn cast does."""
+    rng = np.random.default_rng(11)
+    x = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.05, 1, 30, 200)])
+    x = np.clip(x, -447, 447).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(ofp8.e4m3_encode(x), ref)
+    allc = np.arange(256, dtype=np.uint8)
+    fin = ~np.isnan(ofp8.e4m3_decode(allc))
+    tv = torch.from_numpy(allc).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(ofp8.e4m3_decode(allc)[fin], tv[fin])
+
+
+def pin_bf16_matches_torch_on_fp32_values():
+    """For values already in fp32, one bf16 rounding equals torch's cast."""
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal(50000) * np.exp(rng.uniform(-20, 20, 50000))).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(ofp8.bf16_round(x.astype(np.float64)), ref)
+
+
+def _loop_scores(q, w, keys):
+    """Indexer scores by explicit loops (no matrix routines)."""
+    H, d = q.shape
+    out = []
+    for s in range(keys.shape[0]):
+        tot = 0.0
+        for h in range(H):
+            dot = 0.0
+            for i in range(d):
+                dot += float(q[h, i]) * float(keys[s, i])
+            tot += float(w[h]) * max(dot, 0.0)
+        out.append(tot)
+    return np.array(out)
+
+
+def pin_single_head_unit_weight_is_sort():
+    """H=1, w=1: flat top-k is a stable descending sort of ReLU(q.k)."""
+    rng = np.random.default_rng(13)
+    for trial in range(20):
+        n, d, k = int(rng.integers(1, 40)), int(rng.integers(1, 6)), int(rng.integers(1, 12))
+        q = rng.integers(-3, 4, (1, d)).astype(np.float64)
+        keys = rng.integers(-3, 4, (n, d)).astype(np.float64)
+        s = np.maximum(keys @ q[0], 0)
+        ref = np.argsort(-s, kind="stable")[:k]
+        idx, sc = ho.flat_query(q, np.ones(1), keys, n, k)
+        assert list(idx) == list(ref), (trial, list(idx), list(ref))
+        np.testing.assert_array_equal(sc, s[ref])
+
+
+# ---------------------------------------------------------------- brute force
+
+
+def _brute_topk(scores, k):
+    """Best-sum k-subset; among equal sums the lexicographically smallest
+    sorted index tuple (ties go to lower indices)."""
+    n = len(scores)
+    k = min(k, n)
+    best, best_sum = None, None
+    for comb in itertools.combinations(range(n), k):
+        s = sum(scores[i] for i in comb)
+        if best_sum is None or s > best_sum:
+            best, best_sum = comb, s
+    return set(best) if best is not None else set()
+
+
+def pin_brute_force_flat():
+    rng = np.random.default_rng(14)
+    for trial in range(60):
+        n = int(rng.integers(1, 13))
+        H, d = int(rng.integers(1, 3)), int(rng.integers(1, 4))
+        k = int(rng.integers(1, 7))
+        q = rng.integers(-2, 3, (H, d)).astype(np.float64)
+        w = rng.integers(0, 3, H).astype(np.float64)
+        keys = rng.integers(-2, 3, (n, d)).astype(np.float64)
+        nt = int(rng.integers(0, n + 1))
+        ref = _loop_scores(q, w, keys)
+        np.testing.assert_array_equal(ho.indexer_scores(q, w, keys), ref)
+        idx, _ = ho.flat_query(q, w, keys, nt, k)
+        assert set(idx.tolist()) == _brute_topk(ref[:nt], k), (trial, idx, ref[:nt])
+        assert len(idx) == min(k, nt)
+
+
+def pin_brute_force_hisa():
+    """Enumerate the m-1 blocks before the current one and the k candidates."""
+    rng = np.random.default_rng(15)
+    for trial in range(60):
+        B = int(rng.integers(1, 4))
+        L = int(rng.integers(1, 16))
+        H, d = int(rng.integers(1, 3)), int(rng.integers(1, 3))
+        m, k = int(rng.integers(1, 5)), int(rng.integers(1, 6))
+        q = rng.integers(-2, 3, (H, d)).astype(np.float64)
+        w = rng.integers(0, 3, H).astype(np.float64)
+        keys = rng.integers(-3, 4, (L, d)).astype(np.float64)
+        nt = int(rng.integers(1, L + 1))
+        # pooled keys by explicit loops: block sums / counts (exact for these sizes)
+        nb = -(-L // B)
+        kp = np.zeros((nb, d))
+        for b in range(nb):
+            members = list(range(b * B, min((b + 1) * B, L)))
+            for i in range(d):
+                kp[b, i] = sum(keys[s, i] for s in members) / len(members)
+        kp = kp.astype(np.float32).astype(np.float64)
+        np.testing.assert_array_equal(ho.pool_blocks(keys, B, "f32"), kp)
+        c = (nt - 1) // B
+        bscore = _loop_scores(q, w, kp[:c])
+        if c + 1 <= m:
+            want_blocks = set(range(c + 1))
+        else:
+            want_blocks = _brute_topk(list(bscore), m - 1) | {c}
+        blocks, idx, _ = ho.hisa_query(q, w, keys, kp, nt, B, m, k)
+        assert set(blocks.tolist()) == want_blocks, (trial, blocks, want_blocks)
+        cand = [s for b in sorted(want_blocks) for s in range(b * B, min((b + 1) * B, nt))]
+        tok = _loop_scores(q, w, keys[cand]) if cand else np.zeros(0)
+        want = {cand[i] for i in _brute_topk(list(tok), k)}
+        assert set(idx.tolist()) == want, (trial, idx, want)
+
+
+# ---------------------------------------------------------------- closed forms / special cases
+
+
+def pin_pool_closed_forms():
+    rng = np.random.default_rng(16)
+    keys = rng.standard_normal((37, 5)).astype(np.float32).astype(np.float64)
+    # block size 1: pooled keys are the keys
+    np.testing.assert_array_equal(ho.pool_blocks(keys, 1, "f32"), keys)
+    # arithmetic progression along the sequence: block mean = midpoint
+    ap = np.arange(40, dtype=np.float64)[:, None] * np.ones((1, 3)) * 2.0
+    kp = ho.pool_blocks(ap, 8, "f32")
+    np.testing.assert_array_equal(kp[:, 0], np.array([7, 23, 39, 55, 71], np.float64))
+    # ragged tail: block of 5 keys (35..39) has mean 74
+    kp = ho.pool_blocks(ap, 7, "f32")
+    assert kp[-1, 0] == 74.0 and kp.shape[0] == 6
+    # compression of constant groups
+    const = np.repeat(np.arange(6, dtype=np.float64), 4)[:, None] * np.ones((1, 2))
+    ck = ho.compress_keys(np.concatenate([const, np.ones((3, 2)) * 99]), 4, "bf16")
+    np.testing.assert_array_equal(ck[:, 0], np.arange(6, dtype=np.float64))
+    # mean rounded once to bf16: (1 + (1 + 2^-7)) / 2 = 1 + 2^-8 -> tie -> 1.0
+    two = np.array([[1.0], [1.0 + 2 ** -7]])
+    assert ho.pool_blocks(two, 2, "bf16")[0, 0] == 1.0
+
+
+def pin_m_all_blocks_equals_flat():
+    inp = synthetic.generate(synthetic.small_case(num_keys=333, heads=3, head_dim=8, block_size=16,
+                                                  top_m=1000, top_k=25, needles=3))
+    seq = Sequence(inp, 0)
+    for t in range(0, 333, 7):
+        _, hi, hs = seq.hisa(t)
+        fi, fs = seq.flat(t)
+        assert list(hi) == list(fi), t
+        np.testing.assert_array_equal(hs, fs)
+
+
+def pin_m_one_is_current_block():
+    inp = synthetic.generate(synthetic.small_case(num_keys=200, heads=2, head_dim=4, block_size=10,
+                                                  top_m=1, top_k=50, needles=0))
+    seq = Sequence(inp, 0)
+    for t in (0, 9, 10, 11, 57, 199):
+        nt = int(seq.n_visible[t])
+        blocks, idx, _ = seq.hisa(t)
+        c = (nt - 1) // 10
+        assert list(blocks) == [c]
+        assert sorted(idx.tolist()) == list(range(c * 10, nt))     # k >= |C_t|: all returned
+
+
+def pin_large_k_returns_all_candidates():
+    inp = synthetic.generate(synthetic.small_case(num_keys=256, heads=2, head_dim=4, block_size=16,
+                                                  top_m=3, top_k=48, needles=0))
+    seq = Sequence(inp, 0)
+    for t in (5, 40, 100, 255):
+        blocks, idx, _ = seq.hisa(t)
+        cand = ho.candidate_keys(blocks, int(seq.n_visible[t]), 16)
+        assert sorted(idx.tolist()) == cand.tolist()
+
+
+def pin_scale_invariance():
+    """Positive rescaling of q, k or w (by powers of two, so exactly) leaves the
+    selection unchanged and scales the scores."""
+    inp = synthetic.generate(synthetic.small_case(num_keys=256, heads=3, head_dim=6, block_size=16,
+                                                  top_m=4, top_k=20))
+    seq = Sequence(inp, 0)
+    for t in (30, 128, 255):
+        b0, i0, s0 = seq.hisa(t)
+        q, w, k, kp, nt = seq.q[t], seq.w[t], seq.keys, seq.kpool, int(seq.n_visible[t])
+        b1, i1, s1 = ho.hisa_query(q * 2, w * 0.5, k * 4, kp * 4, nt, 16, 4, 20)
+        assert list(b0) == list(b1) and list(i0) == list(i1)
+        np.testing.assert_array_equal(s1, s0 * 4)
+
+
+def pin_all_negative_gives_lowest_indices():
+    """When every head's dot product is negative all scores are 0 and ties
+    resolve to the lowest indices."""
+    q = np.ones((2, 3))
+    keys = -np.abs(np.random.default_rng(17).standard_normal((30, 3))) - 0.1
+    idx, sc = ho.flat_query(q, np.ones(2), keys, 30, 7)
+    assert list(idx) == list(range(7)) and np.all(sc == 0)
+
+
+def pin_quantize_rows():
+    rng = np.random.default_rng(18)
+    x = rng.standard_normal((50, 64)).astype(np.float32)
+    codes, scale = ho.quantize_e4m3_rows(x)
+    amax = np.abs(x).max(axis=1)
+    np.testing.assert_array_equal(scale, (amax / np.float32(448)).astype(np.float32))
+    # the largest element of each row lands on +-448 (code 0x7E or 0xFE)
+    arg = np.abs(x).argmax(axis=1)
+    assert np.all((codes[np.arange(50), arg] & 0x7F) == 0x7E)
+    # dequantised values are within half an E4M3 step (relative 2^-4) of the input
+    deq = ho.dequantize_e4m3_rows(codes, scale)
+    big = np.abs(x) >= scale[:, None] * 2 ** -6
+    assert np.all(np.abs(deq - x)[big] <= np.abs(x)[big] * 2 ** -4 + 1e-12)
+    # an all-zero row has scale 1 and zero codes
+    c0, s0 = ho.quantize_e4m3_rows(np.zeros((1, 8), np.float32))
+    assert s0[0] == 1.0 and np.all(c0 == 0)
+
+
+# ---------------------------------------------------------------- invariants on a workload
+
+
+def pin_tiny_workload_invariants():
+    inp = synthetic.generate("tiny")
+    wl = inp.workload
+    seq = Sequence(inp, 0)
+    rng = np.random.default_rng(19)
+    ts = sorted(set([0, 1, 63, 64, 65, 127, 128, 511, 1023] + rng.integers(0, 1024, 40).tolist()))
+    found_needles = 0
+    for t in ts:
+        nt = int(seq.n_visible[t])
+        blocks, hi, hs = seq.hisa(t)
+        fi, fs = seq.flat(t)
+        cand = ho.candidate_keys(blocks, nt, wl.block_size)
+        # structure: causal, unique, exactly min(k, |C_t|) / min(k, n_t)
+        assert len(set(hi.tolist())) == len(hi) == min(wl.top_k, len(cand))
+        assert len(set(fi.tolist())) == len(fi) == min(wl.top_k, nt)
+        assert np.all(hi < nt) and np.all(fi < nt)
+        # the token stage keeps every flat winner that is a candidate
+        assert set(hi.tolist()) & set(fi.tolist()) == set(cand.tolist()) & set(fi.tolist())
+        # recall against flat never drops as m grows (the candidate sets nest)
+        rec = [len(set(seq.hisa(t, top_m=m)[1].tolist()) & set(fi.tolist())) for m in (1, 2, 4, 8, 16)]
+        assert rec == sorted(rec), (t, rec)
+        # m = every block: identical to flat
+        assert list(seq.hisa(t, top_m=16)[1]) == list(fi)
+    for s, t in zip(inp.needle_pos[0], inp.needle_query[0]):
+        fi, _ = seq.flat(int(t))
+        found_needles += int(s in set(fi.tolist()))
+    assert found_needles >= len(inp.needle_pos[0]) - 1, found_needles
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

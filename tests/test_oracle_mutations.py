@@ -1,0 +1,99 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that the pins
+catch every one of them."""
+import numpy as np
+import pytest
+
+import oracle_pins
+from oracle import hisa_oracle as ho
+from oracle import ofp8
+
+
+def _no_relu(q_t, w_t, keys):
+    return (np.asarray(keys, np.float64) @ np.asarray(q_t, np.float64).T) @ np.asarray(w_t, np.float64)
+
+
+def _heads_swapped(q_t, w_t, keys):
+    q = np.asarray(q_t, np.float64)[::-1]
+    return np.maximum(np.asarray(keys, np.float64) @ q.T, 0) @ np.asarray(w_t, np.float64)
+
+
+def _ties_high(scores, count):
+    scores = np.asarray(scores, np.float64)
+    n = len(scores)
+    order = np.lexsort((-np.arange(n), -scores))
+    return order[:min(count, n)]
+
+
+def _current_block_late(n_t, block):
+    return n_t // block if n_t > 0 else -1
+
+
+def _blocks_unforced(q_t, w_t, kpool, n_t, block, top_m):
+    c = ho.current_block(n_t, block)
+    if c < 0:
+        return np.zeros(0, np.int64)
+    s = ho.indexer_scores(q_t, w_t, kpool[:c + 1])
+    return np.sort(ho.top_by_score(s, top_m)).astype(np.int64)
+
+
+def _block_sums(keys, block):
+    keys = np.asarray(keys, np.float64)
+    nb = -(-keys.shape[0] // block)
+    return np.stack([keys[b * block:(b + 1) * block].sum(axis=0) for b in range(nb)])
+
+
+def _mean_of_relu_blocks(q_t, w_t, kpool, n_t, block, top_m):
+    # scores blocks by pooling after the ReLU (needs the raw keys; emulate on kpool rows)
+    c = ho.current_block(n_t, block)
+    if c < 0:
+        return np.zeros(0, np.int64)
+    if c + 1 <= top_m:
+        return np.arange(c + 1, dtype=np.int64)
+    s = np.abs(np.asarray(kpool[:c], np.float64) @ np.asarray(q_t, np.float64).T) @ np.asarray(w_t)
+    kept = ho.top_by_score(s, top_m - 1)
+    return np.sort(np.concatenate([kept, [c]])).astype(np.int64)
+
+
+def _cand_leaky(blocks, n_t, block):
+    parts = [np.arange(b * block, min((b + 1) * block, n_t + 1)) for b in sorted(blocks)]
+    return np.concatenate(parts).astype(np.int64) if parts else np.zeros(0, np.int64)
+
+
+def _e4m3_half_away(x):
+    x = np.asarray(x, np.float64)
+    nudged = x + np.sign(x) * np.abs(x) * 1e-9
+    return _orig_e4m3(nudged)
+
+
+def _bf16_via_fp32(x):
+    return _orig_bf16(np.asarray(x, np.float64).astype(np.float32).astype(np.float64))
+
+
+_orig_e4m3 = ofp8.e4m3_encode
+_orig_bf16 = ofp8.bf16_round
+
+MUTATIONS = {
+    "relu_dropped": [(ho, "indexer_scores", _no_relu)],
+    "weights_on_wrong_heads": [(ho, "indexer_scores", _heads_swapped)],
+    "ties_to_higher_index": [(ho, "top_by_score", _ties_high)],
+    "current_block_off_by_one": [(ho, "current_block", _current_block_late)],
+    "current_block_not_forced": [(ho, "select_blocks", _blocks_unforced)],
+    "pool_sum_not_mean": [(ho, "block_means", _block_sums)],
+    "block_score_abs": [(ho, "select_blocks", _mean_of_relu_blocks)],
+    "causal_leak": [(ho, "candidate_keys", _cand_leaky)],
+    "e4m3_ties_away": [(ofp8, "e4m3_encode", _e4m3_half_away), (ho, "e4m3_encode", _e4m3_half_away)],
+    "bf16_double_rounding": [(ofp8, "bf16_round", _bf16_via_fp32), (ho, "bf16_round", _bf16_via_fp32)],
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name, monkeypatch):
+    for mod, attr, fn in MUTATIONS[name]:
+        monkeypatch.setattr(mod, attr, fn)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin()
+        except Exception:       # an assertion, or the mistake breaking a shape
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches the planted mistake {name!r}"
