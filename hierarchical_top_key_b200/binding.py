@@ -1,0 +1,271 @@
+"""Python binding of libhisa (include/hisa.h): argument marshalling only.
+
+Every function here checks tensor shapes/dtypes, allocates outputs and the
+workspace with torch (the library itself never allocates), and calls the C
+entry point of the same name on torch's current CUDA stream.  There is no
+fallback: if libhisa.so is missing or fails to load, ``load()`` raises.
+
+Layouts (row-major, contiguous, on the GPU):
+  q          [batch, Q, H, d]   float32 / bfloat16 / uint8 (E4M3 codes)
+  keys       [batch, L, d]      same dtype as q
+  w          [batch, Q, H]      float32
+  n_visible  [batch, Q]         int32
+  q_scale    [batch, Q]         float32 (E4M3 only);  k_scale [batch, L]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+HISA_F32, HISA_BF16, HISA_E4M3 = 0, 1, 2
+OP_BLOCK, OP_TOKEN, OP_FLAT = 1, 2, 3
+STATUS = {0: "HISA_OK", 1: "HISA_ERR_INVALID_ARG", 2: "HISA_ERR_UNSUPPORTED", 3: "HISA_ERR_WORKSPACE",
+          4: "HISA_ERR_CUDA", 5: "HISA_ERR_TIMEOUT"}
+
+
+class HisaError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("batch", "num_keys", "num_queries", "heads", "head_dim", "block_size", "top_m", "top_k",
+                 "dtype")]
+
+
+_P = ctypes.c_void_p
+_SIGS = {
+    "hisa_pool_blocks": [_P, _P, _P, _P, ctypes.POINTER(Shape), _P],
+    "hisa_compress_keys": [_P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                           ctypes.c_int32, _P],
+    "hisa_quantize_e4m3": [_P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _P, _P, _P],
+    "hisa_block_score_topm": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, ctypes.c_size_t, _P],
+    "hisa_token_score_topk": [_P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t,
+                              _P],
+    "dsa_flat_indexer_topk": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t, _P],
+    "hisa_workspace_size": [ctypes.c_int32, ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)],
+    "hisa_get_status": [_P],
+    "hisa_status_string": [ctypes.c_int],
+    "hisa_last_error": [],
+}
+EXPORTS = tuple(_SIGS)
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libhisa.so (building it first if the sources are newer)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    if path is None:
+        path = library_path()
+        if not _build.up_to_date():
+            _build.build()
+    if not os.path.exists(path):
+        raise RuntimeError(f"libhisa.so not found at {path}; run `python -m hierarchical_top_key_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, args in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_char_p if name in ("hisa_status_string", "hisa_last_error") else ctypes.c_int
+    if path == library_path():
+        _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        msg = load().hisa_last_error().decode(errors="replace")
+        raise HisaError(status, where, msg)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return HISA_F32
+    if t.dtype == torch.bfloat16:
+        return HISA_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return HISA_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need(t: torch.Tensor, name: str, ndim: int):
+    if not t.is_cuda or not t.is_contiguous() or t.dim() != ndim:
+        raise ValueError(f"{name} must be a contiguous CUDA tensor with {ndim} dims, got {tuple(t.shape)}")
+
+
+def make_shape(q: torch.Tensor, k: torch.Tensor, block_size: int = 1, top_m: int = 1, top_k: int = 1) -> Shape:
+    _need(q, "q", 4)
+    _need(k, "keys", 3)
+    b, Q, H, d = q.shape
+    if k.shape[0] != b or k.shape[2] != d:
+        raise ValueError(f"keys {tuple(k.shape)} do not match q {tuple(q.shape)}")
+    if dtype_code(q) != dtype_code(k):
+        raise TypeError("q and keys must share a dtype")
+    return Shape(b, k.shape[1], Q, H, d, block_size, top_m, top_k, dtype_code(q))
+
+
+def workspace_size(op: int, shape: Shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().hisa_workspace_size(op, ctypes.byref(shape), ctypes.byref(n)), "hisa_workspace_size")
+    return n.value
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def get_status():
+    """Synchronise the current stream and raise if a kernel recorded an error."""
+    _check(load().hisa_get_status(_stream()), "hisa_get_status")
+
+
+# ----------------------------------------------------------------- entry points
+
+
+def hisa_pool_blocks(k: torch.Tensor, block_size: int, k_scale: Optional[torch.Tensor] = None):
+    """Mean-pool each run of block_size keys -> (kpool [batch, nb, d], kpool_scale or None)."""
+    _need(k, "keys", 3)
+    b, L, d = k.shape
+    nb = -(-L // block_size)
+    shape = Shape(b, L, 1, 1, d, block_size, 1, 1, dtype_code(k))
+    kpool = torch.empty((b, nb, d), dtype=k.dtype, device=k.device)
+    kps = torch.empty((b, nb), dtype=torch.float32, device=k.device) if k_scale is not None else None
+    _check(load().hisa_pool_blocks(k.data_ptr(), _ptr(k_scale), kpool.data_ptr(), _ptr(kps), ctypes.byref(shape),
+                                   _stream()), "hisa_pool_blocks")
+    return kpool, kps
+
+
+def hisa_compress_keys(k_raw: torch.Tensor, ratio: int) -> torch.Tensor:
+    """Mean of each `ratio` consecutive keys (trailing partial group dropped)."""
+    _need(k_raw, "k_raw", 3)
+    b, S, d = k_raw.shape
+    ck = torch.empty((b, S // ratio, d), dtype=k_raw.dtype, device=k_raw.device)
+    _check(load().hisa_compress_keys(k_raw.data_ptr(), ck.data_ptr(), b, S, d, ratio, dtype_code(k_raw),
+                                     _stream()), "hisa_compress_keys")
+    return ck
+
+
+def hisa_quantize_e4m3(x: torch.Tensor, row_dims: int):
+    """E4M3 codes and per-row fp32 scales; rows are the first `row_dims` dims."""
+    if not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA tensor")
+    rows = 1
+    for s in x.shape[:row_dims]:
+        rows *= s
+    cols = x.numel() // max(rows, 1)
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scale = torch.empty(x.shape[:row_dims], dtype=torch.float32, device=x.device)
+    _check(load().hisa_quantize_e4m3(x.data_ptr(), dtype_code(x), rows, cols, codes.data_ptr(), scale.data_ptr(),
+                                     _stream()), "hisa_quantize_e4m3")
+    return codes, scale
+
+
+def hisa_block_score_topm(q, w, kpool, n_visible, *, num_keys: int, block_size: int, top_m: int,
+                          q_scale=None, kpool_scale=None, workspace: Optional[torch.Tensor] = None):
+    """Coarse stage: block_idx [batch, Q, top_m] int32 (-1 padded, any order)."""
+    b, Q, H, d = q.shape
+    shape = Shape(b, num_keys, Q, H, d, block_size, top_m, 1, dtype_code(q))
+    _need(w, "w", 3)
+    _need(n_visible, "n_visible", 2)
+    out = torch.empty((b, Q, top_m), dtype=torch.int32, device=q.device)
+    ws = workspace if workspace is not None else _workspace(workspace_size(OP_BLOCK, shape), q.device)
+    _check(load().hisa_block_score_topm(q.data_ptr(), _ptr(q_scale), w.data_ptr(), kpool.data_ptr(),
+                                        _ptr(kpool_scale), n_visible.data_ptr(), ctypes.byref(shape),
+                                        out.data_ptr(), ws.data_ptr(), ws.numel(), _stream()),
+           "hisa_block_score_topm")
+    return out
+
+
+def hisa_token_score_topk(q, w, k, n_visible, block_idx, *, block_size: int, top_k: int, q_scale=None,
+                          k_scale=None, want_scores: bool = False):
+    """Refinement stage: (topk_idx [batch, Q, top_k] int32, scores or None)."""
+    top_m = block_idx.shape[-1]
+    shape = make_shape(q, k, block_size, top_m, top_k)
+    _need(block_idx, "block_idx", 3)
+    b, Q = q.shape[:2]
+    idx = torch.empty((b, Q, top_k), dtype=torch.int32, device=q.device)
+    sc = torch.empty((b, Q, top_k), dtype=torch.float32, device=q.device) if want_scores else None
+    _check(load().hisa_token_score_topk(q.data_ptr(), _ptr(q_scale), w.data_ptr(), k.data_ptr(), _ptr(k_scale),
+                                        n_visible.data_ptr(), block_idx.data_ptr(), ctypes.byref(shape),
+                                        idx.data_ptr(), _ptr(sc), None, 0, _stream()), "hisa_token_score_topk")
+    return idx, sc
+
+
+def dsa_flat_indexer_topk(q, w, k, n_visible, *, top_k: int, q_scale=None, k_scale=None,
+                          want_scores: bool = False, workspace: Optional[torch.Tensor] = None):
+    """Flat DSA indexer: (topk_idx [batch, Q, top_k] int32, scores or None)."""
+    shape = make_shape(q, k, 1, 1, top_k)
+    b, Q = q.shape[:2]
+    idx = torch.empty((b, Q, top_k), dtype=torch.int32, device=q.device)
+    sc = torch.empty((b, Q, top_k), dtype=torch.float32, device=q.device) if want_scores else None
+    ws = workspace if workspace is not None else _workspace(workspace_size(OP_FLAT, shape), q.device)
+    _check(load().dsa_flat_indexer_topk(q.data_ptr(), _ptr(q_scale), w.data_ptr(), k.data_ptr(), _ptr(k_scale),
+                                        n_visible.data_ptr(), ctypes.byref(shape), idx.data_ptr(), _ptr(sc),
+                                        ws.data_ptr(), ws.numel(), _stream()), "dsa_flat_indexer_topk")
+    return idx, sc
+
+
+class HisaIndexer:
+    """The whole HISA indexer for one layer: pool -> coarse top-m -> refine top-k.
+
+    Workspaces are allocated once per shape and reused."""
+
+    def __init__(self, block_size: int, top_m: int, top_k: int):
+        self.block_size, self.top_m, self.top_k = block_size, top_m, top_k
+        self._ws = None
+
+    def __call__(self, q, w, k, n_visible, q_scale=None, k_scale=None, want_scores=False, return_blocks=False):
+        kpool, kps = hisa_pool_blocks(k, self.block_size, k_scale)
+        shape = make_shape(q, k, self.block_size, self.top_m, self.top_k)
+        need = workspace_size(OP_BLOCK, shape)
+        if self._ws is None or self._ws.numel() < need or self._ws.device != q.device:
+            self._ws = _workspace(need, q.device)
+        blocks = hisa_block_score_topm(q, w, kpool, n_visible, num_keys=k.shape[1], block_size=self.block_size,
+                                       top_m=self.top_m, q_scale=q_scale, kpool_scale=kps, workspace=self._ws)
+        idx, sc = hisa_token_score_topk(q, w, k, n_visible, blocks, block_size=self.block_size, top_k=self.top_k,
+                                        q_scale=q_scale, k_scale=k_scale, want_scores=want_scores)
+        return (idx, sc, blocks) if return_blocks else (idx, sc)
+
+
+def to_device_inputs(inputs, device="cuda", fp8: bool = False, compress: bool = True):
+    """Upload one synthetic draw (``synthetic.Inputs``) in its storage dtype.
+
+    Returns a dict with q, w, k (compressed by the workload's ratio through the
+    library when `compress`), n_visible, and for fp8 the E4M3 codes/scales
+    produced by the library's quantiser."""
+    wl = inputs.workload
+    tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+    q = torch.from_numpy(inputs.q).to(device=device).to(tdt).contiguous()
+    k = torch.from_numpy(inputs.keys).to(device=device).to(tdt).contiguous()
+    w = torch.from_numpy(inputs.w).to(device=device).contiguous()
+    nv = torch.from_numpy(inputs.n_visible).to(device=device).contiguous()
+    if compress and wl.compress_ratio > 1:
+        k = hisa_compress_keys(k, wl.compress_ratio)
+    out = dict(q=q, w=w, k=k, n_visible=nv, q_scale=None, k_scale=None)
+    if fp8:
+        b, Q, H, d = q.shape
+        qc, qs = hisa_quantize_e4m3(q, 2)
+        kc, ks = hisa_quantize_e4m3(k, 2)
+        out.update(q=qc, k=kc, q_scale=qs, k_scale=ks)
+    return out

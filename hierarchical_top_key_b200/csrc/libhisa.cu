@@ -1,0 +1,339 @@
+// libhisa.cu - the C ABI of include/hisa.h: argument validation, workspace
+// planning and stream-ordered kernel launches.  Every step of the indexers
+// runs in the kernels included below; this file only checks arguments and
+// launches them.
+#include <cstdio>
+#include <cstring>
+#include <cstdarg>
+#include <algorithm>
+
+#include "common.cuh"
+#include "pool.cuh"
+#include "select.cuh"
+#include "score_simt.cuh"
+
+using namespace hisa;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+hisa_status fail(hisa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+hisa_status cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return HISA_OK;
+  return fail(HISA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+hisa_status launch_check(const char* what) { return cuda_check(cudaGetLastError(), what); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int elem_bytes(int dt) { return dt == HISA_F32 ? 4 : dt == HISA_BF16 ? 2 : 1; }
+
+constexpr int kMaxCandidates = 16384;   // top_m * block_size held on chip per query
+constexpr int kMaxTopM = 256;
+
+hisa_status check_shape(const hisa_shape* s, bool need_blocks) {
+  if (!s) return fail(HISA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->batch < 1 || s->num_keys < 1 || s->num_queries < 1)
+    return fail(HISA_ERR_INVALID_ARG, "batch, num_keys, num_queries must be >= 1");
+  if (s->heads < 1 || s->heads > 64) return fail(HISA_ERR_UNSUPPORTED, "heads must be in [1, 64]");
+  if (s->head_dim != 64 && s->head_dim != 128) return fail(HISA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (s->dtype != HISA_F32 && s->dtype != HISA_BF16 && s->dtype != HISA_E4M3)
+    return fail(HISA_ERR_INVALID_ARG, "unknown dtype %d", s->dtype);
+  if (s->top_k < 1) return fail(HISA_ERR_INVALID_ARG, "top_k must be >= 1");
+  if (need_blocks) {
+    if (s->block_size < 1) return fail(HISA_ERR_INVALID_ARG, "block_size must be >= 1");
+    if (s->top_m < 1) return fail(HISA_ERR_INVALID_ARG, "top_m must be >= 1");
+  }
+  return HISA_OK;
+}
+
+int64_t rows_of(const hisa_shape* s) { return static_cast<int64_t>(s->batch) * s->num_queries; }
+int64_t pad4(int64_t n) { return (n + 3) / 4 * 4; }
+int64_t num_blocks(const hisa_shape* s) { return ceil_div(s->num_keys, s->block_size); }
+
+// ------------------------------------------------------------ dispatch helpers
+
+template <int DT, int HT>
+hisa_status launch_score_rows(const hisa_shape* s, const void* q, const float* qsc, const float* w,
+                              const void* keys, const float* ksc, const int32_t* nvis, int block_div,
+                              int L, int64_t row0, int64_t nrows, float* out, int64_t ld, cudaStream_t st) {
+  const int kpc = 2048;
+  const size_t smem = SimtTile<DT, HT>::smem_bytes(s->head_dim);
+  auto kern = score_rows_simt_kernel<DT, HT>;
+  hisa_status e = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(smem)), "score_rows attribute");
+  if (e != HISA_OK) return e;
+  dim3 grid(static_cast<unsigned>(nrows), static_cast<unsigned>(ceil_div(L, kpc)));
+  kern<<<grid, kSimtThreads, smem, st>>>(static_cast<const uint8_t*>(q), qsc, w,
+                                         static_cast<const uint8_t*>(keys), ksc, nvis, block_div,
+                                         s->num_queries, s->heads, s->head_dim, L, row0, out, ld, kpc);
+  return launch_check("score_rows_simt_kernel");
+}
+
+template <int DT>
+hisa_status score_rows_h(const hisa_shape* s, const void* q, const float* qsc, const float* w,
+                         const void* keys, const float* ksc, const int32_t* nvis, int block_div, int L,
+                         int64_t row0, int64_t nrows, float* out, int64_t ld, cudaStream_t st) {
+  if (s->heads <= 4)
+    return launch_score_rows<DT, 4>(s, q, qsc, w, keys, ksc, nvis, block_div, L, row0, nrows, out, ld, st);
+  if (s->heads <= 16)
+    return launch_score_rows<DT, 16>(s, q, qsc, w, keys, ksc, nvis, block_div, L, row0, nrows, out, ld, st);
+  return launch_score_rows<DT, 64>(s, q, qsc, w, keys, ksc, nvis, block_div, L, row0, nrows, out, ld, st);
+}
+
+hisa_status score_rows(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* keys,
+                       const float* ksc, const int32_t* nvis, int block_div, int L, int64_t row0,
+                       int64_t nrows, float* out, int64_t ld, cudaStream_t st) {
+  switch (s->dtype) {
+    case HISA_F32: return score_rows_h<DT_F32>(s, q, qsc, w, keys, ksc, nvis, block_div, L, row0, nrows, out, ld, st);
+    case HISA_BF16: return score_rows_h<DT_BF16>(s, q, qsc, w, keys, ksc, nvis, block_div, L, row0, nrows, out, ld, st);
+    default: return score_rows_h<DT_E4M3>(s, q, qsc, w, keys, ksc, nvis, block_div, L, row0, nrows, out, ld, st);
+  }
+}
+
+template <int DT, int HT>
+hisa_status launch_token_simt(const hisa_shape* s, const void* q, const float* qsc, const float* w,
+                              const void* k, const float* ksc, const int32_t* nvis, const int32_t* bidx,
+                              int32_t* oi, float* os, cudaStream_t st) {
+  const size_t smem = SimtTile<DT, HT>::smem_bytes(s->head_dim) +
+                      static_cast<size_t>(s->top_m) * s->block_size * sizeof(uint32_t);
+  auto kern = token_stage_simt_kernel<DT, HT>;
+  hisa_status e = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(smem)), "token_stage attribute");
+  if (e != HISA_OK) return e;
+  kern<<<static_cast<unsigned>(rows_of(s)), kSimtThreads, smem, st>>>(
+      static_cast<const uint8_t*>(q), qsc, w, static_cast<const uint8_t*>(k), ksc, nvis, bidx,
+      s->num_queries, s->heads, s->head_dim, s->num_keys, s->block_size, s->top_m, s->top_k, oi, os);
+  return launch_check("token_stage_simt_kernel");
+}
+
+template <int DT>
+hisa_status token_simt_h(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* k,
+                         const float* ksc, const int32_t* nvis, const int32_t* bidx, int32_t* oi, float* os,
+                         cudaStream_t st) {
+  if (s->heads <= 4) return launch_token_simt<DT, 4>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st);
+  if (s->heads <= 16) return launch_token_simt<DT, 16>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st);
+  return launch_token_simt<DT, 64>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st);
+}
+
+hisa_status check_indexer_ptrs(const hisa_shape* s, const void* q, const float* q_scale, const float* w,
+                               const void* k, const float* k_scale, const int32_t* n_visible) {
+  if (!q || !w || !k || !n_visible) return fail(HISA_ERR_INVALID_ARG, "q, w, keys and n_visible must be non-NULL");
+  if (!aligned16(q) || !aligned16(k)) return fail(HISA_ERR_INVALID_ARG, "q and keys must be 16-byte aligned");
+  if (!aligned4(w) || !aligned4(n_visible)) return fail(HISA_ERR_INVALID_ARG, "w and n_visible must be 4-byte aligned");
+  if (s->dtype == HISA_E4M3 && (!q_scale || !k_scale))
+    return fail(HISA_ERR_INVALID_ARG, "E4M3 inputs need q_scale and k_scale");
+  return HISA_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+
+extern "C" {
+
+const char* hisa_status_string(hisa_status st) {
+  switch (st) {
+    case HISA_OK: return "HISA_OK";
+    case HISA_ERR_INVALID_ARG: return "HISA_ERR_INVALID_ARG: invalid argument";
+    case HISA_ERR_UNSUPPORTED: return "HISA_ERR_UNSUPPORTED: shape not supported by this build";
+    case HISA_ERR_WORKSPACE: return "HISA_ERR_WORKSPACE: workspace too small";
+    case HISA_ERR_CUDA: return "HISA_ERR_CUDA: CUDA runtime error";
+    case HISA_ERR_TIMEOUT: return "HISA_ERR_TIMEOUT: a device-side bounded wait gave up";
+  }
+  return "unknown hisa_status";
+}
+
+const char* hisa_last_error(void) { return g_last_error; }
+
+hisa_status hisa_get_status(hisa_stream stream) {
+  hisa_status e = cuda_check(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)), "stream sync");
+  if (e != HISA_OK) return e;
+  int v = 0, zero = 0;
+  e = cuda_check(cudaMemcpyFromSymbol(&v, g_status, sizeof(int)), "read status word");
+  if (e != HISA_OK) return e;
+  if (v != 0) {
+    e = cuda_check(cudaMemcpyToSymbol(g_status, &zero, sizeof(int)), "clear status word");
+    if (e != HISA_OK) return e;
+    return fail(static_cast<hisa_status>(v), "device status word reported %d", v);
+  }
+  return HISA_OK;
+}
+
+hisa_status hisa_workspace_size(int32_t op, const hisa_shape* s, size_t* bytes) {
+  if (!bytes) return fail(HISA_ERR_INVALID_ARG, "bytes is NULL");
+  hisa_status e = check_shape(s, op != HISA_OP_FLAT_TOPK);
+  if (e != HISA_OK) return e;
+  switch (op) {
+    case HISA_OP_FLAT_TOPK: *bytes = static_cast<size_t>(rows_of(s) * pad4(s->num_keys) * 4); return HISA_OK;
+    case HISA_OP_BLOCK_SCORE_TOPM: *bytes = static_cast<size_t>(rows_of(s) * pad4(num_blocks(s)) * 4); return HISA_OK;
+    case HISA_OP_TOKEN_SCORE_TOPK: *bytes = 0; return HISA_OK;
+  }
+  return fail(HISA_ERR_INVALID_ARG, "unknown op %d", op);
+}
+
+hisa_status hisa_pool_blocks(const void* k, const float* k_scale, void* kpool, float* kpool_scale,
+                             const hisa_shape* s, hisa_stream stream) {
+  if (!s) return fail(HISA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->batch < 1 || s->num_keys < 1 || s->block_size < 1)
+    return fail(HISA_ERR_INVALID_ARG, "batch, num_keys, block_size must be >= 1");
+  if (s->head_dim != 64 && s->head_dim != 128) return fail(HISA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (!k || !kpool || !aligned16(k) || !aligned16(kpool))
+    return fail(HISA_ERR_INVALID_ARG, "k and kpool must be non-NULL and 16-byte aligned");
+  if (s->dtype == HISA_E4M3 && (!k_scale || !kpool_scale))
+    return fail(HISA_ERR_INVALID_ARG, "E4M3 pooling needs k_scale and kpool_scale");
+  const int nb = static_cast<int>(num_blocks(s));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t threads_total = static_cast<int64_t>(s->batch) * nb * (s->head_dim * elem_bytes(s->dtype) / 16);
+  const int grid = static_cast<int>(std::min<int64_t>(ceil_div(threads_total, 256), 148 * 64));
+  const uint8_t* in = static_cast<const uint8_t*>(k);
+  uint8_t* out = static_cast<uint8_t*>(kpool);
+  switch (s->dtype) {
+    case HISA_F32:
+      segment_mean_kernel<DT_F32><<<grid, 256, 0, st>>>(in, nullptr, out, nullptr, s->batch, s->num_keys, nb,
+                                                        s->head_dim, s->block_size);
+      break;
+    case HISA_BF16:
+      segment_mean_kernel<DT_BF16><<<grid, 256, 0, st>>>(in, nullptr, out, nullptr, s->batch, s->num_keys, nb,
+                                                         s->head_dim, s->block_size);
+      break;
+    case HISA_E4M3:
+      segment_mean_kernel<DT_E4M3><<<grid, 256, 0, st>>>(in, k_scale, out, kpool_scale, s->batch, s->num_keys,
+                                                         nb, s->head_dim, s->block_size);
+      break;
+    default: return fail(HISA_ERR_INVALID_ARG, "unknown dtype %d", s->dtype);
+  }
+  return launch_check("segment_mean_kernel");
+}
+
+hisa_status hisa_compress_keys(const void* k_raw, void* ck, int32_t batch, int32_t num_raw_keys,
+                               int32_t head_dim, int32_t ratio, int32_t dtype, hisa_stream stream) {
+  if (batch < 1 || num_raw_keys < 1 || ratio < 1) return fail(HISA_ERR_INVALID_ARG, "batch, num_raw_keys, ratio must be >= 1");
+  if (head_dim != 64 && head_dim != 128) return fail(HISA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (dtype != HISA_F32 && dtype != HISA_BF16) return fail(HISA_ERR_UNSUPPORTED, "compression takes fp32 or bf16 keys");
+  if (!k_raw || !ck || !aligned16(k_raw) || !aligned16(ck))
+    return fail(HISA_ERR_INVALID_ARG, "k_raw and ck must be non-NULL and 16-byte aligned");
+  const int n_out = num_raw_keys / ratio;
+  if (n_out == 0) return HISA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t threads_total = static_cast<int64_t>(batch) * n_out * (head_dim * elem_bytes(dtype) / 16);
+  const int grid = static_cast<int>(std::min<int64_t>(ceil_div(threads_total, 256), 148 * 64));
+  // the input is viewed as n_out * ratio rows per sequence: the dropped tail
+  // rows are skipped by giving each sequence its true row count
+  const uint8_t* in = static_cast<const uint8_t*>(k_raw);
+  uint8_t* out = static_cast<uint8_t*>(ck);
+  if (dtype == HISA_F32)
+    segment_mean_kernel<DT_F32><<<grid, 256, 0, st>>>(in, nullptr, out, nullptr, batch, num_raw_keys, n_out,
+                                                      head_dim, ratio);
+  else
+    segment_mean_kernel<DT_BF16><<<grid, 256, 0, st>>>(in, nullptr, out, nullptr, batch, num_raw_keys, n_out,
+                                                       head_dim, ratio);
+  return launch_check("segment_mean_kernel (compress)");
+}
+
+hisa_status hisa_quantize_e4m3(const void* x, int32_t x_dtype, int64_t rows, int32_t cols, uint8_t* codes,
+                               float* scale, hisa_stream stream) {
+  if (rows < 0 || cols < 1) return fail(HISA_ERR_INVALID_ARG, "rows must be >= 0 and cols >= 1");
+  if (cols % 16 != 0) return fail(HISA_ERR_UNSUPPORTED, "cols must be a multiple of 16");
+  if (!x || !codes || !scale || !aligned16(x) || !aligned16(codes) || !aligned4(scale))
+    return fail(HISA_ERR_INVALID_ARG, "x/codes must be 16-byte aligned, scale 4-byte aligned, all non-NULL");
+  if (rows == 0) return HISA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int grid = static_cast<int>(std::min<int64_t>(ceil_div(rows, 8), 148 * 32));
+  const uint8_t* in = static_cast<const uint8_t*>(x);
+  if (x_dtype == HISA_F32) quantize_rows_kernel<DT_F32><<<grid, 256, 0, st>>>(in, rows, cols, codes, scale);
+  else if (x_dtype == HISA_BF16) quantize_rows_kernel<DT_BF16><<<grid, 256, 0, st>>>(in, rows, cols, codes, scale);
+  else return fail(HISA_ERR_UNSUPPORTED, "quantisation input must be fp32 or bf16");
+  return launch_check("quantize_rows_kernel");
+}
+
+hisa_status hisa_block_score_topm(const void* q, const float* q_scale, const float* w, const void* kpool,
+                                  const float* kpool_scale, const int32_t* n_visible, const hisa_shape* s,
+                                  int32_t* block_idx, void* workspace, size_t ws_bytes, hisa_stream stream) {
+  hisa_status e = check_shape(s, true);
+  if (e != HISA_OK) return e;
+  e = check_indexer_ptrs(s, q, q_scale, w, kpool, kpool_scale, n_visible);
+  if (e != HISA_OK) return e;
+  if (!block_idx || !aligned4(block_idx)) return fail(HISA_ERR_INVALID_ARG, "block_idx must be non-NULL, 4-byte aligned");
+  const int64_t nb = num_blocks(s);
+  const int64_t ld = pad4(nb);
+  const int64_t rows = rows_of(s);
+  if (!workspace || !aligned16(workspace)) return fail(HISA_ERR_WORKSPACE, "workspace must be non-NULL, 16-byte aligned");
+  const int64_t chunk = std::min<int64_t>(rows, static_cast<int64_t>(ws_bytes / (ld * 4)));
+  if (chunk < 1) return fail(HISA_ERR_WORKSPACE, "workspace holds no row of %lld block scores", (long long)nb);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
+    const int64_t nr = std::min(chunk, rows - r0);
+    e = score_rows(s, q, q_scale, w, kpool, kpool_scale, n_visible, s->block_size, static_cast<int>(nb), r0, nr,
+                   ws, ld, st);
+    if (e != HISA_OK) return e;
+    block_select_kernel<<<static_cast<unsigned>(nr), 512, 0, st>>>(ws, ld, n_visible, r0, s->num_keys, s->block_size, s->top_m,
+                                                                  block_idx);
+    e = launch_check("block_select_kernel");
+    if (e != HISA_OK) return e;
+  }
+  return HISA_OK;
+}
+
+hisa_status hisa_token_score_topk(const void* q, const float* q_scale, const float* w, const void* k,
+                                  const float* k_scale, const int32_t* n_visible, const int32_t* block_idx,
+                                  const hisa_shape* s, int32_t* topk_idx, float* topk_score, void* workspace,
+                                  size_t ws_bytes, hisa_stream stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  hisa_status e = check_shape(s, true);
+  if (e != HISA_OK) return e;
+  e = check_indexer_ptrs(s, q, q_scale, w, k, k_scale, n_visible);
+  if (e != HISA_OK) return e;
+  if (!block_idx || !topk_idx) return fail(HISA_ERR_INVALID_ARG, "block_idx and topk_idx must be non-NULL");
+  if (s->top_m > kMaxTopM) return fail(HISA_ERR_UNSUPPORTED, "top_m must be <= %d", kMaxTopM);
+  if (static_cast<int64_t>(s->top_m) * s->block_size > kMaxCandidates)
+    return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size must be <= %d", kMaxCandidates);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  switch (s->dtype) {
+    case HISA_F32: return token_simt_h<DT_F32>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
+    case HISA_BF16: return token_simt_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
+    default: return token_simt_h<DT_E4M3>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
+  }
+}
+
+hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale, const float* w, const void* k,
+                                  const float* k_scale, const int32_t* n_visible, const hisa_shape* s,
+                                  int32_t* topk_idx, float* topk_score, void* workspace, size_t ws_bytes,
+                                  hisa_stream stream) {
+  hisa_status e = check_shape(s, false);
+  if (e != HISA_OK) return e;
+  e = check_indexer_ptrs(s, q, q_scale, w, k, k_scale, n_visible);
+  if (e != HISA_OK) return e;
+  if (!topk_idx || !aligned4(topk_idx)) return fail(HISA_ERR_INVALID_ARG, "topk_idx must be non-NULL, 4-byte aligned");
+  const int64_t ld = pad4(s->num_keys);
+  const int64_t rows = rows_of(s);
+  if (!workspace || !aligned16(workspace)) return fail(HISA_ERR_WORKSPACE, "workspace must be non-NULL, 16-byte aligned");
+  const int64_t chunk = std::min<int64_t>(rows, static_cast<int64_t>(ws_bytes / (ld * 4)));
+  if (chunk < 1) return fail(HISA_ERR_WORKSPACE, "workspace holds no row of %d scores", s->num_keys);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
+    const int64_t nr = std::min(chunk, rows - r0);
+    e = score_rows(s, q, q_scale, w, k, k_scale, n_visible, 0, s->num_keys, r0, nr, ws, ld, st);
+    if (e != HISA_OK) return e;
+    flat_select_kernel<<<static_cast<unsigned>(nr), 512, 0, st>>>(ws, ld, n_visible, r0, s->num_keys, s->top_k, topk_idx,
+                                                                 topk_score);
+    e = launch_check("flat_select_kernel");
+    if (e != HISA_OK) return e;
+  }
+  return HISA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,212 @@
+/*
+ * hisa.h - C ABI of libhisa: the HISA hierarchical lightning indexer and the
+ * flat DSA lightning indexer on NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  "HISA: Efficient Hierarchical Indexing for Fine-Grained
+ * Sparse Attention" (arXiv 2603.28458, abstract): the DSA indexer scores every
+ * key of a query's prefix and keeps the top-k keys; HISA replaces that flat
+ * scan with (1) a coarse stage that scores pooled block representations and
+ * keeps the best blocks, and (2) a refinement stage that runs the original
+ * indexer only on the keys of the kept blocks, returning the same per-query
+ * set of k token indices that the downstream sparse attention consumes.  The
+ * indexer score used by every entry point is
+ *
+ *     I[t,s] = sum_h w[t,h] * ReLU(q[t,h,:] . k[s,:])
+ *
+ * and a block is represented by the mean of its keys.  A query t sees keys
+ * 0 .. n_visible[t]-1; its current block is c_t = (n_visible[t]-1) / B.  The
+ * coarse stage scores only the blocks b < c_t and always keeps c_t.  Ties at
+ * the k-th (or m-th) place go to the lower index.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers, 16-byte aligned, dense and
+ *    row-major in the layouts given below; the caller owns every buffer,
+ *    including the workspace.  The library allocates no memory.
+ *  - Work is enqueued on `stream` and runs asynchronously; the return value
+ *    reports only host-side validation and launch errors.  On a validation
+ *    error nothing is enqueued and the outputs are untouched.
+ *  - Kernels that wait on on-chip barriers do so with a bounded spin; if a
+ *    wait gives up, the kernel records HISA_ERR_TIMEOUT in a device status
+ *    word and exits cleanly.  hisa_get_status() reads (and clears) that word.
+ *  - Index outputs are -1 padded.  Index sets are returned in an unspecified
+ *    order; when a score output is given, score[i] belongs to index[i].
+ *  - dtype HISA_E4M3: q and keys are OFP8 E4M3 codes with one fp32 scale per
+ *    query token (over all H*d values) and one per key; the value of a code
+ *    is code * scale.  For the other dtypes the scale pointers are ignored
+ *    and may be NULL.
+ */
+#ifndef HISA_H_
+#define HISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HISA_API __attribute__((visibility("default")))
+#else
+#define HISA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HISA_OK = 0,
+  HISA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size or value   */
+  HISA_ERR_UNSUPPORTED = 2,   /* a valid shape this build has no kernel for     */
+  HISA_ERR_WORKSPACE = 3,     /* workspace smaller than one unit of work        */
+  HISA_ERR_CUDA = 4,          /* a CUDA runtime call failed                     */
+  HISA_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up             */
+} hisa_status;
+
+typedef enum { HISA_F32 = 0, HISA_BF16 = 1, HISA_E4M3 = 2 } hisa_dtype;
+
+/* Problem shape.  batch independent sequences, each with num_keys keys (L)
+ * and num_queries queries (Q); heads H and head_dim d of the indexer; block
+ * size B; top_m blocks and top_k tokens kept per query; dtype of q and keys
+ * (a hisa_dtype value).  w is always fp32. */
+typedef struct {
+  int32_t batch;
+  int32_t num_keys;
+  int32_t num_queries;
+  int32_t heads;
+  int32_t head_dim;
+  int32_t block_size;
+  int32_t top_m;
+  int32_t top_k;
+  int32_t dtype;
+} hisa_shape;
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* hisa_stream;
+
+/* op codes for hisa_workspace_size */
+enum {
+  HISA_OP_BLOCK_SCORE_TOPM = 1,
+  HISA_OP_TOKEN_SCORE_TOPK = 2,
+  HISA_OP_FLAT_TOPK = 3
+};
+
+/*
+ * Block pooling (HISA coarse stage input; HISA abstract, "pooled block
+ * representations").  kpool[b] = mean of keys b*B .. min((b+1)*B, L)-1, the
+ * mean taken exactly (fp64 accumulation) and rounded once to the key dtype.
+ * For HISA_E4M3 the mean is of the dequantised keys, rounded to fp32, then
+ * re-quantised with one scale per block: scale = max|mean| / 448 (1 for an
+ * all-zero block), code = E4M3(mean / scale), round to nearest even,
+ * saturating.
+ *   k            [batch, L, d] in shape->dtype
+ *   k_scale      [batch, L] fp32 (E4M3 only)
+ *   kpool        [batch, ceil(L/B), d] in shape->dtype          (output)
+ *   kpool_scale  [batch, ceil(L/B)] fp32 (E4M3 only)             (output)
+ * Uses batch, num_keys, head_dim, block_size, dtype.
+ */
+HISA_API hisa_status hisa_pool_blocks(const void* k, const float* k_scale, void* kpool,
+                             float* kpool_scale, const hisa_shape* shape,
+                             hisa_stream stream);
+
+/*
+ * Key compression ("StreamIndex: Memory-Bounded Compressed Sparse Attention
+ * via Streaming Top-k", arXiv 2605.02568, abstract: the indexer runs over keys
+ * compressed by a fixed ratio, 4 in V4-Flash).  ck[j] = mean of raw keys
+ * j*ratio .. j*ratio+ratio-1, exact mean rounded once to the dtype; a trailing
+ * incomplete group is dropped.  dtype HISA_F32 or HISA_BF16.
+ *   k_raw [batch, S, d] -> ck [batch, S / ratio, d]
+ */
+HISA_API hisa_status hisa_compress_keys(const void* k_raw, void* ck, int32_t batch,
+                               int32_t num_raw_keys, int32_t head_dim,
+                               int32_t ratio, int32_t dtype, hisa_stream stream);
+
+/*
+ * Per-row FP8 quantisation of q or keys (the E4M3 variant of the indexer):
+ * scale[r] = max_j |x[r,j]| / 448 in fp32 (1 when the row is all zero),
+ * codes[r,j] = E4M3(x[r,j] / scale[r]) with the division in fp32, round to
+ * nearest even, saturating to +-448.
+ *   x      [rows, cols] fp32 (x_dtype HISA_F32) or bf16 (HISA_BF16)
+ *   codes  [rows, cols] uint8 (output), scale [rows] fp32 (output)
+ * For q use rows = batch*Q, cols = H*d; for keys rows = batch*L, cols = d.
+ */
+HISA_API hisa_status hisa_quantize_e4m3(const void* x, int32_t x_dtype, int64_t rows,
+                               int32_t cols, uint8_t* codes, float* scale,
+                               hisa_stream stream);
+
+/*
+ * HISA coarse stage (HISA abstract, stage 1): for each query t,
+ *   S_b[t,b] = sum_h w[t,h] * ReLU(q[t,h,:] . kpool[b,:])   for b < c_t,
+ * then block_idx[t,:] = {c_t} plus the top_m-1 blocks by S_b (ties -> lower
+ * b); every block 0..c_t when c_t+1 <= top_m; nothing when n_visible[t]==0.
+ *   q          [batch, Q, H, d] in dtype;  q_scale [batch, Q] fp32 (E4M3)
+ *   w          [batch, Q, H] fp32
+ *   kpool      [batch, ceil(L/B), d] in dtype; kpool_scale [batch, ceil(L/B)]
+ *   n_visible  [batch, Q] int32, 0 <= n_visible <= L
+ *   block_idx  [batch, Q, top_m] int32 (output), -1 padded, any order
+ *   workspace  device scratch of at least
+ *              hisa_workspace_size(HISA_OP_BLOCK_SCORE_TOPM) bytes
+ */
+HISA_API hisa_status hisa_block_score_topm(const void* q, const float* q_scale,
+                                  const float* w, const void* kpool,
+                                  const float* kpool_scale,
+                                  const int32_t* n_visible,
+                                  const hisa_shape* shape, int32_t* block_idx,
+                                  void* workspace, size_t ws_bytes,
+                                  hisa_stream stream);
+
+/*
+ * HISA refinement stage (HISA abstract, stage 2): candidates C_t = keys of
+ * the blocks in block_idx[t,:] (entries -1 are skipped, repeats count once)
+ * that are visible (s < n_visible[t]); topk_idx[t,:] = the top_k of C_t by
+ * I[t,s] (ties -> lower s), all of C_t then -1 padding when |C_t| < top_k.
+ * Candidate scores stay on chip; nothing of size [Q, H, L] is formed.
+ *   k          [batch, L, d] in dtype; k_scale [batch, L] fp32 (E4M3)
+ *   block_idx  [batch, Q, top_m] int32, each entry -1 or in [0, ceil(L/B))
+ *   topk_idx   [batch, Q, top_k] int32 (output)
+ *   topk_score [batch, Q, top_k] fp32 (output, may be NULL; -inf padding)
+ * Requires top_m * block_size <= 16384.
+ */
+HISA_API hisa_status hisa_token_score_topk(const void* q, const float* q_scale,
+                                  const float* w, const void* k,
+                                  const float* k_scale,
+                                  const int32_t* n_visible,
+                                  const int32_t* block_idx,
+                                  const hisa_shape* shape, int32_t* topk_idx,
+                                  float* topk_score, void* workspace,
+                                  size_t ws_bytes, hisa_stream stream);
+
+/*
+ * Flat DSA indexer (the comparison path; HISA abstract: the flat scan of
+ * every prefix key): topk_idx[t,:] = top_k of {0 .. n_visible[t]-1} by
+ * I[t,s], ties -> lower s, -1 padded when n_visible[t] < top_k.
+ * Scores go through the workspace as fp32 rows of at most L values (never
+ * [Q, H, L]); with less workspace than hisa_workspace_size(HISA_OP_FLAT_TOPK)
+ * the queries are processed in chunks that fit.
+ * Arguments as for hisa_token_score_topk (block_size and top_m unused).
+ */
+HISA_API hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale,
+                                  const float* w, const void* k,
+                                  const float* k_scale,
+                                  const int32_t* n_visible,
+                                  const hisa_shape* shape, int32_t* topk_idx,
+                                  float* topk_score, void* workspace,
+                                  size_t ws_bytes, hisa_stream stream);
+
+/* Workspace bytes that let `op` run on `shape` in one pass (0 if none). */
+HISA_API hisa_status hisa_workspace_size(int32_t op, const hisa_shape* shape,
+                                size_t* bytes);
+
+/* Synchronises `stream`, then returns and clears the device status word
+ * (HISA_OK, or HISA_ERR_TIMEOUT if a bounded wait gave up since the last
+ * call); HISA_ERR_CUDA if the synchronisation itself failed. */
+HISA_API hisa_status hisa_get_status(hisa_stream stream);
+
+/* Static description of a status code. */
+HISA_API const char* hisa_status_string(hisa_status status);
+
+/* Message of the last validation or CUDA error on the calling thread. */
+HISA_API const char* hisa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HISA_H_ */

@@ -1,0 +1,86 @@
+"""The C ABI without a GPU: the library loads, exports every entry point
+include/hisa.h declares, and validates arguments on the host (no kernel is
+launched by any call here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hierarchical_top_key_b200 import binding as hb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "hisa.h")).read()
+    return re.findall(r"HISA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+
+
+@pytest.fixture(scope="module")
+def L():
+    return hb.load()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert {"hisa_pool_blocks", "hisa_block_score_topm", "hisa_token_score_topk", "dsa_flat_indexer_topk"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/hisa.h but not exported"
+    assert set(names) == set(hb.EXPORTS), "binding signatures out of step with the header"
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert L.hisa_status_string(code).decode().startswith(hb.STATUS[code])
+
+
+def _shape(**kw):
+    base = dict(batch=1, num_keys=32768, num_queries=32768, heads=64, head_dim=128, block_size=128, top_m=32,
+                top_k=2048, dtype=hb.HISA_BF16)
+    base.update(kw)
+    return hb.Shape(**base)
+
+
+def test_workspace_sizes(L):
+    s = _shape()
+    assert hb.workspace_size(hb.OP_FLAT, s) == 32768 * 32768 * 4
+    assert hb.workspace_size(hb.OP_BLOCK, s) == 32768 * 256 * 4
+    assert hb.workspace_size(hb.OP_TOKEN, s) == 0
+    s = _shape(num_keys=1001, num_queries=3, batch=2, block_size=64)
+    assert hb.workspace_size(hb.OP_FLAT, s) == 6 * 1004 * 4          # rows padded to 16 bytes
+    assert hb.workspace_size(hb.OP_BLOCK, s) == 6 * 16 * 4           # ceil(1001/64)=16
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("head_dim", 96, 2), ("heads", 65, 2), ("heads", 0, 2), ("batch", 0, 1), ("top_k", 0, 1),
+    ("dtype", 7, 1), ("block_size", 0, 1), ("top_m", 0, 1)])
+def test_shape_validation(L, field, value, status):
+    s = _shape(**{field: value})
+    n = ctypes.c_size_t(0)
+    assert L.hisa_workspace_size(hb.OP_BLOCK, ctypes.byref(s), ctypes.byref(n)) == status
+    assert L.hisa_last_error()
+
+
+def test_pointer_validation_returns_before_any_launch(L):
+    s = _shape()
+    # NULL inputs
+    assert L.dsa_flat_indexer_topk(None, None, None, None, None, None, ctypes.byref(s), None, None, None, 0,
+                                   None) == 1
+    # misaligned q (never dereferenced: validation fails first)
+    assert L.hisa_token_score_topk(0x1001, None, 0x2000, 0x3000, None, 0x4000, 0x5000, ctypes.byref(s), 0x6000,
+                                   None, None, 0, None) == 1
+    # E4M3 without scales
+    s8 = _shape(dtype=hb.HISA_E4M3)
+    assert L.hisa_block_score_topm(0x1000, None, 0x2000, 0x3000, None, 0x4000, ctypes.byref(s8), 0x5000, 0x6000,
+                                   1 << 30, None) == 1
+    # workspace too small for one row of block scores
+    assert L.hisa_block_score_topm(0x1000, None, 0x2000, 0x3000, None, 0x4000, ctypes.byref(s), 0x5000, 0x6000,
+                                   16, None) == 3
+    # too many candidates for the on-chip refinement buffer
+    big = _shape(top_m=512, block_size=128)
+    assert L.hisa_token_score_topk(0x1000, None, 0x2000, 0x3000, None, 0x4000, 0x5000, ctypes.byref(big), 0x6000,
+                                   None, None, 0, None) == 2
+    assert L.hisa_pool_blocks(None, None, None, None, ctypes.byref(s), None) == 1
+    assert L.hisa_quantize_e4m3(0x1000, hb.HISA_BF16, 10, 100, 0x2000, 0x3000, None) == 2   # cols % 16
+    assert L.hisa_compress_keys(0x1000, 0x2000, 1, 100, 128, 4, hb.HISA_E4M3, None) == 2
