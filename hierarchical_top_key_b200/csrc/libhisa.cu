@@ -6,11 +6,15 @@
 #include <cstring>
 #include <cstdarg>
 #include <algorithm>
+#include <vector>
+
+#include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "pool.cuh"
 #include "select.cuh"
 #include "score_simt.cuh"
+#include "score_tc.cuh"
 
 using namespace hisa;
 
@@ -91,13 +95,144 @@ hisa_status score_rows_h(const hisa_shape* s, const void* q, const float* qsc, c
   return launch_score_rows<DT, 64>(s, q, qsc, w, keys, ksc, nvis, block_div, L, row0, nrows, out, ld, st);
 }
 
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
+}
+
+// ------------------------------------------------------------ TMA descriptors
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+
+hisa_status tensor_map_2d(CUtensorMap* map, const void* base, int dtype, uint64_t rows, uint64_t cols,
+                          uint32_t box_rows) {
+  if (!g_encode_tiled) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+      return fail(HISA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const int es = elem_bytes(dtype);
+  const CUtensorMapDataType ty = dtype == HISA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * es};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode_tiled(map, ty, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HISA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return HISA_OK;
+}
+
+// ------------------------------------------------------------ dense scoring plan
+
+// Tensor-core path: bf16 or E4M3 rows of 128/256 bytes, and H that divides 256
+// into whole query groups.
+bool dense_tc_ok(const hisa_shape* s) {
+  const int rb = s->head_dim * elem_bytes(s->dtype);
+  return (s->dtype == HISA_BF16 || s->dtype == HISA_E4M3) && (rb == 128 || rb == 256) &&
+         (s->heads == 16 || s->heads == 32 || s->heads == 64);
+}
+
+int dense_group(const hisa_shape* s) { return dense_tc_ok(s) ? kDenseN / s->heads : 1; }
+
+struct RowChunk {
+  int64_t gg0;
+  int ngroups;
+  int64_t row0, nrows;
+};
+
+// Split the (sequence, query-group) space into chunks whose score rows fit
+// in `cap_rows`; every chunk holds whole groups.
+hisa_status plan_chunks(const hisa_shape* s, int G, int64_t cap_rows, std::vector<RowChunk>& out) {
+  const int64_t gps = ceil_div(s->num_queries, G);
+  const int64_t total = gps * s->batch;
+  auto row_of = [&](int64_t gg) { return (gg / gps) * s->num_queries + (gg % gps) * G; };
+  auto row_end = [&](int64_t gg) {
+    return (gg / gps) * s->num_queries + std::min<int64_t>((gg % gps) * G + G, s->num_queries);
+  };
+  out.clear();
+  int64_t gg = 0;
+  while (gg < total) {
+    const int64_t start = gg, r0 = row_of(gg);
+    while (gg < total && row_end(gg) - r0 <= cap_rows && gg - start < (1 << 30)) ++gg;
+    if (gg == start) return fail(HISA_ERR_WORKSPACE, "workspace holds fewer score rows than one query group (%d)", G);
+    out.push_back({start, static_cast<int>(gg - start), r0, row_end(gg - 1) - r0});
+  }
+  return HISA_OK;
+}
+
+template <int DT, int H>
+hisa_status launch_dense_tc(const hisa_shape* s, const CUtensorMap& qmap, const CUtensorMap& kmap, DenseParams p,
+                            cudaStream_t st) {
+  const int rb = s->head_dim * Elem<DT>::bytes;
+  const int tiles_per_group = static_cast<int>(ceil_div(p.L, kDenseTileM));
+  const int sms = num_sms();
+  if (p.ngroups >= 2 * sms) {
+    p.kc_tiles = std::max(tiles_per_group, 1);
+  } else {
+    p.kc_tiles = static_cast<int>(std::max<int64_t>(2, ceil_div(static_cast<int64_t>(tiles_per_group) * p.ngroups, 4 * sms)));
+  }
+  p.max_chunks = static_cast<int>(ceil_div(std::max(tiles_per_group, 1), p.kc_tiles));
+  if (rb == 256) {
+    p.q_bufs = p.kc_tiles > 4 ? 1 : 2;
+    p.stages = p.kc_tiles > 4 ? 4 : 2;
+  } else {
+    p.q_bufs = 2;
+    p.stages = 8;
+  }
+  const size_t smem = dense_smem_bytes(rb, p.stages, p.q_bufs);
+  auto kern = dense_score_tc_kernel<DT, H>;
+  hisa_status e = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(smem)), "dense_score_tc attribute");
+  if (e != HISA_OK) return e;
+  const int64_t units = static_cast<int64_t>(p.ngroups) * p.max_chunks;
+  const int grid = static_cast<int>(std::min<int64_t>(units, sms));
+  kern<<<grid, kDenseThreads, smem, st>>>(qmap, kmap, p);
+  return launch_check("dense_score_tc_kernel");
+}
+
+template <int DT>
+hisa_status dense_tc_h(const hisa_shape* s, const CUtensorMap& qm, const CUtensorMap& km, const DenseParams& p,
+                       cudaStream_t st) {
+  switch (s->heads) {
+    case 16: return launch_dense_tc<DT, 16>(s, qm, km, p, st);
+    case 32: return launch_dense_tc<DT, 32>(s, qm, km, p, st);
+    default: return launch_dense_tc<DT, 64>(s, qm, km, p, st);
+  }
+}
+
+// Score rows of one chunk: out[(b*Q+t) - row0][s] for the visible keys.
 hisa_status score_rows(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* keys,
-                       const float* ksc, const int32_t* nvis, int block_div, int L, int64_t row0,
-                       int64_t nrows, float* out, int64_t ld, cudaStream_t st) {
+                       const float* ksc, const int32_t* nvis, int block_div, int L, const RowChunk& c, float* out,
+                       int64_t ld, cudaStream_t st) {
+  if (dense_tc_ok(s)) {
+    CUtensorMap qm, km;
+    hisa_status e = tensor_map_2d(&qm, q, s->dtype, static_cast<uint64_t>(rows_of(s)) * s->heads, s->head_dim, kDenseN);
+    if (e != HISA_OK) return e;
+    e = tensor_map_2d(&km, keys, s->dtype, static_cast<uint64_t>(s->batch) * L, s->head_dim, kDenseTileM);
+    if (e != HISA_OK) return e;
+    DenseParams p{};
+    p.Q = s->num_queries; p.H = s->heads; p.d = s->head_dim; p.L = L;
+    p.G = kDenseN / s->heads;
+    p.groups_per_seq = static_cast<int>(ceil_div(s->num_queries, p.G));
+    p.block_div = block_div;
+    p.gg0 = c.gg0; p.ngroups = c.ngroups; p.row0 = c.row0;
+    p.w = w; p.n_visible = nvis; p.q_scale = qsc; p.k_scale = ksc; p.out = out; p.ld = ld;
+    return s->dtype == HISA_BF16 ? dense_tc_h<DT_BF16>(s, qm, km, p, st) : dense_tc_h<DT_E4M3>(s, qm, km, p, st);
+  }
   switch (s->dtype) {
-    case HISA_F32: return score_rows_h<DT_F32>(s, q, qsc, w, keys, ksc, nvis, block_div, L, row0, nrows, out, ld, st);
-    case HISA_BF16: return score_rows_h<DT_BF16>(s, q, qsc, w, keys, ksc, nvis, block_div, L, row0, nrows, out, ld, st);
-    default: return score_rows_h<DT_E4M3>(s, q, qsc, w, keys, ksc, nvis, block_div, L, row0, nrows, out, ld, st);
+    case HISA_F32: return score_rows_h<DT_F32>(s, q, qsc, w, keys, ksc, nvis, block_div, L, c.row0, c.nrows, out, ld, st);
+    case HISA_BF16: return score_rows_h<DT_BF16>(s, q, qsc, w, keys, ksc, nvis, block_div, L, c.row0, c.nrows, out, ld, st);
+    default: return score_rows_h<DT_E4M3>(s, q, qsc, w, keys, ksc, nvis, block_div, L, c.row0, c.nrows, out, ld, st);
   }
 }
 
@@ -269,17 +404,16 @@ hisa_status hisa_block_score_topm(const void* q, const float* q_scale, const flo
   const int64_t ld = pad4(nb);
   const int64_t rows = rows_of(s);
   if (!workspace || !aligned16(workspace)) return fail(HISA_ERR_WORKSPACE, "workspace must be non-NULL, 16-byte aligned");
-  const int64_t chunk = std::min<int64_t>(rows, static_cast<int64_t>(ws_bytes / (ld * 4)));
-  if (chunk < 1) return fail(HISA_ERR_WORKSPACE, "workspace holds no row of %lld block scores", (long long)nb);
+  std::vector<RowChunk> chunks;
+  e = plan_chunks(s, dense_group(s), std::min<int64_t>(rows, static_cast<int64_t>(ws_bytes / (ld * 4))), chunks);
+  if (e != HISA_OK) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
-  for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
-    const int64_t nr = std::min(chunk, rows - r0);
-    e = score_rows(s, q, q_scale, w, kpool, kpool_scale, n_visible, s->block_size, static_cast<int>(nb), r0, nr,
-                   ws, ld, st);
+  for (const RowChunk& c : chunks) {
+    e = score_rows(s, q, q_scale, w, kpool, kpool_scale, n_visible, s->block_size, static_cast<int>(nb), c, ws, ld, st);
     if (e != HISA_OK) return e;
-    block_select_kernel<<<static_cast<unsigned>(nr), 512, 0, st>>>(ws, ld, n_visible, r0, s->num_keys, s->block_size, s->top_m,
-                                                                  block_idx);
+    block_select_kernel<<<static_cast<unsigned>(c.nrows), 512, 0, st>>>(ws, ld, n_visible, c.row0, s->num_keys,
+                                                                        s->block_size, s->top_m, block_idx);
     e = launch_check("block_select_kernel");
     if (e != HISA_OK) return e;
   }
@@ -320,16 +454,16 @@ hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale, const flo
   const int64_t ld = pad4(s->num_keys);
   const int64_t rows = rows_of(s);
   if (!workspace || !aligned16(workspace)) return fail(HISA_ERR_WORKSPACE, "workspace must be non-NULL, 16-byte aligned");
-  const int64_t chunk = std::min<int64_t>(rows, static_cast<int64_t>(ws_bytes / (ld * 4)));
-  if (chunk < 1) return fail(HISA_ERR_WORKSPACE, "workspace holds no row of %d scores", s->num_keys);
+  std::vector<RowChunk> chunks;
+  e = plan_chunks(s, dense_group(s), std::min<int64_t>(rows, static_cast<int64_t>(ws_bytes / (ld * 4))), chunks);
+  if (e != HISA_OK) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
-  for (int64_t r0 = 0; r0 < rows; r0 += chunk) {
-    const int64_t nr = std::min(chunk, rows - r0);
-    e = score_rows(s, q, q_scale, w, k, k_scale, n_visible, 0, s->num_keys, r0, nr, ws, ld, st);
+  for (const RowChunk& c : chunks) {
+    e = score_rows(s, q, q_scale, w, k, k_scale, n_visible, 0, s->num_keys, c, ws, ld, st);
     if (e != HISA_OK) return e;
-    flat_select_kernel<<<static_cast<unsigned>(nr), 512, 0, st>>>(ws, ld, n_visible, r0, s->num_keys, s->top_k, topk_idx,
-                                                                 topk_score);
+    flat_select_kernel<<<static_cast<unsigned>(c.nrows), 512, 0, st>>>(ws, ld, n_visible, c.row0, s->num_keys,
+                                                                       s->top_k, topk_idx, topk_score);
     e = launch_check("flat_select_kernel");
     if (e != HISA_OK) return e;
   }

@@ -1,0 +1,301 @@
+// score_tc.cuh - tensor-core (tcgen05) dense causal indexer scoring for the
+// flat DSA indexer and the HISA coarse stage.
+//
+// One MMA tile computes D[s, (t,h)] = k[s,:] . q[t,h,:] for 128 keys s (the
+// A operand, M = 128) against a group of G queries x H heads (the B operand,
+// N = G*H = 256), K = head_dim, accumulating in fp32 in TMEM.  The epilogue
+// reduces over heads inside each thread (TMEM lane = key), so the indexer
+// score I[t,s] = sum_h w[t,h] * max(D[s,(t,h)], 0) costs one max and one FMA
+// per accumulator element and no cross-thread traffic; E4M3 scales are applied
+// to the reduced score.  Scores are written as fp32 rows (one per query) for
+// the row-wise top-k that follows; the [queries, heads, keys] tensor never
+// exists outside TMEM.
+//
+// Persistent, warp-specialised CTA (one per SM):
+//   warp 0      TMA producer: q group (one or two buffers) and key tiles (ring)
+//   warp 1      TMEM owner and MMA issuer (one thread)
+//   warps 2..9  epilogue: TMEM -> registers -> weighted ReLU sum -> global
+// Two TMEM accumulators (2 x 256 columns) let the MMA of tile i+1 overlap the
+// epilogue of tile i.  Work units are (query group, chunk of key tiles); the
+// schedule is static and identical in every role.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace hisa {
+
+constexpr int kDenseTileM = 128;
+constexpr int kDenseN = 256;
+constexpr int kDenseEpiWarps = 8;
+constexpr int kDenseThreads = 64 + 32 * kDenseEpiWarps;
+
+struct DenseParams {
+  int Q, H, d, L;           // L: key rows per sequence (keys, or pooled blocks)
+  int G;                    // queries per group (kDenseN / H)
+  int groups_per_seq;
+  int block_div;            // 0: flat (vis = n); > 0: coarse (vis = (n-1)/block_div)
+  int kc_tiles;             // key tiles per work unit
+  int max_chunks;           // units per group
+  int stages;               // key-tile ring depth (<= 8)
+  int q_bufs;               // q group buffers (1 or 2)
+  int64_t gg0;              // first (sequence, group) handled by this launch
+  int ngroups;
+  int64_t row0;             // output row of query (b, t) is b*Q + t - row0
+  const float* w;
+  const int32_t* n_visible;
+  const float* q_scale;
+  const float* k_scale;
+  float* out;
+  int64_t ld;
+};
+
+struct DenseUnit {
+  int b, t0, nq, tile0, ntiles;
+};
+
+__device__ __forceinline__ int dense_vis(const DenseParams& p, int n) {
+  int v = p.block_div > 0 ? (n > 0 ? (n - 1) / p.block_div : 0) : n;
+  return max(0, min(v, p.L));
+}
+
+// Unit u: groups in descending order (longest causal prefixes first), chunks
+// of kc_tiles key tiles.  ntiles <= 0 means the unit has no visible key.
+__device__ __forceinline__ DenseUnit dense_unit(const DenseParams& p, int64_t u) {
+  DenseUnit U;
+  const int64_t gi = p.ngroups - 1 - u / p.max_chunks;
+  const int chunk = static_cast<int>(u % p.max_chunks);
+  const int64_t gg = p.gg0 + gi;
+  U.b = static_cast<int>(gg / p.groups_per_seq);
+  const int g = static_cast<int>(gg % p.groups_per_seq);
+  U.t0 = g * p.G;
+  U.nq = min(p.G, p.Q - U.t0);
+  int vmax = 0;
+  for (int j = 0; j < U.nq; ++j) vmax = max(vmax, dense_vis(p, __ldg(p.n_visible + static_cast<int64_t>(U.b) * p.Q + U.t0 + j)));
+  const int tiles = (vmax + kDenseTileM - 1) / kDenseTileM;
+  U.tile0 = chunk * p.kc_tiles;
+  U.ntiles = min(p.kc_tiles, tiles - U.tile0);
+  return U;
+}
+
+// Snake order over rounds of gridDim.x units balances the causal triangle.
+__device__ __forceinline__ int64_t dense_unit_index(int64_t round) {
+  const int64_t base = round * gridDim.x;
+  return base + ((round & 1) ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x);
+}
+
+template <int DT, int H>
+__global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, const DenseParams p) {
+  using namespace sm100;
+  constexpr int G = kDenseN / H;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int row_bytes = p.d * Elem<DT>::bytes;           // 128 or 256
+  const int panels = row_bytes / 128;
+  const int panel_elems = 128 / Elem<DT>::bytes;
+  const uint32_t q_bytes = kDenseN * row_bytes;          // per q buffer
+  const uint32_t k_bytes = kDenseTileM * row_bytes;      // per key stage
+  uint8_t* q_buf = smem;                                 // [q_bufs][panels][256][128B]
+  uint8_t* k_buf = smem + p.q_bufs * q_bytes;            // [stages][panels][128][128B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(k_buf + p.stages * k_bytes);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = bars + p.stages;
+  uint64_t* q_full = bars + 2 * p.stages;                // [2]
+  uint64_t* q_empty = q_full + 2;                        // [2]
+  uint64_t* acc_full = q_empty + 2;                      // [2]
+  uint64_t* acc_empty = acc_full + 2;                    // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* w_s = reinterpret_cast<float*>(tmem_slot + 4);  // [8 warps][G/2 * H] = [4 * G * H]
+  float* qsc_s = w_s + 4 * kDenseN;                      // [8 warps][G/2]
+  int* vis_s = reinterpret_cast<int*>(qsc_s + 4 * G);    // [8 warps][G/2]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full + i, 1); mbar_init(q_empty + i, 1);
+      mbar_init(acc_full + i, 1); mbar_init(acc_empty + i, kDenseEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (warp == 0 && lane == 0) { tma_prefetch_desc(&qmap); tma_prefetch_desc(&kmap); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int64_t total_units = static_cast<int64_t>(p.ngroups) * p.max_chunks;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int64_t kt = 0;
+      int un = 0;
+      int64_t last_k[8];
+      for (int s = 0; s < 8; ++s) last_k[s] = -1;
+      int last_q[2] = {-1, -1};
+      bool ok = true;
+      for (int64_t r = 0; ok && r * gridDim.x < total_units; ++r) {
+        const int64_t u = dense_unit_index(r);
+        if (u >= total_units) continue;
+        const DenseUnit U = dense_unit(p, u);
+        if (U.ntiles <= 0) continue;
+        const int qb = un % p.q_bufs;
+        if (!(ok = mbar_wait(q_empty + qb, ((un / p.q_bufs) & 1) ^ 1, abort_flag))) break;
+        mbar_arrive_expect_tx(q_full + qb, q_bytes);
+        const int qrow = (U.b * p.Q + U.t0) * p.H;
+        for (int pn = 0; pn < panels; ++pn)
+          tma_load_2d(q_buf + qb * q_bytes + pn * (kDenseN * 128), &qmap, q_full + qb, pn * panel_elems, qrow);
+        last_q[qb] = un;
+        for (int i = 0; i < U.ntiles; ++i, ++kt) {
+          const int st = static_cast<int>(kt % p.stages);
+          if (!(ok = mbar_wait(k_empty + st, static_cast<uint32_t>(((kt / p.stages) & 1) ^ 1), abort_flag))) break;
+          mbar_arrive_expect_tx(k_full + st, k_bytes);
+          const int krow = U.b * p.L + (U.tile0 + i) * kDenseTileM;
+          for (int pn = 0; pn < panels; ++pn)
+            tma_load_2d(k_buf + st * k_bytes + pn * (kDenseTileM * 128), &kmap, k_full + st, pn * panel_elems, krow);
+          last_k[st] = kt;
+        }
+        ++un;
+      }
+      if (!ok) {   // drain the copies this thread issued before leaving
+        for (int s = 0; s < p.stages; ++s)
+          if (last_k[s] >= 0) mbar_drain(k_full + s, static_cast<uint32_t>((last_k[s] / p.stages) & 1));
+        for (int i = 0; i < 2; ++i)
+          if (last_q[i] >= 0) mbar_drain(q_full + i, static_cast<uint32_t>((last_q[i] / p.q_bufs) & 1));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc(kDenseTileM, kDenseN, DT == DT_BF16 ? 1u : 0u);
+      const int ksteps = row_bytes / 32;       // 32 bytes of K per MMA (16 bf16 / 32 e4m3)
+      int64_t kt = 0, tc = 0;
+      int un = 0;
+      bool ok = true;
+      for (int64_t r = 0; ok && r * gridDim.x < total_units; ++r) {
+        const int64_t u = dense_unit_index(r);
+        if (u >= total_units) continue;
+        const DenseUnit U = dense_unit(p, u);
+        if (U.ntiles <= 0) continue;
+        const int qb = un % p.q_bufs;
+        if (!(ok = mbar_wait(q_full + qb, (un / p.q_bufs) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(q_buf + qb * q_bytes);
+        for (int i = 0; i < U.ntiles; ++i, ++kt, ++tc) {
+          const int st = static_cast<int>(kt % p.stages);
+          const int ab = static_cast<int>(tc & 1);
+          if (!(ok = mbar_wait(acc_empty + ab, static_cast<uint32_t>(((tc >> 1) & 1) ^ 1), abort_flag))) break;
+          if (!(ok = mbar_wait(k_full + st, static_cast<uint32_t>((kt / p.stages) & 1), abort_flag))) break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(k_buf + st * k_bytes);
+          const uint32_t d_tmem = tmem_base + ab * kDenseN;
+          for (int ks = 0; ks < ksteps; ++ks) {
+            const int pn = ks >> 2, off = (ks & 3) * 32;
+            const uint64_t a = desc_k_sw128(k_addr + pn * (kDenseTileM * 128) + off);
+            const uint64_t b = desc_k_sw128(q_addr + pn * (kDenseN * 128) + off);
+            mma<DT>(d_tmem, a, b, idesc, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(k_empty + st);
+          mma_commit(acc_full + ab);
+        }
+        if (ok) mma_commit(q_empty + qb);
+        ++un;
+      }
+      mma_commit(drain);
+      mbar_drain(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // Each warp stages the weights, visibility and scales of its own queries
+    // (no cross-warp barrier inside the loop, so an abort cannot strand a
+    // warp); lane 0 alone waits on the accumulator barrier.
+    const int e = warp - 2;
+    const int quarter = warp & 3;                 // TMEM lanes this warp may access
+    const int half = e >> 2;                      // which half of the group's queries
+    constexpr int QPT = G / 2;                    // queries per thread
+    float* w_w = w_s + e * (QPT * H);
+    float* qsc_w = qsc_s + e * QPT;
+    int* vis_w = vis_s + e * QPT;
+    int64_t tc = 0;
+    bool ok = true;
+    for (int64_t r = 0; ok && r * gridDim.x < total_units; ++r) {
+      const int64_t u = dense_unit_index(r);
+      if (u >= total_units) continue;
+      const DenseUnit U = dense_unit(p, u);
+      if (U.ntiles <= 0) continue;
+      const int64_t qrow0 = static_cast<int64_t>(U.b) * p.Q + U.t0;
+      __syncwarp();
+      for (int i = lane; i < QPT * H; i += 32) {
+        const int j = half * QPT + i / H;
+        w_w[i] = j < U.nq ? __ldg(p.w + (qrow0 + j) * p.H + (i % H)) : 0.f;
+      }
+      for (int jq = lane; jq < QPT; jq += 32) {
+        const int j = half * QPT + jq;
+        vis_w[jq] = j < U.nq ? dense_vis(p, __ldg(p.n_visible + qrow0 + j)) : 0;
+        qsc_w[jq] = (DT == DT_E4M3 && j < U.nq) ? __ldg(p.q_scale + qrow0 + j) : 1.f;
+      }
+      __syncwarp();
+      for (int i = 0; i < U.ntiles; ++i, ++tc) {
+        const int ab = static_cast<int>(tc & 1);
+        int okl = 1;
+        if (lane == 0) okl = mbar_wait(acc_full + ab, static_cast<uint32_t>((tc >> 1) & 1), abort_flag) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+        if (!ok) break;
+        tc_fence_after();
+        const int s = (U.tile0 + i) * kDenseTileM + quarter * 32 + lane;
+        float ksc = 1.f;
+        if (DT == DT_E4M3 && s < p.L) ksc = __ldg(p.k_scale + static_cast<int64_t>(U.b) * p.L + s);
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * kDenseN;
+#pragma unroll 1
+        for (int jq = 0; jq < QPT; ++jq) {
+          const int j = half * QPT + jq;
+          const float* wq = w_w + jq * H;
+          float acc = 0.f;
+          if (H >= 32) {
+#pragma unroll
+            for (int c0 = 0; c0 < H; c0 += 32) {
+              uint32_t v[32];
+              tmem_ld32(t_row + j * H + c0, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) acc = fmaf(wq[c0 + c], fmaxf(__uint_as_float(v[c]), 0.f), acc);
+            }
+          } else {
+            uint32_t v[16];
+            tmem_ld16(t_row + j * H, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 16; ++c) acc = fmaf(wq[c], fmaxf(__uint_as_float(v[c]), 0.f), acc);
+          }
+          if (s < vis_w[jq]) {
+            if (DT == DT_E4M3) acc *= qsc_w[jq] * ksc;
+            p.out[(qrow0 + j - p.row0) * p.ld + s] = acc;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty + ab);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// Bytes of dynamic shared memory the dense kernel needs.
+inline size_t dense_smem_bytes(int row_bytes, int stages, int q_bufs) {
+  return 1024 /*alignment slack*/ + q_bufs * static_cast<size_t>(kDenseN) * row_bytes +
+         static_cast<size_t>(stages) * kDenseTileM * row_bytes + 8 * (2 * stages + 9) + 16 + 4 * 4 * kDenseN +
+         2 * 4 * 4 * 64 + 64;
+}
+
+}  // namespace hisa

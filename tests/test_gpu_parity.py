@@ -47,6 +47,8 @@ SMALL = {
 def _sample_queries(wl, n_rand, seed=0, max_boundaries=24):
     Q = wl.num_queries
     B = wl.block_size
+    if n_rand >= Q:
+        return list(range(Q))
     pick = {0, 1, Q - 1, Q - 2}
     rng = np.random.default_rng(seed)
     bounds = list(range(0, Q, max(1, B)))
