@@ -15,6 +15,7 @@
 #include "select.cuh"
 #include "score_simt.cuh"
 #include "score_tc.cuh"
+#include "token_tc.cuh"
 
 using namespace hisa;
 
@@ -261,6 +262,59 @@ hisa_status token_simt_h(const hisa_shape* s, const void* q, const float* qsc, c
   return launch_token_simt<DT, 64>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st);
 }
 
+constexpr size_t kSmemBudget = 232448;   // 227 KB opt-in dynamic shared memory per CTA
+
+bool token_tc_ok(const hisa_shape* s) {
+  const int rb = s->head_dim * elem_bytes(s->dtype);
+  return (s->dtype == HISA_BF16 || s->dtype == HISA_E4M3) && (rb == 128 || rb == 256) &&
+         (s->heads == 16 || s->heads == 32 || s->heads == 64) &&
+         (s->block_size == 16 || s->block_size == 32 || s->block_size == 64 || s->block_size == 128) &&
+         s->top_m <= kTokMaxBlocks;
+}
+
+template <int DT, int H>
+hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* k,
+                            const float* ksc, const int32_t* nvis, const int32_t* bidx, int32_t* oi, float* os,
+                            cudaStream_t st) {
+  const int rb = s->head_dim * Elem<DT>::bytes;
+  TokenParams p{};
+  p.rows = rows_of(s);
+  p.Q = s->num_queries; p.H = s->heads; p.d = s->head_dim; p.L = s->num_keys; p.B = s->block_size;
+  p.top_m = s->top_m; p.top_k = s->top_k;
+  p.nb = static_cast<int>(num_blocks(s));
+  p.max_cand = static_cast<int>(ceil_div(static_cast<int64_t>(s->top_m) * s->block_size, kTokTileM) * kTokTileM);
+  p.w = w; p.n_visible = nvis; p.block_idx = bidx; p.q_scale = qsc; p.k_scale = ksc; p.out_idx = oi; p.out_score = os;
+  const size_t fixed = token_smem_bytes(rb, H, 0, p.max_cand) + 16 * 8;
+  const size_t kb = static_cast<size_t>(kTokTileM) * rb;
+  if (fixed + 2 * kb > kSmemBudget)
+    return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size too large for the on-chip candidate buffers");
+  p.stages = static_cast<int>(std::min<size_t>(6, (kSmemBudget - fixed) / kb));
+  const size_t smem = token_smem_bytes(rb, H, p.stages, p.max_cand);
+  CUtensorMap qm, km;
+  hisa_status e = tensor_map_2d(&qm, q, s->dtype, static_cast<uint64_t>(p.rows) * H, s->head_dim, H);
+  if (e != HISA_OK) return e;
+  e = tensor_map_2d(&km, k, s->dtype, static_cast<uint64_t>(s->batch) * s->num_keys, s->head_dim, s->block_size);
+  if (e != HISA_OK) return e;
+  auto kern = token_tc_kernel<DT, H>;
+  e = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
+                 "token_tc attribute");
+  if (e != HISA_OK) return e;
+  const int grid = static_cast<int>(std::min<int64_t>(p.rows, num_sms()));
+  kern<<<grid, kTokThreads, smem, st>>>(qm, km, p);
+  return launch_check("token_tc_kernel");
+}
+
+template <int DT>
+hisa_status token_tc_h(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* k,
+                       const float* ksc, const int32_t* nvis, const int32_t* bidx, int32_t* oi, float* os,
+                       cudaStream_t st) {
+  switch (s->heads) {
+    case 16: return launch_token_tc<DT, 16>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st);
+    case 32: return launch_token_tc<DT, 32>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st);
+    default: return launch_token_tc<DT, 64>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st);
+  }
+}
+
 hisa_status check_indexer_ptrs(const hisa_shape* s, const void* q, const float* q_scale, const float* w,
                                const void* k, const float* k_scale, const int32_t* n_visible) {
   if (!q || !w || !k || !n_visible) return fail(HISA_ERR_INVALID_ARG, "q, w, keys and n_visible must be non-NULL");
@@ -435,6 +489,11 @@ hisa_status hisa_token_score_topk(const void* q, const float* q_scale, const flo
   if (static_cast<int64_t>(s->top_m) * s->block_size > kMaxCandidates)
     return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size must be <= %d", kMaxCandidates);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (token_tc_ok(s)) {
+    return s->dtype == HISA_BF16
+               ? token_tc_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st)
+               : token_tc_h<DT_E4M3>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
+  }
   switch (s->dtype) {
     case HISA_F32: return token_simt_h<DT_F32>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
     case HISA_BF16: return token_simt_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);

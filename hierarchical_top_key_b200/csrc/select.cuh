@@ -13,11 +13,27 @@
 
 namespace hisa {
 
+// A set of threads that selects together: the whole CTA, or a run of whole
+// warps synchronised by a named barrier.
+struct CtaGroup {
+  __device__ __forceinline__ static int tid() { return threadIdx.x; }
+  __device__ __forceinline__ static int size() { return blockDim.x; }
+  __device__ __forceinline__ static void sync() { __syncthreads(); }
+};
+template <int BASE, int N, int ID>
+struct WarpRange {
+  static_assert(BASE % 32 == 0 && N % 32 == 0, "whole warps");
+  __device__ __forceinline__ static int tid() { return static_cast<int>(threadIdx.x) - BASE; }
+  __device__ __forceinline__ static int size() { return N; }
+  __device__ __forceinline__ static void sync() { asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(N) : "memory"); }
+};
+
 struct SelectSmem {
   uint32_t hist[256];
   uint32_t warp_cnt[32];
   uint32_t digit;
   uint32_t above;
+  uint32_t at_digit;       // histogram count of the chosen digit (last pass: elements equal to T)
   uint32_t n_gt_slots;     // running slot counter for key > T
   uint32_t eq_base;        // equal-to-T elements seen in earlier chunks
   uint32_t n_valid;
@@ -25,54 +41,57 @@ struct SelectSmem {
 
 // Block-wide exclusive prefix of a 0/1 flag over the threads (in thread
 // order); returns the prefix and writes the block total to *total.
+template <class Grp = CtaGroup>
 __device__ __forceinline__ uint32_t block_flag_prefix(bool flag, SelectSmem& sm, uint32_t* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int lane = Grp::tid() & 31, wid = Grp::tid() >> 5, nw = Grp::size() >> 5;
   const uint32_t ball = __ballot_sync(0xffffffffu, flag);
   if (lane == 0) sm.warp_cnt[wid] = __popc(ball);
-  __syncthreads();
+  Grp::sync();
   uint32_t off = 0, tot = 0;
   for (int i = 0; i < nw; ++i) {
     const uint32_t c = sm.warp_cnt[i];
     off += (i < wid) ? c : 0;
     tot += c;
   }
-  __syncthreads();
+  Grp::sync();
   *total = tot;
   return off + __popc(ball & ((1u << lane) - 1u));
 }
 
 // Count of keys != 0 among positions [0, n).
-template <class KeyAt>
+template <class KeyAt, class Grp = CtaGroup>
 __device__ uint32_t block_count_valid(KeyAt key_at, int n, SelectSmem& sm) {
   uint32_t c = 0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) c += key_at(i) != 0u;
+  for (int i = Grp::tid(); i < n; i += Grp::size()) c += key_at(i) != 0u;
   c = __reduce_add_sync(0xffffffffu, c);
-  if (threadIdx.x == 0) sm.n_valid = 0;
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) atomicAdd(&sm.n_valid, c);
-  __syncthreads();
-  return sm.n_valid;
+  if (Grp::tid() == 0) sm.n_valid = 0;
+  Grp::sync();
+  if ((Grp::tid() & 31) == 0) atomicAdd(&sm.n_valid, c);
+  Grp::sync();
+  const uint32_t v = sm.n_valid;
+  Grp::sync();
+  return v;
 }
 
 // Emit(slot, position, key) for the k largest keys among [0, n).  Requires
 // blockDim.x to be a multiple of 32 (<= 1024) and more than k valid keys.
 // Returns nothing; every slot 0..k-1 is emitted exactly once.
-template <class KeyAt, class Emit>
+template <class KeyAt, class Emit, class Grp = CtaGroup>
 __device__ void block_radix_topk(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem& sm) {
   uint32_t prefix = 0, remaining = k;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) sm.hist[i] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    for (int i = Grp::tid(); i < 256; i += Grp::size()) sm.hist[i] = 0;
+    Grp::sync();
+    for (int i = Grp::tid(); i < n; i += Grp::size()) {
       const uint32_t key = key_at(i);
       if (key != 0u && ((key ^ prefix) & hi_mask) == 0u) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
     }
-    __syncthreads();
-    if (threadIdx.x < 32) {
+    Grp::sync();
+    if (Grp::tid() < 32) {
       // lane l holds bins 255-8l .. 248-8l (descending), suffix sums across lanes
-      const int lane = threadIdx.x;
+      const int lane = Grp::tid();
       uint32_t h[8], t = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) { h[j] = sm.hist[255 - 8 * lane - j]; t += h[j]; }
@@ -89,52 +108,68 @@ __device__ void block_radix_topk(KeyAt key_at, int n, uint32_t k, Emit emit, Sel
         uint32_t c = excl;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          if (c + h[j] >= remaining) { sm.digit = 255 - 8 * lane - j; sm.above = c; break; }
+          if (c + h[j] >= remaining) { sm.digit = 255 - 8 * lane - j; sm.above = c; sm.at_digit = h[j]; break; }
           c += h[j];
         }
       }
     }
-    __syncthreads();
+    Grp::sync();
     prefix |= sm.digit << shift;
     remaining -= sm.above;
-    __syncthreads();
+    Grp::sync();
   }
   // prefix is the k-th largest key; `remaining` elements equal to it are taken
   const uint32_t T = prefix, need_eq = remaining, n_gt = k - remaining;
-  if (threadIdx.x == 0) { sm.n_gt_slots = 0; sm.eq_base = 0; }
-  __syncthreads();
-  for (int base = 0; base < n; base += blockDim.x) {
-    const int i = base + threadIdx.x;
+  const uint32_t n_eq = sm.at_digit;
+  if (Grp::tid() == 0) { sm.n_gt_slots = 0; sm.eq_base = 0; }
+  Grp::sync();
+  if (need_eq == n_eq) {
+    // no tie is cut at the boundary: every key >= T is taken, in any order
+    for (int base = 0; base < n; base += Grp::size()) {
+      const int i = base + Grp::tid();
+      const uint32_t key = i < n ? key_at(i) : 0u;
+      const bool take = key >= T && key != 0u;
+      const uint32_t ball = __ballot_sync(0xffffffffu, take);
+      uint32_t base_slot = 0;
+      if ((Grp::tid() & 31) == 0 && ball) base_slot = atomicAdd(&sm.n_gt_slots, __popc(ball));
+      base_slot = __shfl_sync(0xffffffffu, base_slot, 0);
+      if (take) emit(base_slot + __popc(ball & ((1u << (Grp::tid() & 31)) - 1u)), i, key);
+    }
+    Grp::sync();
+    return;
+  }
+  for (int base = 0; base < n; base += Grp::size()) {
+    const int i = base + Grp::tid();
     const uint32_t key = i < n ? key_at(i) : 0u;
     if (key > T) {
       const uint32_t slot = atomicAdd(&sm.n_gt_slots, 1u);
       emit(slot, i, key);
     }
     uint32_t tot;
-    const uint32_t rank = block_flag_prefix(key == T && key != 0u, sm, &tot);
+    const uint32_t rank = block_flag_prefix<Grp>(key == T && key != 0u, sm, &tot);
     const uint32_t r = sm.eq_base + rank;
     if (key == T && key != 0u && r < need_eq) emit(n_gt + r, i, key);
-    __syncthreads();
-    if (threadIdx.x == 0) sm.eq_base += tot;
-    __syncthreads();
+    Grp::sync();
+    if (Grp::tid() == 0) sm.eq_base += tot;
+    Grp::sync();
   }
 }
 
 // Emit every valid key (key != 0) among [0, n) in position order into slots
 // 0..n_valid-1 (used when there are no more than k of them).
-template <class KeyAt, class Emit>
+template <class KeyAt, class Emit, class Grp = CtaGroup>
 __device__ void block_emit_all(KeyAt key_at, int n, Emit emit, SelectSmem& sm) {
-  if (threadIdx.x == 0) sm.eq_base = 0;
-  __syncthreads();
-  for (int base = 0; base < n; base += blockDim.x) {
-    const int i = base + threadIdx.x;
+  if (Grp::tid() == 0) sm.eq_base = 0;
+  Grp::sync();
+  for (int base = 0; base < n; base += Grp::size()) {
+    const int i = base + Grp::tid();
     const uint32_t key = i < n ? key_at(i) : 0u;
     uint32_t tot;
-    const uint32_t rank = block_flag_prefix(key != 0u, sm, &tot);
+    const uint32_t rank = block_flag_prefix<Grp>(key != 0u, sm, &tot);
     if (key != 0u) emit(sm.eq_base + rank, i, key);
-    __syncthreads();
-    if (threadIdx.x == 0) sm.eq_base += tot;
-    __syncthreads();
+    Grp::sync();
+    if (Grp::tid() == 0) sm.eq_base += tot;
+    Grp::sync();
   }
 }
 

@@ -1,0 +1,370 @@
+// token_tc.cuh - fused HISA refinement stage on tensor cores.
+//
+// For each query t: the keys of its retained blocks are gathered by TMA
+// (each block is a contiguous run of B key rows, so one tile load per block),
+// scored against q[t] with tcgen05 (M = 128 candidate keys, N = H heads,
+// K = head_dim, fp32 accumulators in TMEM), reduced over heads with the
+// weighted ReLU in-thread, kept in shared memory as ordering keys, and the
+// top-k is selected on chip.  Candidate scores never reach global memory.
+//
+// Persistent, warp-specialised CTA (one per SM), queries processed as a
+// pipeline of jobs:
+//   warp 0       job set-up (whole warp: read, filter, dedupe and sort the
+//                block list; stage w[t]) then TMA issue (lane 0)
+//   warp 1       TMEM owner and MMA issuer
+//   warps 2..5   scorer: TMEM -> weighted ReLU sum -> candidate keys in smem
+//   warps 6..13  selector: radix top-k over the candidate keys, emit indices
+// Rings: job slots (4), q buffers (2), key stages, TMEM accumulators (4 x H
+// columns), candidate buffers (2).  Blocks are sorted ascending so candidate
+// position order is key order, which makes ties resolve to the lower key.
+#pragma once
+#include "common.cuh"
+#include "select.cuh"
+#include "sm100.cuh"
+
+namespace hisa {
+
+constexpr int kTokTileM = 128;
+constexpr int kTokJobs = 4;
+constexpr int kTokAcc = 4;
+constexpr int kTokScorerWarps = 4;
+constexpr int kTokSelectWarps = 8;
+constexpr int kTokSelectBase = 32 * (2 + kTokScorerWarps);
+constexpr int kTokThreads = kTokSelectBase + 32 * kTokSelectWarps;
+constexpr int kTokMaxBlocks = 256;
+
+struct TokenParams {
+  int64_t rows;            // batch * Q
+  int Q, H, d, L, B, top_m, top_k;
+  int nb;                  // ceil(L / B)
+  int max_cand;            // top_m * B rounded up to whole tiles
+  int stages;
+  const float* w;
+  const int32_t* n_visible;
+  const int32_t* block_idx;
+  const float* q_scale;
+  const float* k_scale;
+  int32_t* out_idx;
+  float* out_score;
+};
+
+struct TokJob {
+  int64_t row;
+  int b, n, nblk, ntiles;
+  float qsc;
+  float w[64];
+  int blk[kTokMaxBlocks];
+};
+
+__device__ __forceinline__ int64_t tok_job_row(const TokenParams& p, int64_t j) {
+  // largest prefixes first
+  return p.rows - 1 - (static_cast<int64_t>(blockIdx.x) + j * gridDim.x);
+}
+
+template <int DT, int H>
+__global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, const TokenParams p) {
+  using namespace sm100;
+  using SelGrp = WarpRange<kTokSelectBase, 32 * kTokSelectWarps, 2>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int row_bytes = p.d * Elem<DT>::bytes;
+  const int panels = row_bytes / 128;
+  const int panel_elems = 128 / Elem<DT>::bytes;
+  const uint32_t q_bytes = H * row_bytes;
+  const uint32_t k_bytes = kTokTileM * row_bytes;
+  const int blocks_per_tile = kTokTileM / p.B;
+  uint8_t* q_buf = smem;                                         // [2][panels][H][128B]
+  uint8_t* k_buf = q_buf + 2 * q_bytes;                          // [stages][panels][128][128B]
+  uint32_t* cand = reinterpret_cast<uint32_t*>(k_buf + p.stages * k_bytes);   // [2][max_cand]
+  TokJob* jobs = reinterpret_cast<TokJob*>(cand + 2 * p.max_cand);            // [kTokJobs]
+  SelectSmem* sel = reinterpret_cast<SelectSmem*>(jobs + kTokJobs);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uintptr_t>(sel + 1) + 7 & ~uintptr_t(7));
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = k_full + p.stages;
+  uint64_t* q_full = k_empty + p.stages;          // [2]
+  uint64_t* q_empty = q_full + 2;                 // [2]
+  uint64_t* acc_full = q_empty + 2;               // [kTokAcc]
+  uint64_t* acc_empty = acc_full + kTokAcc;       // [kTokAcc]
+  uint64_t* job_full = acc_empty + kTokAcc;       // [kTokJobs]
+  uint64_t* job_empty = job_full + kTokJobs;      // [kTokJobs]
+  uint64_t* cand_full = job_empty + kTokJobs;     // [2]
+  uint64_t* cand_empty = cand_full + 2;           // [2]
+  uint64_t* drain = cand_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* sel_ok = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full + i, 1); mbar_init(q_empty + i, 1);
+      mbar_init(cand_full + i, kTokScorerWarps); mbar_init(cand_empty + i, 1);
+    }
+    for (int i = 0; i < kTokAcc; ++i) { mbar_init(acc_full + i, 1); mbar_init(acc_empty + i, kTokScorerWarps); }
+    for (int i = 0; i < kTokJobs; ++i) { mbar_init(job_full + i, 1); mbar_init(job_empty + i, 1); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTokAcc * H < 32 ? 32 : kTokAcc * H);
+  if (warp == 0 && lane == 0) { tma_prefetch_desc(&qmap); tma_prefetch_desc(&kmap); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int64_t njobs = p.rows > blockIdx.x ? (p.rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ job set-up + TMA
+    int64_t kt = 0;
+    int64_t last_k[8];
+    for (int s = 0; s < 8; ++s) last_k[s] = -1;
+    int64_t last_q[2] = {-1, -1};
+    bool ok = true;
+    for (int64_t j = 0; j < njobs; ++j) {
+      const int slot = static_cast<int>(j % kTokJobs);
+      int okl = 1;
+      if (lane == 0) okl = mbar_wait(job_empty + slot, static_cast<uint32_t>(((j / kTokJobs) & 1) ^ 1), abort_flag);
+      if (!(ok = __shfl_sync(0xffffffffu, okl, 0) != 0)) break;
+      TokJob& J = jobs[slot];
+      const int64_t row = tok_job_row(p, j);
+      const int b = static_cast<int>(row / p.Q);
+      const int n = max(0, min(__ldg(p.n_visible + row), p.L));
+      // raw block list -> J.blk (scratch), then rank-sort the valid, distinct entries
+      for (int i = lane; i < p.top_m; i += 32) J.blk[i] = __ldg(p.block_idx + row * p.top_m + i);
+      __syncwarp();
+      // keep = valid and not a repeat of an earlier entry; rank = number of
+      // kept values below it.  O(top_m) work per entry, ballots carry the keep set.
+      constexpr int KW = kTokMaxBlocks / 32;
+      int mine[KW];
+      uint32_t keepmask[KW];
+#pragma unroll
+      for (int k = 0; k < KW; ++k) {
+        const int i = lane + 32 * k;
+        int x = -1;
+        bool keep = false;
+        if (32 * k < p.top_m && i < p.top_m) {
+          x = J.blk[i];
+          keep = x >= 0 && x < p.nb && x * p.B < n;
+          for (int i2 = 0; keep && i2 < i; ++i2) keep = J.blk[i2] != x;
+        }
+        mine[k] = keep ? x : -1;
+        keepmask[k] = __ballot_sync(0xffffffffu, keep);
+      }
+      int rank[KW];
+      int cnt = 0;
+#pragma unroll
+      for (int k = 0; k < KW; ++k) {
+        cnt += __popc(keepmask[k]);
+        rank[k] = 0;
+        if (mine[k] >= 0) {
+          int r = 0;
+#pragma unroll
+          for (int k2 = 0; k2 < KW; ++k2) {
+            uint32_t m2 = keepmask[k2];
+            while (m2) {
+              const int bit = __ffs(m2) - 1;
+              m2 &= m2 - 1;
+              r += J.blk[32 * k2 + bit] < mine[k];
+            }
+          }
+          rank[k] = r;
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int k = 0; k < KW; ++k)
+        if (mine[k] >= 0) J.blk[rank[k]] = mine[k];
+      for (int h = lane; h < 64; h += 32) J.w[h] = h < p.H ? __ldg(p.w + row * p.H + h) : 0.f;
+      if (lane == 0) {
+        J.row = row;
+        J.b = b;
+        J.n = n;
+        J.nblk = cnt;
+        J.ntiles = (cnt * p.B + kTokTileM - 1) / kTokTileM;
+        J.qsc = DT == DT_E4M3 ? __ldg(p.q_scale + row) : 1.f;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(job_full + slot);
+        // q[t]
+        const int qb = static_cast<int>(j & 1);
+        if ((ok = mbar_wait(q_empty + qb, static_cast<uint32_t>(((j >> 1) & 1) ^ 1), abort_flag))) {
+          mbar_arrive_expect_tx(q_full + qb, q_bytes);
+          for (int pn = 0; pn < panels; ++pn)
+            tma_load_2d(q_buf + qb * q_bytes + pn * (H * 128), &qmap, q_full + qb, pn * panel_elems,
+                        static_cast<int>(row * p.H));
+          last_q[qb] = j;
+          // key tiles: blocks_per_tile consecutive retained blocks per tile
+          const int ntiles = (cnt * p.B + kTokTileM - 1) / kTokTileM;
+          for (int tl = 0; ok && tl < ntiles; ++tl, ++kt) {
+            const int st = static_cast<int>(kt % p.stages);
+            if (!(ok = mbar_wait(k_empty + st, static_cast<uint32_t>(((kt / p.stages) & 1) ^ 1), abort_flag))) break;
+            const int first = tl * blocks_per_tile;
+            const int nblk_t = min(blocks_per_tile, cnt - first);
+            mbar_arrive_expect_tx(k_full + st, static_cast<uint32_t>(nblk_t * p.B * row_bytes));
+            for (int q = 0; q < nblk_t; ++q) {
+              const int krow = b * p.L + J.blk[first + q] * p.B;
+              for (int pn = 0; pn < panels; ++pn)
+                tma_load_2d(k_buf + st * k_bytes + pn * (kTokTileM * 128) + q * p.B * 128, &kmap, k_full + st,
+                            pn * panel_elems, krow);
+            }
+            last_k[st] = kt;
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+    }
+    if (!ok && lane == 0) {
+      for (int s = 0; s < p.stages; ++s)
+        if (last_k[s] >= 0) mbar_drain(k_full + s, static_cast<uint32_t>((last_k[s] / p.stages) & 1));
+      for (int i = 0; i < 2; ++i)
+        if (last_q[i] >= 0) mbar_drain(q_full + i, static_cast<uint32_t>((last_q[i] >> 1) & 1));
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc(kTokTileM, H, DT == DT_BF16 ? 1u : 0u);
+      const int ksteps = row_bytes / 32;
+      int64_t kt = 0, tc = 0;
+      bool ok = true;
+      for (int64_t j = 0; ok && j < njobs; ++j) {
+        const int slot = static_cast<int>(j % kTokJobs);
+        if (!(ok = mbar_wait(job_full + slot, static_cast<uint32_t>((j / kTokJobs) & 1), abort_flag))) break;
+        const int ntiles = jobs[slot].ntiles;
+        const int qb = static_cast<int>(j & 1);
+        if (!(ok = mbar_wait(q_full + qb, static_cast<uint32_t>((j >> 1) & 1), abort_flag))) break;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(q_buf + qb * q_bytes);
+        for (int i = 0; i < ntiles; ++i, ++kt, ++tc) {
+          const int st = static_cast<int>(kt % p.stages);
+          const int ab = static_cast<int>(tc % kTokAcc);
+          if (!(ok = mbar_wait(acc_empty + ab, static_cast<uint32_t>(((tc / kTokAcc) & 1) ^ 1), abort_flag))) break;
+          if (!(ok = mbar_wait(k_full + st, static_cast<uint32_t>((kt / p.stages) & 1), abort_flag))) break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(k_buf + st * k_bytes);
+          const uint32_t d_tmem = tmem_base + ab * H;
+          for (int ks = 0; ks < ksteps; ++ks) {
+            const int pn = ks >> 2, off = (ks & 3) * 32;
+            mma<DT>(d_tmem, desc_k_sw128(k_addr + pn * (kTokTileM * 128) + off),
+                    desc_k_sw128(q_addr + pn * (H * 128) + off), idesc, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(k_empty + st);
+          mma_commit(acc_full + ab);
+        }
+        if (ok) mma_commit(q_empty + qb);
+      }
+      mma_commit(drain);
+      mbar_drain(drain, 0);
+    }
+  } else if (warp < 2 + kTokScorerWarps) {
+    // ------------------------------------------------------------ scorer
+    const int quarter = warp & 3;
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    int64_t tc = 0;
+    bool ok = true;
+    for (int64_t j = 0; ok && j < njobs; ++j) {
+      const int slot = static_cast<int>(j % kTokJobs);
+      const int cb = static_cast<int>(j & 1);
+      int okl = 1;
+      if (lane == 0) {
+        okl = mbar_wait(job_full + slot, static_cast<uint32_t>((j / kTokJobs) & 1), abort_flag) &&
+              mbar_wait(cand_empty + cb, static_cast<uint32_t>(((j >> 1) & 1) ^ 1), abort_flag);
+      }
+      if (!(ok = __shfl_sync(0xffffffffu, okl, 0) != 0)) break;
+      const TokJob& J = jobs[slot];
+      const int ntiles = J.ntiles;
+      uint32_t* cj = cand + cb * p.max_cand;
+      float ksc = 1.f;
+      for (int i = 0; i < ntiles; ++i, ++tc) {
+        const int ab = static_cast<int>(tc % kTokAcc);
+        if (lane == 0) okl = mbar_wait(acc_full + ab, static_cast<uint32_t>((tc / kTokAcc) & 1), abort_flag);
+        if (!(ok = __shfl_sync(0xffffffffu, okl, 0) != 0)) break;
+        tc_fence_after();
+        const int c = i * kTokTileM + quarter * 32 + lane;        // candidate position
+        const int slot_b = c / p.B;
+        const int s = slot_b < J.nblk ? J.blk[slot_b] * p.B + c % p.B : p.L;
+        const bool valid = s < J.n;
+        if (DT == DT_E4M3 && valid) ksc = __ldg(p.k_scale + static_cast<int64_t>(J.b) * p.L + s);
+        float acc = 0.f;
+        if (H >= 32) {
+#pragma unroll
+          for (int c0 = 0; c0 < H; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(t_lane + ab * H + c0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc = fmaf(J.w[c0 + e], fmaxf(__uint_as_float(v[e]), 0.f), acc);
+          }
+        } else {
+          uint32_t v[16];
+          tmem_ld16(t_lane + ab * H, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) acc = fmaf(J.w[e], fmaxf(__uint_as_float(v[e]), 0.f), acc);
+        }
+        if (DT == DT_E4M3) acc *= J.qsc * ksc;
+        cj[c] = valid ? float_key(acc) : 0u;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty + ab);
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(cand_full + cb);
+    }
+  } else {
+    // ------------------------------------------------------------ selector
+    const int stid = SelGrp::tid();
+    for (int64_t j = 0; j < njobs; ++j) {
+      const int slot = static_cast<int>(j % kTokJobs);
+      const int cb = static_cast<int>(j & 1);
+      if (stid == 0) *sel_ok = mbar_wait(cand_full + cb, static_cast<uint32_t>((j >> 1) & 1), abort_flag) ? 1 : 0;
+      SelGrp::sync();
+      if (!*sel_ok) break;
+      const TokJob& J = jobs[slot];
+      const uint32_t* cj = cand + cb * p.max_cand;
+      const int ncand = J.ntiles * kTokTileM;
+      int32_t* oi = p.out_idx + J.row * p.top_k;
+      float* os = p.out_score ? p.out_score + J.row * p.top_k : nullptr;
+      auto key_at = [&](int i) { return cj[i]; };
+      auto emit = [&](uint32_t slot_out, int i, uint32_t key) {
+        oi[slot_out] = J.blk[i / p.B] * p.B + i % p.B;
+        if (os) os[slot_out] = key_float(key);
+      };
+      const uint32_t n_valid = block_count_valid<decltype(key_at), SelGrp>(key_at, ncand, *sel);
+      if (n_valid <= static_cast<uint32_t>(p.top_k)) {
+        block_emit_all<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, emit, *sel);
+        for (int i = n_valid + stid; i < p.top_k; i += SelGrp::size()) {
+          oi[i] = -1;
+          if (os) os[i] = -__int_as_float(0x7f800000);
+        }
+      } else {
+        block_radix_topk<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, static_cast<uint32_t>(p.top_k),
+                                                                   emit, *sel);
+      }
+      SelGrp::sync();
+      if (stid == 0) {
+        mbar_arrive(cand_empty + cb);
+        mbar_arrive(job_empty + slot);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTokAcc * H < 32 ? 32 : kTokAcc * H);
+  }
+}
+
+inline size_t token_smem_bytes(int row_bytes, int H, int stages, int max_cand) {
+  return 1024 + 2 * static_cast<size_t>(H) * row_bytes + static_cast<size_t>(stages) * kTokTileM * row_bytes +
+         2 * static_cast<size_t>(max_cand) * 4 + kTokJobs * sizeof(TokJob) + sizeof(SelectSmem) + 8 +
+         8 * (2 * stages + 4 + 2 * kTokAcc + 2 * kTokJobs + 4 + 1) + 16;
+}
+
+}  // namespace hisa
