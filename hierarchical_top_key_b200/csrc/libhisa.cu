@@ -214,7 +214,7 @@ hisa_status dense_tc_h(const hisa_shape* s, const CUtensorMap& qm, const CUtenso
 // Score rows of one chunk: out[(b*Q+t) - row0][s] for the visible keys.
 hisa_status score_rows(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* keys,
                        const float* ksc, const int32_t* nvis, int block_div, int L, const RowChunk& c, float* out,
-                       int64_t ld, cudaStream_t st) {
+                       int64_t ld, cudaStream_t st, uint32_t* minmax = nullptr) {
   if (dense_tc_ok(s)) {
     CUtensorMap qm, km;
     hisa_status e = tensor_map_2d(&qm, q, s->dtype, static_cast<uint64_t>(rows_of(s)) * s->heads, s->head_dim, kDenseN);
@@ -227,7 +227,7 @@ hisa_status score_rows(const hisa_shape* s, const void* q, const float* qsc, con
     p.groups_per_seq = static_cast<int>(ceil_div(s->num_queries, p.G));
     p.block_div = block_div;
     p.gg0 = c.gg0; p.ngroups = c.ngroups; p.row0 = c.row0;
-    p.w = w; p.n_visible = nvis; p.q_scale = qsc; p.k_scale = ksc; p.out = out; p.ld = ld;
+    p.w = w; p.n_visible = nvis; p.q_scale = qsc; p.k_scale = ksc; p.out = out; p.ld = ld; p.minmax = minmax;
     return s->dtype == HISA_BF16 ? dense_tc_h<DT_BF16>(s, qm, km, p, st) : dense_tc_h<DT_E4M3>(s, qm, km, p, st);
   }
   switch (s->dtype) {
@@ -269,7 +269,7 @@ bool token_tc_ok(const hisa_shape* s) {
   return (s->dtype == HISA_BF16 || s->dtype == HISA_E4M3) && (rb == 128 || rb == 256) &&
          (s->heads == 16 || s->heads == 32 || s->heads == 64) &&
          (s->block_size == 16 || s->block_size == 32 || s->block_size == 64 || s->block_size == 128) &&
-         s->top_m <= kTokMaxBlocks;
+         s->top_m <= kTokMaxBlocks && num_blocks(s) <= 32 * kTokMaxBitmapWords;
 }
 
 template <int DT, int H>
@@ -364,7 +364,7 @@ hisa_status hisa_workspace_size(int32_t op, const hisa_shape* s, size_t* bytes) 
   hisa_status e = check_shape(s, op != HISA_OP_FLAT_TOPK);
   if (e != HISA_OK) return e;
   switch (op) {
-    case HISA_OP_FLAT_TOPK: *bytes = static_cast<size_t>(rows_of(s) * pad4(s->num_keys) * 4); return HISA_OK;
+    case HISA_OP_FLAT_TOPK: *bytes = static_cast<size_t>(rows_of(s) * (pad4(s->num_keys) * 4 + 8)); return HISA_OK;
     case HISA_OP_BLOCK_SCORE_TOPM: *bytes = static_cast<size_t>(rows_of(s) * pad4(num_blocks(s)) * 4); return HISA_OK;
     case HISA_OP_TOKEN_SCORE_TOPK: *bytes = 0; return HISA_OK;
   }
@@ -513,16 +513,29 @@ hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale, const flo
   const int64_t ld = pad4(s->num_keys);
   const int64_t rows = rows_of(s);
   if (!workspace || !aligned16(workspace)) return fail(HISA_ERR_WORKSPACE, "workspace must be non-NULL, 16-byte aligned");
+  // workspace: score rows [chunk][ld] fp32, then (min, max) ordering keys per row
+  const int64_t row_bytes = ld * 4 + 8;
   std::vector<RowChunk> chunks;
-  e = plan_chunks(s, dense_group(s), std::min<int64_t>(rows, static_cast<int64_t>(ws_bytes / (ld * 4))), chunks);
+  e = plan_chunks(s, dense_group(s), std::min<int64_t>(rows, static_cast<int64_t>(ws_bytes / row_bytes)), chunks);
   if (e != HISA_OK) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
+  int64_t max_rows = 0;
+  for (const RowChunk& c : chunks) max_rows = std::max(max_rows, c.nrows);
+  uint32_t* minmax = reinterpret_cast<uint32_t*>(ws + max_rows * ld);
+  const bool fused_range = dense_tc_ok(s);
   for (const RowChunk& c : chunks) {
-    e = score_rows(s, q, q_scale, w, k, k_scale, n_visible, 0, s->num_keys, c, ws, ld, st);
+    if (fused_range) {
+      init_minmax_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(c.nrows, 256), 1024)), 256, 0, st>>>(
+          minmax, c.nrows);
+      e = launch_check("init_minmax_kernel");
+      if (e != HISA_OK) return e;
+    }
+    e = score_rows(s, q, q_scale, w, k, k_scale, n_visible, 0, s->num_keys, c, ws, ld, st,
+                   fused_range ? minmax : nullptr);
     if (e != HISA_OK) return e;
-    flat_select_kernel<<<static_cast<unsigned>(c.nrows), 512, 0, st>>>(ws, ld, n_visible, c.row0, s->num_keys,
-                                                                       s->top_k, topk_idx, topk_score);
+    flat_select_kernel<<<static_cast<unsigned>(c.nrows), 512, 0, st>>>(
+        ws, ld, fused_range ? minmax : nullptr, n_visible, c.row0, s->num_keys, s->top_k, topk_idx, topk_score);
     e = launch_check("flat_select_kernel");
     if (e != HISA_OK) return e;
   }

@@ -206,15 +206,10 @@ __global__ void __launch_bounds__(kSimtThreads) token_stage_simt_kernel(
     oi[slot] = static_cast<int32_t>(key_of(i));
     if (os) os[slot] = key_float(key);
   };
-  const uint32_t n_valid = block_count_valid(key_at, ncand, sel);
-  if (n_valid <= static_cast<uint32_t>(top_k)) {
-    block_emit_all(key_at, ncand, emit, sel);
-    for (int i = n_valid + threadIdx.x; i < top_k; i += blockDim.x) {
-      oi[i] = -1;
-      if (os) os[i] = -__int_as_float(0x7f800000);
-    }
-  } else {
-    block_radix_topk(key_at, ncand, static_cast<uint32_t>(top_k), emit, sel);
+  const uint32_t nv = block_topk(key_at, ncand, static_cast<uint32_t>(top_k), emit, sel);
+  for (int i = static_cast<int>(nv) + threadIdx.x; i < top_k; i += blockDim.x) {
+    oi[i] = -1;
+    if (os) os[i] = -__int_as_float(0x7f800000);
   }
 }
 

@@ -47,6 +47,7 @@ struct DenseParams {
   const float* k_scale;
   float* out;
   int64_t ld;
+  uint32_t* minmax;         // nullable: per output row, (min, max) ordering key written
 };
 
 struct DenseUnit {
@@ -133,11 +134,12 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int64_t kt = 0;
+      int st = 0;
+      uint32_t kph = 0;
       int un = 0;
-      int64_t last_k[8];
-      for (int s = 0; s < 8; ++s) last_k[s] = -1;
-      int last_q[2] = {-1, -1};
+      int8_t last_ph[8];
+      for (int s = 0; s < 8; ++s) last_ph[s] = -1;
+      int8_t last_qph[2] = {-1, -1};
       bool ok = true;
       for (int64_t r = 0; ok && r * gridDim.x < total_units; ++r) {
         const int64_t u = dense_unit_index(r);
@@ -150,23 +152,23 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
         const int qrow = (U.b * p.Q + U.t0) * p.H;
         for (int pn = 0; pn < panels; ++pn)
           tma_load_2d(q_buf + qb * q_bytes + pn * (kDenseN * 128), &qmap, q_full + qb, pn * panel_elems, qrow);
-        last_q[qb] = un;
-        for (int i = 0; i < U.ntiles; ++i, ++kt) {
-          const int st = static_cast<int>(kt % p.stages);
-          if (!(ok = mbar_wait(k_empty + st, static_cast<uint32_t>(((kt / p.stages) & 1) ^ 1), abort_flag))) break;
+        last_qph[qb] = static_cast<int8_t>((un / p.q_bufs) & 1);
+        for (int i = 0; i < U.ntiles; ++i) {
+          if (!(ok = mbar_wait(k_empty + st, kph ^ 1, abort_flag))) break;
           mbar_arrive_expect_tx(k_full + st, k_bytes);
           const int krow = U.b * p.L + (U.tile0 + i) * kDenseTileM;
           for (int pn = 0; pn < panels; ++pn)
             tma_load_2d(k_buf + st * k_bytes + pn * (kDenseTileM * 128), &kmap, k_full + st, pn * panel_elems, krow);
-          last_k[st] = kt;
+          last_ph[st] = static_cast<int8_t>(kph);
+          if (++st == p.stages) { st = 0; kph ^= 1; }
         }
         ++un;
       }
       if (!ok) {   // drain the copies this thread issued before leaving
         for (int s = 0; s < p.stages; ++s)
-          if (last_k[s] >= 0) mbar_drain(k_full + s, static_cast<uint32_t>((last_k[s] / p.stages) & 1));
+          if (last_ph[s] >= 0) mbar_drain(k_full + s, static_cast<uint32_t>(last_ph[s]));
         for (int i = 0; i < 2; ++i)
-          if (last_q[i] >= 0) mbar_drain(q_full + i, static_cast<uint32_t>((last_q[i] / p.q_bufs) & 1));
+          if (last_qph[i] >= 0) mbar_drain(q_full + i, static_cast<uint32_t>(last_qph[i]));
       }
     }
   } else if (warp == 1) {
@@ -174,7 +176,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc(kDenseTileM, kDenseN, DT == DT_BF16 ? 1u : 0u);
       const int ksteps = row_bytes / 32;       // 32 bytes of K per MMA (16 bf16 / 32 e4m3)
-      int64_t kt = 0, tc = 0;
+      int st = 0, ab = 0;
+      uint32_t kph = 0, aph = 0;
       int un = 0;
       bool ok = true;
       for (int64_t r = 0; ok && r * gridDim.x < total_units; ++r) {
@@ -186,11 +189,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
         if (!(ok = mbar_wait(q_full + qb, (un / p.q_bufs) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(q_buf + qb * q_bytes);
-        for (int i = 0; i < U.ntiles; ++i, ++kt, ++tc) {
-          const int st = static_cast<int>(kt % p.stages);
-          const int ab = static_cast<int>(tc & 1);
-          if (!(ok = mbar_wait(acc_empty + ab, static_cast<uint32_t>(((tc >> 1) & 1) ^ 1), abort_flag))) break;
-          if (!(ok = mbar_wait(k_full + st, static_cast<uint32_t>((kt / p.stages) & 1), abort_flag))) break;
+        for (int i = 0; i < U.ntiles; ++i) {
+          if (!(ok = mbar_wait(acc_empty + ab, aph ^ 1, abort_flag))) break;
+          if (!(ok = mbar_wait(k_full + st, kph, abort_flag))) break;
           tc_fence_after();
           const uint32_t k_addr = smem_u32(k_buf + st * k_bytes);
           const uint32_t d_tmem = tmem_base + ab * kDenseN;
@@ -202,6 +203,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
           }
           mma_commit(k_empty + st);
           mma_commit(acc_full + ab);
+          if (++st == p.stages) { st = 0; kph ^= 1; }
+          ab ^= 1;
+          aph ^= ab == 0 ? 1u : 0u;
         }
         if (ok) mma_commit(q_empty + qb);
         ++un;
@@ -240,6 +244,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
         qsc_w[jq] = (DT == DT_E4M3 && j < U.nq) ? __ldg(p.q_scale + qrow0 + j) : 1.f;
       }
       __syncwarp();
+      uint32_t kmin[QPT], kmax[QPT];
+#pragma unroll
+      for (int jq = 0; jq < QPT; ++jq) { kmin[jq] = 0xFFFFFFFFu; kmax[jq] = 0u; }
       for (int i = 0; i < U.ntiles; ++i, ++tc) {
         const int ab = static_cast<int>(tc & 1);
         int okl = 1;
@@ -251,7 +258,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
         float ksc = 1.f;
         if (DT == DT_E4M3 && s < p.L) ksc = __ldg(p.k_scale + static_cast<int64_t>(U.b) * p.L + s);
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * kDenseN;
-#pragma unroll 1
+#pragma unroll
         for (int jq = 0; jq < QPT; ++jq) {
           const int j = half * QPT + jq;
           const float* wq = w_w + jq * H;
@@ -275,11 +282,26 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
           if (s < vis_w[jq]) {
             if (DT == DT_E4M3) acc *= qsc_w[jq] * ksc;
             p.out[(qrow0 + j - p.row0) * p.ld + s] = acc;
+            const uint32_t key = float_key(acc);
+            kmin[jq] = min(kmin[jq], key);
+            kmax[jq] = max(kmax[jq], key);
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty + ab);
+      }
+      if (ok && p.minmax != nullptr) {
+#pragma unroll
+        for (int jq = 0; jq < QPT; ++jq) {
+          const uint32_t lo = __reduce_min_sync(0xffffffffu, kmin[jq]);
+          const uint32_t hi = __reduce_max_sync(0xffffffffu, kmax[jq]);
+          const int j = half * QPT + jq;
+          if (lane == 0 && j < U.nq && hi != 0u) {
+            atomicMin(p.minmax + 2 * (qrow0 + j - p.row0), lo);
+            atomicMax(p.minmax + 2 * (qrow0 + j - p.row0) + 1, hi);
+          }
+        }
       }
     }
   }

@@ -28,15 +28,18 @@ struct WarpRange {
   __device__ __forceinline__ static void sync() { asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(N) : "memory"); }
 };
 
+constexpr int kDigitBits = 11;
+constexpr int kDigitBins = 1 << kDigitBits;
+
 struct SelectSmem {
-  uint32_t hist[256];
+  uint32_t hist[kDigitBins];
   uint32_t warp_cnt[32];
+  uint32_t kmin, kmax, n_valid;
   uint32_t digit;
   uint32_t above;
-  uint32_t at_digit;       // histogram count of the chosen digit (last pass: elements equal to T)
-  uint32_t n_gt_slots;     // running slot counter for key > T
+  uint32_t at_digit;       // histogram count of the chosen digit
+  uint32_t n_slots;        // running slot counter for unordered emission
   uint32_t eq_base;        // equal-to-T elements seen in earlier chunks
-  uint32_t n_valid;
 };
 
 // Block-wide exclusive prefix of a 0/1 flag over the threads (in thread
@@ -58,146 +61,207 @@ __device__ __forceinline__ uint32_t block_flag_prefix(bool flag, SelectSmem& sm,
   return off + __popc(ball & ((1u << lane) - 1u));
 }
 
-// Count of keys != 0 among positions [0, n).
-template <class KeyAt, class Grp = CtaGroup>
-__device__ uint32_t block_count_valid(KeyAt key_at, int n, SelectSmem& sm) {
-  uint32_t c = 0;
-  for (int i = Grp::tid(); i < n; i += Grp::size()) c += key_at(i) != 0u;
-  c = __reduce_add_sync(0xffffffffu, c);
-  if (Grp::tid() == 0) sm.n_valid = 0;
+// Emit every key >= T (and != 0) into slots taken from a shared counter, in
+// no particular order.  One warp-aggregated atomic per warp and chunk.
+template <class KeyAt, class Emit, class Grp>
+__device__ void emit_at_least(KeyAt key_at, int n, uint32_t T, Emit emit, SelectSmem& sm) {
+  if (Grp::tid() == 0) sm.n_slots = 0;
   Grp::sync();
-  if ((Grp::tid() & 31) == 0) atomicAdd(&sm.n_valid, c);
+  const int lane = Grp::tid() & 31;
+  for (int base = 0; base < n; base += Grp::size()) {
+    const int i = base + Grp::tid();
+    const uint32_t key = i < n ? key_at(i) : 0u;
+    const bool take = key >= T && key != 0u;
+    const uint32_t ball = __ballot_sync(0xffffffffu, take);
+    uint32_t slot0 = 0;
+    if (lane == 0 && ball) slot0 = atomicAdd(&sm.n_slots, __popc(ball));
+    slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+    if (take) emit(slot0 + __popc(ball & ((1u << lane) - 1u)), i, key);
+  }
   Grp::sync();
-  const uint32_t v = sm.n_valid;
-  Grp::sync();
-  return v;
 }
 
-// Emit(slot, position, key) for the k largest keys among [0, n).  Requires
-// blockDim.x to be a multiple of 32 (<= 1024) and more than k valid keys.
-// Returns nothing; every slot 0..k-1 is emitted exactly once.
+// Top-k of the keys at positions [0, n) (key 0 = absent): calls
+// Emit(slot, position, key) exactly once for each slot 0..min(k, valid)-1 and
+// returns the number of valid keys.  Ties at the k-th place go to the lower
+// position.  Radix select on the bits that vary between the smallest and the
+// largest key, 11 bits per pass; spreading the digits over that range keeps
+// histogram atomics on distinct bins.
+// As block_topk below, with the range and count of the valid keys given.
 template <class KeyAt, class Emit, class Grp = CtaGroup>
-__device__ void block_radix_topk(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem& sm) {
-  uint32_t prefix = 0, remaining = k;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
-    for (int i = Grp::tid(); i < 256; i += Grp::size()) sm.hist[i] = 0;
+__device__ uint32_t block_topk_range(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem& sm, uint32_t kmin,
+                                     uint32_t kmax, uint32_t n_valid);
+
+template <class KeyAt, class Emit, class Grp = CtaGroup>
+__device__ uint32_t block_topk(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem& sm) {
+  const int lane = Grp::tid() & 31;
+  // ---- range and count of the valid keys
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u, cnt = 0;
+  for (int i = Grp::tid(); i < n; i += Grp::size()) {
+    const uint32_t key = key_at(i);
+    if (key != 0u) { lo = min(lo, key); hi = max(hi, key); ++cnt; }
+  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if (Grp::tid() == 0) { sm.kmin = 0xFFFFFFFFu; sm.kmax = 0u; sm.n_valid = 0u; }
+  Grp::sync();
+  if (lane == 0) { atomicMin(&sm.kmin, lo); atomicMax(&sm.kmax, hi); atomicAdd(&sm.n_valid, cnt); }
+  Grp::sync();
+  const uint32_t kmin = sm.kmin, kmax = sm.kmax, n_valid = sm.n_valid;
+  Grp::sync();
+  return block_topk_range<KeyAt, Emit, Grp>(key_at, n, k, emit, sm, kmin, kmax, n_valid);
+}
+
+template <class KeyAt, class Emit, class Grp>
+__device__ uint32_t block_topk_range(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem& sm, uint32_t kmin,
+                                     uint32_t kmax, uint32_t n_valid) {
+  const int lane = Grp::tid() & 31;
+  if (n_valid <= k) {
+    emit_at_least<KeyAt, Emit, Grp>(key_at, n, 1u, emit, sm);
+    return n_valid;
+  }
+  // ---- digits below the common prefix of kmin and kmax
+  int shift = kmin == kmax ? 0 : 32 - __clz(kmin ^ kmax);
+  uint32_t prefix = kmax & (shift == 32 ? 0u : ~((1u << shift) - 1u));
+  uint32_t remaining = k, n_eq = n_valid;
+  while (shift > 0) {
+    const int dig = min(kDigitBits, shift);
+    shift -= dig;
+    const int nbins = 1 << dig;
+    const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
+    for (int i = Grp::tid(); i < nbins; i += Grp::size()) sm.hist[i] = 0;
     Grp::sync();
-    for (int i = Grp::tid(); i < n; i += Grp::size()) {
-      const uint32_t key = key_at(i);
-      if (key != 0u && ((key ^ prefix) & hi_mask) == 0u) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
+    for (int base = 0; base < n; base += Grp::size()) {
+      const int i = base + Grp::tid();
+      const uint32_t key = i < n ? key_at(i) : 0u;
+      const bool act = key != 0u && (static_cast<uint64_t>(key ^ prefix) >> (shift + dig)) == 0;
+      if (act) atomicAdd(&sm.hist[(key >> shift) & dmask], 1u);
     }
     Grp::sync();
-    if (Grp::tid() < 32) {
-      // lane l holds bins 255-8l .. 248-8l (descending), suffix sums across lanes
-      const int lane = Grp::tid();
-      uint32_t h[8], t = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { h[j] = sm.hist[255 - 8 * lane - j]; t += h[j]; }
+    {
+      // block-parallel search from the top bin: thread i owns bins
+      // [nbins-1-i*per, nbins-(i+1)*per]; exclusive prefix of the per-thread
+      // sums across the group finds the bin holding the `remaining`-th key
+      const int nt = Grp::size();
+      const int per = nbins >= nt ? nbins / nt : 1;
+      const int top = nbins - 1 - Grp::tid() * per;
+      uint32_t t = 0;
+      for (int j = 0; j < per; ++j)
+        if (top - j >= 0) t += sm.hist[top - j];
       uint32_t incl = t;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += o;
       }
+      if (lane == 31) sm.warp_cnt[Grp::tid() >> 5] = incl;
+      Grp::sync();
+      uint32_t woff = 0;
+      for (int wi = 0; wi < (Grp::tid() >> 5); ++wi) woff += sm.warp_cnt[wi];
+      incl += woff;
       const uint32_t excl = incl - t;
-      const uint32_t ball = __ballot_sync(0xffffffffu, incl >= remaining);
-      const int src = __ffs(ball) - 1;
-      if (lane == src) {
+      if (t > 0 && excl < remaining && incl >= remaining) {
         uint32_t c = excl;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (c + h[j] >= remaining) { sm.digit = 255 - 8 * lane - j; sm.above = c; sm.at_digit = h[j]; break; }
-          c += h[j];
+        for (int j = 0; j < per; ++j) {
+          const uint32_t h = sm.hist[top - j];
+          if (c + h >= remaining) { sm.digit = top - j; sm.above = c; sm.at_digit = h; break; }
+          c += h;
         }
       }
     }
     Grp::sync();
     prefix |= sm.digit << shift;
     remaining -= sm.above;
+    n_eq = sm.at_digit;
     Grp::sync();
+    if (n_eq == remaining) {
+      // the whole boundary bin is taken: every key >= prefix (lower bits 0) is in
+      emit_at_least<KeyAt, Emit, Grp>(key_at, n, prefix, emit, sm);
+      return n_valid;
+    }
   }
-  // prefix is the k-th largest key; `remaining` elements equal to it are taken
+  // prefix == T, the k-th largest key; `remaining` of the n_eq keys equal to T
+  // are taken, the lowest positions first
   const uint32_t T = prefix, need_eq = remaining, n_gt = k - remaining;
-  const uint32_t n_eq = sm.at_digit;
-  if (Grp::tid() == 0) { sm.n_gt_slots = 0; sm.eq_base = 0; }
+  if (Grp::tid() == 0) { sm.n_slots = 0; sm.eq_base = 0; }
   Grp::sync();
-  if (need_eq == n_eq) {
-    // no tie is cut at the boundary: every key >= T is taken, in any order
-    for (int base = 0; base < n; base += Grp::size()) {
-      const int i = base + Grp::tid();
-      const uint32_t key = i < n ? key_at(i) : 0u;
-      const bool take = key >= T && key != 0u;
-      const uint32_t ball = __ballot_sync(0xffffffffu, take);
-      uint32_t base_slot = 0;
-      if ((Grp::tid() & 31) == 0 && ball) base_slot = atomicAdd(&sm.n_gt_slots, __popc(ball));
-      base_slot = __shfl_sync(0xffffffffu, base_slot, 0);
-      if (take) emit(base_slot + __popc(ball & ((1u << (Grp::tid() & 31)) - 1u)), i, key);
-    }
-    Grp::sync();
-    return;
-  }
   for (int base = 0; base < n; base += Grp::size()) {
     const int i = base + Grp::tid();
     const uint32_t key = i < n ? key_at(i) : 0u;
-    if (key > T) {
-      const uint32_t slot = atomicAdd(&sm.n_gt_slots, 1u);
-      emit(slot, i, key);
-    }
+    const bool gt = key > T;
+    const uint32_t ball = __ballot_sync(0xffffffffu, gt);
+    uint32_t slot0 = 0;
+    if (lane == 0 && ball) slot0 = atomicAdd(&sm.n_slots, __popc(ball));
+    slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+    if (gt) emit(slot0 + __popc(ball & ((1u << lane) - 1u)), i, key);
     uint32_t tot;
-    const uint32_t rank = block_flag_prefix<Grp>(key == T && key != 0u, sm, &tot);
+    const uint32_t rank = block_flag_prefix<Grp>(key == T, sm, &tot);
     const uint32_t r = sm.eq_base + rank;
-    if (key == T && key != 0u && r < need_eq) emit(n_gt + r, i, key);
+    if (key == T && r < need_eq) emit(n_gt + r, i, key);
     Grp::sync();
     if (Grp::tid() == 0) sm.eq_base += tot;
     Grp::sync();
+    if (sm.eq_base >= need_eq && base + Grp::size() < n) {
+      // every tied key needed is placed; the rest only contributes keys > T
+      for (int b2 = base + Grp::size(); b2 < n; b2 += Grp::size()) {
+        const int i2 = b2 + Grp::tid();
+        const uint32_t key2 = i2 < n ? key_at(i2) : 0u;
+        const bool gt2 = key2 > T;
+        const uint32_t ball2 = __ballot_sync(0xffffffffu, gt2);
+        uint32_t s2 = 0;
+        if (lane == 0 && ball2) s2 = atomicAdd(&sm.n_slots, __popc(ball2));
+        s2 = __shfl_sync(0xffffffffu, s2, 0);
+        if (gt2) emit(s2 + __popc(ball2 & ((1u << lane) - 1u)), i2, key2);
+      }
+      break;
+    }
   }
-}
-
-// Emit every valid key (key != 0) among [0, n) in position order into slots
-// 0..n_valid-1 (used when there are no more than k of them).
-template <class KeyAt, class Emit, class Grp = CtaGroup>
-__device__ void block_emit_all(KeyAt key_at, int n, Emit emit, SelectSmem& sm) {
-  if (Grp::tid() == 0) sm.eq_base = 0;
   Grp::sync();
-  for (int base = 0; base < n; base += Grp::size()) {
-    const int i = base + Grp::tid();
-    const uint32_t key = i < n ? key_at(i) : 0u;
-    uint32_t tot;
-    const uint32_t rank = block_flag_prefix<Grp>(key != 0u, sm, &tot);
-    if (key != 0u) emit(sm.eq_base + rank, i, key);
-    Grp::sync();
-    if (Grp::tid() == 0) sm.eq_base += tot;
-    Grp::sync();
-  }
+  (void)n_eq;
+  return n_valid;
 }
 
 // ---------------------------------------------------------------- row kernels
 
 // Flat DSA top-k over fp32 score rows: row r holds scores of keys 0..n_r-1.
+// `minmax` (nullable) holds, per row, the smallest and largest ordering key
+// the scoring kernel wrote, which saves the range pass over the row.
 __global__ void __launch_bounds__(512) flat_select_kernel(
-    const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_visible,
-    int64_t row0, int L, int top_k, int32_t* __restrict__ out_idx, float* __restrict__ out_score) {
+    const float* __restrict__ scores, int64_t ld, const uint32_t* __restrict__ minmax,
+    const int32_t* __restrict__ n_visible, int64_t row0, int L, int top_k, int32_t* __restrict__ out_idx,
+    float* __restrict__ out_score) {
   __shared__ SelectSmem sm;
   const int64_t r = row0 + blockIdx.x;
   const float* row = scores + static_cast<int64_t>(blockIdx.x) * ld;
   const int n = max(0, min(n_visible[r], L));
   int32_t* oi = out_idx + r * top_k;
   float* os = out_score ? out_score + r * top_k : nullptr;
-  auto key_at = [&](int i) { return float_key(row[i]); };
   auto emit = [&](uint32_t slot, int i, uint32_t key) {
     oi[slot] = i;
     if (os) os[slot] = key_float(key);
   };
-  if (n <= top_k) {
-    for (int i = threadIdx.x; i < top_k; i += blockDim.x) {
-      oi[i] = i < n ? i : -1;
-      if (os) os[i] = i < n ? row[i] : -__int_as_float(0x7f800000);
-    }
-    return;
+  auto key_at = [&](int i) { return float_key(row[i]); };
+  uint32_t nv;
+  if (minmax != nullptr && n > 0) {
+    nv = block_topk_range(key_at, n, static_cast<uint32_t>(top_k), emit, sm, minmax[2 * blockIdx.x],
+                          minmax[2 * blockIdx.x + 1], static_cast<uint32_t>(n));
+  } else {
+    nv = block_topk(key_at, n, static_cast<uint32_t>(top_k), emit, sm);
   }
-  block_radix_topk(key_at, n, static_cast<uint32_t>(top_k), emit, sm);
+  for (int i = static_cast<int>(nv) + threadIdx.x; i < top_k; i += blockDim.x) {
+    oi[i] = -1;
+    if (os) os[i] = -__int_as_float(0x7f800000);
+  }
+}
+
+// (smallest, largest) ordering-key pairs start empty.
+__global__ void init_minmax_kernel(uint32_t* minmax, int64_t rows) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < rows;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    minmax[2 * i] = 0xFFFFFFFFu;
+    minmax[2 * i + 1] = 0u;
+  }
 }
 
 // HISA block selection over fp32 block-score rows: row r holds scores of the
@@ -219,7 +283,7 @@ __global__ void __launch_bounds__(512) block_select_kernel(
   if (top_m == 1) return;
   auto key_at = [&](int i) { return float_key(row[i]); };
   auto emit = [&](uint32_t slot, int i, uint32_t) { oi[1 + slot] = i; };
-  block_radix_topk(key_at, c, static_cast<uint32_t>(top_m - 1), emit, sm);
+  block_topk(key_at, c, static_cast<uint32_t>(top_m - 1), emit, sm);
 }
 
 }  // namespace hisa

@@ -10,10 +10,11 @@
 // Persistent, warp-specialised CTA (one per SM), queries processed as a
 // pipeline of jobs:
 //   warp 0       job set-up (whole warp: read, filter, dedupe and sort the
-//                block list; stage w[t]) then TMA issue (lane 0)
+//                block list; stage w[t]), running up to four jobs ahead
 //   warp 1       TMEM owner and MMA issuer
-//   warps 2..5   scorer: TMEM -> weighted ReLU sum -> candidate keys in smem
-//   warps 6..13  selector: radix top-k over the candidate keys, emit indices
+//   warp 2       TMA issuer: q[t] and one tile load per retained block
+//   warps 3..6   scorer: TMEM -> weighted ReLU sum -> candidate keys in smem
+//   warps 7..14  selector: radix top-k over the candidate keys, emit indices
 // Rings: job slots (4), q buffers (2), key stages, TMEM accumulators (4 x H
 // columns), candidate buffers (2).  Blocks are sorted ascending so candidate
 // position order is key order, which makes ties resolve to the lower key.
@@ -29,9 +30,11 @@ constexpr int kTokJobs = 4;
 constexpr int kTokAcc = 4;
 constexpr int kTokScorerWarps = 4;
 constexpr int kTokSelectWarps = 8;
-constexpr int kTokSelectBase = 32 * (2 + kTokScorerWarps);
+constexpr int kTokScorerBase = 3;                 // first scorer warp
+constexpr int kTokSelectBase = 32 * (kTokScorerBase + kTokScorerWarps);
 constexpr int kTokThreads = kTokSelectBase + 32 * kTokSelectWarps;
-constexpr int kTokMaxBlocks = 256;
+constexpr int kTokMaxBlocks = 256;                // top_m limit
+constexpr int kTokMaxBitmapWords = 256;           // blocks per sequence limit / 32
 
 struct TokenParams {
   int64_t rows;            // batch * Q
@@ -48,11 +51,11 @@ struct TokenParams {
   float* out_score;
 };
 
-struct TokJob {
+struct alignas(16) TokJob {
   int64_t row;
   int b, n, nblk, ntiles;
   float qsc;
-  float w[64];
+  alignas(16) float w[64];
   int blk[kTokMaxBlocks];
 };
 
@@ -79,7 +82,8 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
   uint32_t* cand = reinterpret_cast<uint32_t*>(k_buf + p.stages * k_bytes);   // [2][max_cand]
   TokJob* jobs = reinterpret_cast<TokJob*>(cand + 2 * p.max_cand);            // [kTokJobs]
   SelectSmem* sel = reinterpret_cast<SelectSmem*>(jobs + kTokJobs);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uintptr_t>(sel + 1) + 7 & ~uintptr_t(7));
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(sel + 1);                     // [kTokMaxBitmapWords]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uintptr_t>(bitmap + kTokMaxBitmapWords) + 7 & ~uintptr_t(7));
   uint64_t* k_full = bars;
   uint64_t* k_empty = k_full + p.stages;
   uint64_t* q_full = k_empty + p.stages;          // [2]
@@ -117,11 +121,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
   const int64_t njobs = p.rows > blockIdx.x ? (p.rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ job set-up + TMA
-    int64_t kt = 0;
-    int64_t last_k[8];
-    for (int s = 0; s < 8; ++s) last_k[s] = -1;
-    int64_t last_q[2] = {-1, -1};
+    // ------------------------------------------------------------ job set-up
     bool ok = true;
     for (int64_t j = 0; j < njobs; ++j) {
       const int slot = static_cast<int>(j % kTokJobs);
@@ -131,105 +131,117 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
       TokJob& J = jobs[slot];
       const int64_t row = tok_job_row(p, j);
       const int b = static_cast<int>(row / p.Q);
-      const int n = max(0, min(__ldg(p.n_visible + row), p.L));
-      // raw block list -> J.blk (scratch), then rank-sort the valid, distinct entries
-      for (int i = lane; i < p.top_m; i += 32) J.blk[i] = __ldg(p.block_idx + row * p.top_m + i);
-      __syncwarp();
-      // keep = valid and not a repeat of an earlier entry; rank = number of
-      // kept values below it.  O(top_m) work per entry, ballots carry the keep set.
+      // every global read of the job at once: visibility, block list, weights
+      const int n_raw = __ldg(p.n_visible + row);
       constexpr int KW = kTokMaxBlocks / 32;
-      int mine[KW];
-      uint32_t keepmask[KW];
+      int x[KW];
 #pragma unroll
       for (int k = 0; k < KW; ++k) {
         const int i = lane + 32 * k;
-        int x = -1;
-        bool keep = false;
-        if (32 * k < p.top_m && i < p.top_m) {
-          x = J.blk[i];
-          keep = x >= 0 && x < p.nb && x * p.B < n;
-          for (int i2 = 0; keep && i2 < i; ++i2) keep = J.blk[i2] != x;
-        }
-        mine[k] = keep ? x : -1;
-        keepmask[k] = __ballot_sync(0xffffffffu, keep);
+        x[k] = (32 * k < p.top_m && i < p.top_m) ? __ldg(p.block_idx + row * p.top_m + i) : -1;
       }
-      int rank[KW];
-      int cnt = 0;
-#pragma unroll
-      for (int k = 0; k < KW; ++k) {
-        cnt += __popc(keepmask[k]);
-        rank[k] = 0;
-        if (mine[k] >= 0) {
-          int r = 0;
-#pragma unroll
-          for (int k2 = 0; k2 < KW; ++k2) {
-            uint32_t m2 = keepmask[k2];
-            while (m2) {
-              const int bit = __ffs(m2) - 1;
-              m2 &= m2 - 1;
-              r += J.blk[32 * k2 + bit] < mine[k];
-            }
-          }
-          rank[k] = r;
-        }
-      }
+      const float w0 = lane < p.H ? __ldg(p.w + row * p.H + lane) : 0.f;
+      const float w1 = lane + 32 < p.H ? __ldg(p.w + row * p.H + lane + 32) : 0.f;
+      const float qsc = (DT == DT_E4M3 && lane == 0) ? __ldg(p.q_scale + row) : 1.f;
+      const int n = max(0, min(n_raw, p.L));
+      // retained blocks -> bitmap (repeats collapse, invalid entries dropped),
+      // then the set bits are compacted in ascending order
+      const int nvis_blocks = min(p.nb, (n + p.B - 1) / p.B);   // blocks holding a visible key
+      const int nwords = (nvis_blocks + 31) >> 5;
+      for (int wi = lane; wi < nwords; wi += 32) bitmap[wi] = 0u;
       __syncwarp();
 #pragma unroll
       for (int k = 0; k < KW; ++k)
-        if (mine[k] >= 0) J.blk[rank[k]] = mine[k];
-      for (int h = lane; h < 64; h += 32) J.w[h] = h < p.H ? __ldg(p.w + row * p.H + h) : 0.f;
+        if (x[k] >= 0 && x[k] < nvis_blocks) atomicOr(bitmap + (x[k] >> 5), 1u << (x[k] & 31));
+      __syncwarp();
+      const int wpl = (nwords + 31) >> 5;                        // words per lane, in order
+      int local = 0;
+      for (int i = 0; i < wpl; ++i) {
+        const int wi = lane * wpl + i;
+        if (wi < nwords) local += __popc(bitmap[wi]);
+      }
+      int incl = local;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const int cnt = __shfl_sync(0xffffffffu, incl, 31);
+      int pos = incl - local;
+      for (int i = 0; i < wpl; ++i) {
+        const int wi = lane * wpl + i;
+        if (wi >= nwords) break;
+        uint32_t bits = bitmap[wi];
+        while (bits) {
+          const int bit = __ffs(bits) - 1;
+          bits &= bits - 1;
+          J.blk[pos++] = (wi << 5) + bit;
+        }
+      }
+      J.w[lane] = w0;
+      J.w[lane + 32] = w1;
       if (lane == 0) {
         J.row = row;
         J.b = b;
         J.n = n;
         J.nblk = cnt;
         J.ntiles = (cnt * p.B + kTokTileM - 1) / kTokTileM;
-        J.qsc = DT == DT_E4M3 ? __ldg(p.q_scale + row) : 1.f;
+        J.qsc = qsc;
       }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(job_full + slot);
-        // q[t]
+      if (lane == 0) mbar_arrive(job_full + slot);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ TMA issue
+    if (lane == 0) {
+      int st = 0;
+      uint32_t kph = 0;
+      int8_t last_ph[8];
+      for (int i = 0; i < 8; ++i) last_ph[i] = -1;
+      int8_t last_qph[2] = {-1, -1};
+      bool ok = true;
+      for (int64_t j = 0; ok && j < njobs; ++j) {
+        const int slot = static_cast<int>(j % kTokJobs);
+        if (!(ok = mbar_wait(job_full + slot, static_cast<uint32_t>((j / kTokJobs) & 1), abort_flag))) break;
+        const TokJob& J = jobs[slot];
         const int qb = static_cast<int>(j & 1);
-        if ((ok = mbar_wait(q_empty + qb, static_cast<uint32_t>(((j >> 1) & 1) ^ 1), abort_flag))) {
-          mbar_arrive_expect_tx(q_full + qb, q_bytes);
-          for (int pn = 0; pn < panels; ++pn)
-            tma_load_2d(q_buf + qb * q_bytes + pn * (H * 128), &qmap, q_full + qb, pn * panel_elems,
-                        static_cast<int>(row * p.H));
-          last_q[qb] = j;
-          // key tiles: blocks_per_tile consecutive retained blocks per tile
-          const int ntiles = (cnt * p.B + kTokTileM - 1) / kTokTileM;
-          for (int tl = 0; ok && tl < ntiles; ++tl, ++kt) {
-            const int st = static_cast<int>(kt % p.stages);
-            if (!(ok = mbar_wait(k_empty + st, static_cast<uint32_t>(((kt / p.stages) & 1) ^ 1), abort_flag))) break;
-            const int first = tl * blocks_per_tile;
-            const int nblk_t = min(blocks_per_tile, cnt - first);
-            mbar_arrive_expect_tx(k_full + st, static_cast<uint32_t>(nblk_t * p.B * row_bytes));
-            for (int q = 0; q < nblk_t; ++q) {
-              const int krow = b * p.L + J.blk[first + q] * p.B;
-              for (int pn = 0; pn < panels; ++pn)
-                tma_load_2d(k_buf + st * k_bytes + pn * (kTokTileM * 128) + q * p.B * 128, &kmap, k_full + st,
-                            pn * panel_elems, krow);
-            }
-            last_k[st] = kt;
+        const uint32_t qph = static_cast<uint32_t>((j >> 1) & 1);
+        if (!(ok = mbar_wait(q_empty + qb, qph ^ 1, abort_flag))) break;
+        mbar_arrive_expect_tx(q_full + qb, q_bytes);
+        for (int pn = 0; pn < panels; ++pn)
+          tma_load_2d(q_buf + qb * q_bytes + pn * (H * 128), &qmap, q_full + qb, pn * panel_elems,
+                      static_cast<int>(J.row * p.H));
+        last_qph[qb] = static_cast<int8_t>(qph);
+        const int kb = J.b * p.L;
+        for (int tl = 0; tl < J.ntiles; ++tl) {
+          if (!(ok = mbar_wait(k_empty + st, kph ^ 1, abort_flag))) break;
+          const int first = tl * blocks_per_tile;
+          const int nblk_t = min(blocks_per_tile, J.nblk - first);
+          mbar_arrive_expect_tx(k_full + st, static_cast<uint32_t>(nblk_t * p.B * row_bytes));
+          for (int q = 0; q < nblk_t; ++q) {
+            const int krow = kb + J.blk[first + q] * p.B;
+            for (int pn = 0; pn < panels; ++pn)
+              tma_load_2d(k_buf + st * k_bytes + pn * (kTokTileM * 128) + q * p.B * 128, &kmap, k_full + st,
+                          pn * panel_elems, krow);
           }
+          last_ph[st] = static_cast<int8_t>(kph);
+          if (++st == p.stages) { st = 0; kph ^= 1; }
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-    }
-    if (!ok && lane == 0) {
-      for (int s = 0; s < p.stages; ++s)
-        if (last_k[s] >= 0) mbar_drain(k_full + s, static_cast<uint32_t>((last_k[s] / p.stages) & 1));
-      for (int i = 0; i < 2; ++i)
-        if (last_q[i] >= 0) mbar_drain(q_full + i, static_cast<uint32_t>((last_q[i] >> 1) & 1));
+      if (!ok) {   // drain the copies this thread issued before leaving
+        for (int i = 0; i < p.stages; ++i)
+          if (last_ph[i] >= 0) mbar_drain(k_full + i, static_cast<uint32_t>(last_ph[i]));
+        for (int i = 0; i < 2; ++i)
+          if (last_qph[i] >= 0) mbar_drain(q_full + i, static_cast<uint32_t>(last_qph[i]));
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc(kTokTileM, H, DT == DT_BF16 ? 1u : 0u);
       const int ksteps = row_bytes / 32;
-      int64_t kt = 0, tc = 0;
+      int st = 0, ab = 0;
+      uint32_t kph = 0, aph = 0;
       bool ok = true;
       for (int64_t j = 0; ok && j < njobs; ++j) {
         const int slot = static_cast<int>(j % kTokJobs);
@@ -239,11 +251,9 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
         if (!(ok = mbar_wait(q_full + qb, static_cast<uint32_t>((j >> 1) & 1), abort_flag))) break;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(q_buf + qb * q_bytes);
-        for (int i = 0; i < ntiles; ++i, ++kt, ++tc) {
-          const int st = static_cast<int>(kt % p.stages);
-          const int ab = static_cast<int>(tc % kTokAcc);
-          if (!(ok = mbar_wait(acc_empty + ab, static_cast<uint32_t>(((tc / kTokAcc) & 1) ^ 1), abort_flag))) break;
-          if (!(ok = mbar_wait(k_full + st, static_cast<uint32_t>((kt / p.stages) & 1), abort_flag))) break;
+        for (int i = 0; i < ntiles; ++i) {
+          if (!(ok = mbar_wait(acc_empty + ab, aph ^ 1, abort_flag))) break;
+          if (!(ok = mbar_wait(k_full + st, kph, abort_flag))) break;
           tc_fence_after();
           const uint32_t k_addr = smem_u32(k_buf + st * k_bytes);
           const uint32_t d_tmem = tmem_base + ab * H;
@@ -254,17 +264,21 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
           }
           mma_commit(k_empty + st);
           mma_commit(acc_full + ab);
+          if (++st == p.stages) { st = 0; kph ^= 1; }
+          if (++ab == kTokAcc) { ab = 0; aph ^= 1; }
         }
         if (ok) mma_commit(q_empty + qb);
       }
       mma_commit(drain);
       mbar_drain(drain, 0);
     }
-  } else if (warp < 2 + kTokScorerWarps) {
+  } else if (warp >= kTokScorerBase && warp < kTokScorerBase + kTokScorerWarps) {
     // ------------------------------------------------------------ scorer
     const int quarter = warp & 3;
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    int64_t tc = 0;
+    const int bshift = __ffs(p.B) - 1;
+    int ab = 0;
+    uint32_t aph = 0;
     bool ok = true;
     for (int64_t j = 0; ok && j < njobs; ++j) {
       const int slot = static_cast<int>(j % kTokJobs);
@@ -279,26 +293,34 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
       const int ntiles = J.ntiles;
       uint32_t* cj = cand + cb * p.max_cand;
       float ksc = 1.f;
-      for (int i = 0; i < ntiles; ++i, ++tc) {
-        const int ab = static_cast<int>(tc % kTokAcc);
-        if (lane == 0) okl = mbar_wait(acc_full + ab, static_cast<uint32_t>((tc / kTokAcc) & 1), abort_flag);
+      for (int i = 0; i < ntiles; ++i) {
+        if (lane == 0) okl = mbar_wait(acc_full + ab, aph, abort_flag);
         if (!(ok = __shfl_sync(0xffffffffu, okl, 0) != 0)) break;
         tc_fence_after();
         const int c = i * kTokTileM + quarter * 32 + lane;        // candidate position
-        const int slot_b = c / p.B;
-        const int s = slot_b < J.nblk ? J.blk[slot_b] * p.B + c % p.B : p.L;
+        const int slot_b = c >> bshift;
+        const int s = slot_b < J.nblk ? (J.blk[slot_b] << bshift) + (c & (p.B - 1)) : p.L;
         const bool valid = s < J.n;
         if (DT == DT_E4M3 && valid) ksc = __ldg(p.k_scale + static_cast<int64_t>(J.b) * p.L + s);
         float acc = 0.f;
         if (H >= 32) {
+          // all TMEM loads of the row first, one wait, then four independent
+          // accumulation chains over float4 weight reads
+          uint32_t v[H];
 #pragma unroll
-          for (int c0 = 0; c0 < H; c0 += 32) {
-            uint32_t v[32];
-            tmem_ld32(t_lane + ab * H + c0, v);
-            tmem_wait_ld();
+          for (int c0 = 0; c0 < H; c0 += 32) tmem_ld32(t_lane + ab * H + c0, *reinterpret_cast<uint32_t(*)[32]>(v + c0));
+          tmem_wait_ld();
+          float a4[4] = {0.f, 0.f, 0.f, 0.f};
+          const float4* w4 = reinterpret_cast<const float4*>(J.w);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) acc = fmaf(J.w[c0 + e], fmaxf(__uint_as_float(v[e]), 0.f), acc);
+          for (int e = 0; e < H / 4; ++e) {
+            const float4 wv = w4[e];
+            a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * e + 0]), 0.f), a4[0]);
+            a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * e + 1]), 0.f), a4[1]);
+            a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * e + 2]), 0.f), a4[2]);
+            a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * e + 3]), 0.f), a4[3]);
           }
+          acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
         } else {
           uint32_t v[16];
           tmem_ld16(t_lane + ab * H, v);
@@ -311,6 +333,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty + ab);
+        if (++ab == kTokAcc) { ab = 0; aph ^= 1; }
       }
       if (!ok) break;
       __syncwarp();
@@ -331,20 +354,16 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
       int32_t* oi = p.out_idx + J.row * p.top_k;
       float* os = p.out_score ? p.out_score + J.row * p.top_k : nullptr;
       auto key_at = [&](int i) { return cj[i]; };
+      const int bshift = __ffs(p.B) - 1;
       auto emit = [&](uint32_t slot_out, int i, uint32_t key) {
-        oi[slot_out] = J.blk[i / p.B] * p.B + i % p.B;
+        oi[slot_out] = (J.blk[i >> bshift] << bshift) + (i & (p.B - 1));
         if (os) os[slot_out] = key_float(key);
       };
-      const uint32_t n_valid = block_count_valid<decltype(key_at), SelGrp>(key_at, ncand, *sel);
-      if (n_valid <= static_cast<uint32_t>(p.top_k)) {
-        block_emit_all<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, emit, *sel);
-        for (int i = n_valid + stid; i < p.top_k; i += SelGrp::size()) {
-          oi[i] = -1;
-          if (os) os[i] = -__int_as_float(0x7f800000);
-        }
-      } else {
-        block_radix_topk<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, static_cast<uint32_t>(p.top_k),
-                                                                   emit, *sel);
+      const uint32_t nv = block_topk<decltype(key_at), decltype(emit), SelGrp>(
+          key_at, ncand, static_cast<uint32_t>(p.top_k), emit, *sel);
+      for (int i = static_cast<int>(nv) + stid; i < p.top_k; i += SelGrp::size()) {
+        oi[i] = -1;
+        if (os) os[i] = -__int_as_float(0x7f800000);
       }
       SelGrp::sync();
       if (stid == 0) {
@@ -363,7 +382,8 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
 
 inline size_t token_smem_bytes(int row_bytes, int H, int stages, int max_cand) {
   return 1024 + 2 * static_cast<size_t>(H) * row_bytes + static_cast<size_t>(stages) * kTokTileM * row_bytes +
-         2 * static_cast<size_t>(max_cand) * 4 + kTokJobs * sizeof(TokJob) + sizeof(SelectSmem) + 8 +
+         2 * static_cast<size_t>(max_cand) * 4 + kTokJobs * sizeof(TokJob) + sizeof(SelectSmem) +
+         4 * kTokMaxBitmapWords + 8 +
          8 * (2 * stages + 4 + 2 * kTokAcc + 2 * kTokJobs + 4 + 1) + 16;
 }
 

@@ -44,11 +44,11 @@ def _shape(**kw):
 
 def test_workspace_sizes(L):
     s = _shape()
-    assert hb.workspace_size(hb.OP_FLAT, s) == 32768 * 32768 * 4
+    assert hb.workspace_size(hb.OP_FLAT, s) == 32768 * (32768 * 4 + 8)
     assert hb.workspace_size(hb.OP_BLOCK, s) == 32768 * 256 * 4
     assert hb.workspace_size(hb.OP_TOKEN, s) == 0
     s = _shape(num_keys=1001, num_queries=3, batch=2, block_size=64)
-    assert hb.workspace_size(hb.OP_FLAT, s) == 6 * 1004 * 4          # rows padded to 16 bytes
+    assert hb.workspace_size(hb.OP_FLAT, s) == 6 * (1004 * 4 + 8)    # rows padded to 16 bytes, + row range
     assert hb.workspace_size(hb.OP_BLOCK, s) == 6 * 16 * 4           # ceil(1001/64)=16
 
 
