@@ -47,6 +47,7 @@ _SIGS = {
                            ctypes.c_int32, _P],
     "hisa_quantize_e4m3": [_P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _P, _P, _P],
     "hisa_block_score_topm": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, ctypes.c_size_t, _P],
+    "hisa_block_score_topm_static": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P],
     "hisa_token_score_topk": [_P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t,
                               _P],
     "dsa_flat_indexer_topk": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t, _P],
@@ -194,6 +195,22 @@ def hisa_block_score_topm(q, w, kpool, n_visible, *, num_keys: int, block_size: 
                                         _ptr(kpool_scale), n_visible.data_ptr(), ctypes.byref(shape),
                                         out.data_ptr(), ws.data_ptr(), ws.numel(), _stream()),
            "hisa_block_score_topm")
+    return out
+
+
+def hisa_block_score_topm_static(q, w, kpool, n_visible, *, num_keys: int, block_size: int, top_m: int,
+                                 q_scale=None, kpool_scale=None):
+    """Coarse stage using the library's built-in score scratch: no workspace is
+    allocated, by torch or by the library (see include/hisa.h for its size
+    limit and the rule that calls must not overlap)."""
+    b, Q, H, d = q.shape
+    shape = Shape(b, num_keys, Q, H, d, block_size, top_m, 1, dtype_code(q))
+    _need(w, "w", 3)
+    _need(n_visible, "n_visible", 2)
+    out = torch.empty((b, Q, top_m), dtype=torch.int32, device=q.device)
+    _check(load().hisa_block_score_topm_static(q.data_ptr(), _ptr(q_scale), w.data_ptr(), kpool.data_ptr(),
+                                               _ptr(kpool_scale), n_visible.data_ptr(), ctypes.byref(shape),
+                                               out.data_ptr(), _stream()), "hisa_block_score_topm_static")
     return out
 
 

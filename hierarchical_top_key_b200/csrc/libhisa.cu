@@ -6,6 +6,7 @@
 #include <cstring>
 #include <cstdarg>
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include <cudaTypedefs.h>
@@ -540,6 +541,70 @@ hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale, const flo
     if (e != HISA_OK) return e;
   }
   return HISA_OK;
+}
+
+}  // extern "C"
+
+// =================================================================== no-allocation variant
+//
+// hisa_block_score_topm_static: the coarse stage for callers that cannot
+// allocate device memory at call time (code running inside another runtime's
+// memory arena, plug-ins handed only input and output pointers, or hosts that
+// forbid cudaMalloc on the serving path).  Its block-score rows live in one
+// file-scope device array instead of a caller workspace.
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB of fp32 block scores
+
+// Held by every GPU that loads the library, until the process exits.  In host
+// code this name is only a host-side handle; its device address comes from
+// cudaGetSymbolAddress below.
+static __device__ __align__(256) float g_static_block_scores[kStaticScratchBytes / sizeof(float)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, resolved once
+// per device with that device current.
+hisa_status static_scratch(float** out) {
+  int dev = 0;
+  hisa_status e = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (e != HISA_OK) return e;
+  if (dev < 0 || dev >= kMaxDevices) return fail(HISA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cuda_check(cudaGetSymbolAddress(&p, g_static_block_scores), "cudaGetSymbolAddress(block-score scratch)");
+    if (e != HISA_OK) return e;
+    g_static_ptr[dev] = p;
+  }
+  *out = static_cast<float*>(g_static_ptr[dev]);
+  return HISA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+hisa_status hisa_block_score_topm_static(const void* q, const float* q_scale, const float* w, const void* kpool,
+                                         const float* kpool_scale, const int32_t* n_visible, const hisa_shape* s,
+                                         int32_t* block_idx, hisa_stream stream) {
+  hisa_status e = check_shape(s, true);
+  if (e != HISA_OK) return e;
+  const size_t need = static_cast<size_t>(rows_of(s)) * static_cast<size_t>(pad4(num_blocks(s))) * sizeof(float);
+  if (need > kStaticScratchBytes)
+    return fail(HISA_ERR_WORKSPACE,
+                "block scores need %zu bytes; the built-in scratch holds %zu (use hisa_block_score_topm with a "
+                "caller workspace)", need, kStaticScratchBytes);
+  float* scratch = nullptr;
+  e = static_scratch(&scratch);
+  if (e != HISA_OK) return e;
+  // every score row the selection reads is written first by the scoring
+  // kernel, so nothing in the scratch has to start at zero
+  return hisa_block_score_topm(q, q_scale, w, kpool, kpool_scale, n_visible, s, block_idx, scratch,
+                               kStaticScratchBytes, stream);
 }
 
 }  // extern "C"

@@ -190,6 +190,32 @@ HISA_API hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale,
                                   float* topk_score, void* workspace,
                                   size_t ws_bytes, hisa_stream stream);
 
+/*
+ * hisa_block_score_topm without a caller workspace, for callers that cannot
+ * allocate device memory when they call the indexer (for example code that
+ * runs inside another runtime's memory arena, or a plug-in that is handed only
+ * its input and output pointers).  The paper has no counterpart; this is an
+ * interface convenience.  Same arguments and results as hisa_block_score_topm
+ * minus the workspace.
+ *  - The block scores are kept in one 16 MiB array built into the library;
+ *    every GPU that loads the library reserves it until the process exits.
+ *    Shapes with batch*Q*round_up(ceil(L/B), 4)*4 bytes above 16 MiB return
+ *    HISA_ERR_WORKSPACE without launching anything.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *    The first call on each device looks up the array's device address on the
+ *    current device (cudaGetSymbolAddress); make that first call before any
+ *    stream capture.
+ *  - All calls share the array and it keeps the last call's contents (nothing
+ *    in it needs to start cleared).  Calls that overlap on the GPU, on
+ *    different streams or different host threads, race on it: order them.
+ */
+HISA_API hisa_status hisa_block_score_topm_static(const void* q, const float* q_scale,
+                                  const float* w, const void* kpool,
+                                  const float* kpool_scale,
+                                  const int32_t* n_visible,
+                                  const hisa_shape* shape, int32_t* block_idx,
+                                  hisa_stream stream);
+
 /* Workspace bytes that let `op` run on `shape` in one pass (0 if none). */
 HISA_API hisa_status hisa_workspace_size(int32_t op, const hisa_shape* shape,
                                 size_t* bytes);
