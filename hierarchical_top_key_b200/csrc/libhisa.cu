@@ -525,6 +525,9 @@ hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale, const flo
   for (const RowChunk& c : chunks) max_rows = std::max(max_rows, c.nrows);
   uint32_t* minmax = reinterpret_cast<uint32_t*>(ws + max_rows * ld);
   const bool fused_range = dense_tc_ok(s);
+  e = cuda_check(cudaFuncSetAttribute(flat_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(sizeof(TwoPassSmem))), "flat_select attribute");
+  if (e != HISA_OK) return e;
   for (const RowChunk& c : chunks) {
     if (fused_range) {
       init_minmax_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(c.nrows, 256), 1024)), 256, 0, st>>>(
@@ -535,7 +538,7 @@ hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale, const flo
     e = score_rows(s, q, q_scale, w, k, k_scale, n_visible, 0, s->num_keys, c, ws, ld, st,
                    fused_range ? minmax : nullptr);
     if (e != HISA_OK) return e;
-    flat_select_kernel<<<static_cast<unsigned>(c.nrows), 512, 0, st>>>(
+    flat_select_kernel<<<static_cast<unsigned>(c.nrows), 512, sizeof(TwoPassSmem), st>>>(
         ws, ld, fused_range ? minmax : nullptr, n_visible, c.row0, s->num_keys, s->top_k, topk_idx, topk_score);
     e = launch_check("flat_select_kernel");
     if (e != HISA_OK) return e;

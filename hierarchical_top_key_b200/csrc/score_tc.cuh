@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* w_s = reinterpret_cast<float*>(tmem_slot + 4);  // [8 warps][G/2 * H] = [4 * G * H]
+  float* w_s = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(tmem_slot + 2) + 15) & ~uintptr_t(15));
+                                                         // [8 warps][G/2 * H] = [4 * G * H], 16-byte aligned
   float* qsc_s = w_s + 4 * kDenseN;                      // [8 warps][G/2]
   int* vis_s = reinterpret_cast<int*>(qsc_s + 4 * G);    // [8 warps][G/2]
 
@@ -264,14 +265,24 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
           const float* wq = w_w + jq * H;
           float acc = 0.f;
           if (H >= 32) {
+            // the query's H columns in one batch of TMEM loads, one wait, then
+            // four independent accumulation chains over float4 weights
+            uint32_t v[H];
 #pragma unroll
-            for (int c0 = 0; c0 < H; c0 += 32) {
-              uint32_t v[32];
-              tmem_ld32(t_row + j * H + c0, v);
-              tmem_wait_ld();
+            for (int c0 = 0; c0 < H; c0 += 32)
+              tmem_ld32(t_row + j * H + c0, *reinterpret_cast<uint32_t(*)[32]>(v + c0));
+            tmem_wait_ld();
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+            const float4* w4 = reinterpret_cast<const float4*>(wq);
 #pragma unroll
-              for (int c = 0; c < 32; ++c) acc = fmaf(wq[c0 + c], fmaxf(__uint_as_float(v[c]), 0.f), acc);
+            for (int e = 0; e < H / 4; ++e) {
+              const float4 wv = w4[e];
+              a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * e + 0]), 0.f), a4[0]);
+              a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * e + 1]), 0.f), a4[1]);
+              a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * e + 2]), 0.f), a4[2]);
+              a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * e + 3]), 0.f), a4[3]);
             }
+            acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
           } else {
             uint32_t v[16];
             tmem_ld16(t_row + j * H, v);
@@ -316,7 +327,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
 // Bytes of dynamic shared memory the dense kernel needs.
 inline size_t dense_smem_bytes(int row_bytes, int stages, int q_bufs) {
   return 1024 /*alignment slack*/ + q_bufs * static_cast<size_t>(kDenseN) * row_bytes +
-         static_cast<size_t>(stages) * kDenseTileM * row_bytes + 8 * (2 * stages + 9) + 16 + 4 * 4 * kDenseN +
+         static_cast<size_t>(stages) * kDenseTileM * row_bytes + 8 * (2 * stages + 9) + 32 + 4 * 4 * kDenseN +
          2 * 4 * 4 * 64 + 64;
 }
 

@@ -224,14 +224,160 @@ __device__ uint32_t block_topk_range(KeyAt key_at, int n, uint32_t k, Emit emit,
 
 // ---------------------------------------------------------------- row kernels
 
+// Two-pass top-k over positions [0, n) whose valid keys lie in [kmin, kmax]
+// (key 0 marks an absent position and is skipped).  Pass 1: histogram over
+// 2048 bins spaced linearly in score value between the smallest and largest
+// score (a monotone map, so whole bins are ordered; linear spacing spreads
+// the bulk of the scores, where ordering-key bits would pile it into the few
+// bins of a handful of exponents).  Pass 2: every key above the boundary bin is emitted;
+// the boundary bin's (key, position) pairs go to an on-chip buffer of `cap`
+// entries (a power of two), where the remaining places are chosen exactly
+// (larger key first, then lower position).  Returns false, having emitted
+// nothing, when the boundary bin would overflow the buffer; the caller then
+// falls back to block_topk_range.
+template <class KeyAt, class Emit, class Grp>
+__device__ bool two_pass_topk(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem& sm, uint32_t* buf_key,
+                              int32_t* buf_pos, uint32_t* buf_count, int cap, uint32_t kmin, uint32_t kmax) {
+  const int lane = Grp::tid() & 31;
+  const int nbins = kDigitBins;
+  const float smin = key_float(kmin), smax = key_float(kmax);
+  float scale = smax > smin ? static_cast<float>(nbins) / (smax - smin) : 0.f;
+  if (!(scale < 1e30f)) scale = 0.f;                 // overflowing or degenerate range: one bin
+  auto bin_of = [&](uint32_t key) -> uint32_t {
+    const int b = static_cast<int>((key_float(key) - smin) * scale);
+    return static_cast<uint32_t>(min(max(b, 0), nbins - 1));
+  };
+  for (int i = Grp::tid(); i < nbins; i += Grp::size()) sm.hist[i] = 0;
+  if (Grp::tid() == 0) { *buf_count = 0; sm.n_slots = 0; }
+  Grp::sync();
+  for (int i = Grp::tid(); i < n; i += Grp::size()) {
+    const uint32_t key = key_at(i);
+    if (key != 0u) atomicAdd(&sm.hist[bin_of(key)], 1u);
+  }
+  Grp::sync();
+  uint32_t remaining = k;
+  {
+    const int nt = Grp::size();
+    const int per = nbins >= nt ? nbins / nt : 1;
+    const int top = nbins - 1 - Grp::tid() * per;
+    uint32_t t = 0;
+    for (int j = 0; j < per; ++j)
+      if (top - j >= 0) t += sm.hist[top - j];
+    uint32_t incl = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) sm.warp_cnt[Grp::tid() >> 5] = incl;
+    Grp::sync();
+    uint32_t woff = 0;
+    for (int wi = 0; wi < (Grp::tid() >> 5); ++wi) woff += sm.warp_cnt[wi];
+    incl += woff;
+    const uint32_t excl = incl - t;
+    if (t > 0 && excl < remaining && incl >= remaining) {
+      uint32_t c = excl;
+      for (int j = 0; j < per; ++j) {
+        const uint32_t h = sm.hist[top - j];
+        if (c + h >= remaining) { sm.digit = top - j; sm.above = c; sm.at_digit = h; break; }
+        c += h;
+      }
+    }
+  }
+  Grp::sync();
+  const uint32_t D = sm.digit, above = sm.above, n_eq = sm.at_digit;
+  remaining -= above;
+  Grp::sync();
+  const bool take_bin = n_eq == remaining;
+  if (!take_bin && n_eq > static_cast<uint32_t>(cap)) return false;
+  // pass 2: emit keys above the boundary bin; buffer the bin (or take all of it)
+  for (int base = 0; base < n; base += Grp::size()) {
+    const int i = base + Grp::tid();
+    const uint32_t key = i < n ? key_at(i) : 0u;
+    const bool valid = key != 0u;
+    const uint32_t dg = valid ? bin_of(key) : 0u;
+    const bool gt = valid && (dg > D || (take_bin && dg == D));
+    const uint32_t ball = __ballot_sync(0xffffffffu, gt);
+    uint32_t slot0 = 0;
+    if (lane == 0 && ball) slot0 = atomicAdd(&sm.n_slots, __popc(ball));
+    slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+    if (gt) emit(slot0 + __popc(ball & ((1u << lane) - 1u)), i, key);
+    if (!take_bin) {
+      const bool eq = valid && dg == D;
+      const uint32_t be = __ballot_sync(0xffffffffu, eq);
+      uint32_t b0 = 0;
+      if (lane == 0 && be) b0 = atomicAdd(buf_count, __popc(be));
+      b0 = __shfl_sync(0xffffffffu, b0, 0);
+      if (eq) {
+        const uint32_t at = b0 + __popc(be & ((1u << lane) - 1u));
+        buf_key[at] = key;
+        buf_pos[at] = i;
+      }
+    }
+  }
+  Grp::sync();
+  if (take_bin) return true;
+  // choose `remaining` of the n_eq buffered keys: larger key first, then lower position
+  const int nb = static_cast<int>(n_eq);
+  if (nb <= 256) {
+    for (int e = Grp::tid(); e < nb; e += Grp::size()) {
+      const uint32_t ke = buf_key[e];
+      const int pe = buf_pos[e];
+      uint32_t rank = 0;
+      for (int f = 0; f < nb; ++f) {
+        const uint32_t kf = buf_key[f];
+        rank += (kf > ke || (kf == ke && buf_pos[f] < pe)) ? 1u : 0u;
+      }
+      if (rank < remaining) emit(above + rank, pe, ke);
+    }
+  } else {
+    // bitonic sort of the buffer (padded to a power of two) by (key desc, position asc)
+    int np2 = 1;
+    while (np2 < nb) np2 <<= 1;
+    for (int i = nb + Grp::tid(); i < np2; i += Grp::size()) { buf_key[i] = 0u; buf_pos[i] = 0x7FFFFFFF; }
+    Grp::sync();
+    for (int size = 2; size <= np2; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = Grp::tid(); i < np2 / 2; i += Grp::size()) {
+          const int lo = 2 * i - (i & (stride - 1));
+          const int hi = lo + stride;
+          const bool desc = (lo & size) == 0;          // this run sorts "best first"
+          const uint32_t ka = buf_key[lo], kb = buf_key[hi];
+          const int pa = buf_pos[lo], pb = buf_pos[hi];
+          const bool b_better = kb > ka || (kb == ka && pb < pa);
+          if (b_better == desc) {
+            buf_key[lo] = kb; buf_key[hi] = ka;
+            buf_pos[lo] = pb; buf_pos[hi] = pa;
+          }
+        }
+        Grp::sync();
+      }
+    }
+    for (int e = Grp::tid(); e < static_cast<int>(remaining); e += Grp::size()) emit(above + e, buf_pos[e], buf_key[e]);
+  }
+  Grp::sync();
+  return true;
+}
+
+constexpr int kTwoPassCap = 4096;
+
+struct TwoPassSmem {
+  uint32_t key[kTwoPassCap];
+  int32_t pos[kTwoPassCap];
+  uint32_t count;
+};
+
 // Flat DSA top-k over fp32 score rows: row r holds scores of keys 0..n_r-1.
 // `minmax` (nullable) holds, per row, the smallest and largest ordering key
-// the scoring kernel wrote, which saves the range pass over the row.
+// the scoring kernel wrote; with it the row is read twice (histogram, then
+// emission), without it the generic multi-pass selection runs.
 __global__ void __launch_bounds__(512) flat_select_kernel(
     const float* __restrict__ scores, int64_t ld, const uint32_t* __restrict__ minmax,
     const int32_t* __restrict__ n_visible, int64_t row0, int L, int top_k, int32_t* __restrict__ out_idx,
     float* __restrict__ out_score) {
   __shared__ SelectSmem sm;
+  extern __shared__ __align__(16) uint8_t flat_dyn[];
+  TwoPassSmem& tp = *reinterpret_cast<TwoPassSmem*>(flat_dyn);
   const int64_t r = row0 + blockIdx.x;
   const float* row = scores + static_cast<int64_t>(blockIdx.x) * ld;
   const int n = max(0, min(n_visible[r], L));
@@ -241,14 +387,15 @@ __global__ void __launch_bounds__(512) flat_select_kernel(
     oi[slot] = i;
     if (os) os[slot] = key_float(key);
   };
-  auto key_at = [&](int i) { return float_key(row[i]); };
-  uint32_t nv;
-  if (minmax != nullptr && n > 0) {
-    nv = block_topk_range(key_at, n, static_cast<uint32_t>(top_k), emit, sm, minmax[2 * blockIdx.x],
-                          minmax[2 * blockIdx.x + 1], static_cast<uint32_t>(n));
-  } else {
-    nv = block_topk(key_at, n, static_cast<uint32_t>(top_k), emit, sm);
+  auto key_at = [&](int i) { return float_key(__ldcg(row + i)); };
+  uint32_t nv = static_cast<uint32_t>(n);
+  bool done = false;
+  if (minmax != nullptr && n > top_k) {
+    done = two_pass_topk<decltype(key_at), decltype(emit), CtaGroup>(
+        key_at, n, static_cast<uint32_t>(top_k), emit, sm, tp.key, tp.pos, &tp.count, kTwoPassCap,
+        minmax[2 * blockIdx.x], minmax[2 * blockIdx.x + 1]);
   }
+  if (!done) nv = block_topk(key_at, n, static_cast<uint32_t>(top_k), emit, sm);
   for (int i = static_cast<int>(nv) + threadIdx.x; i < top_k; i += blockDim.x) {
     oi[i] = -1;
     if (os) os[i] = -__int_as_float(0x7f800000);

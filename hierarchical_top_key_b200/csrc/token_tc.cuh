@@ -11,11 +11,15 @@
 // pipeline of jobs:
 //   warp 0       job set-up (whole warp: read, filter, dedupe and sort the
 //                block list; stage w[t]), running up to four jobs ahead
-//   warp 1       TMEM owner and MMA issuer
-//   warp 2       TMA issuer: q[t] and one tile load per retained block
-//   warps 3..6   scorer: TMEM -> weighted ReLU sum -> candidate keys in smem
-//   warps 7..14  selector: radix top-k over the candidate keys, emit indices
-// Rings: job slots (4), q buffers (2), key stages, TMEM accumulators (4 x H
+//   warps 1, 2   MMA issuers, alternate tiles (warp 1 owns TMEM).  An M=128,
+//                N=64 MMA is bound by per-thread issue, not by the tensor
+//                core, so two issuers nearly double the rate.
+//   warp 3       TMA issuer: q[t] and one tile load per retained block
+//   warps 4..11  scorers, two groups of four on alternate tiles: TMEM ->
+//                weighted ReLU sum -> candidate keys in smem, plus each
+//                job's key range and valid count
+//   warps 12..15 selector: two-pass radix top-k over the candidate keys
+// Rings: job slots (4), q buffers (2), key stages, TMEM accumulators (8 x H
 // columns), candidate buffers (2).  Blocks are sorted ascending so candidate
 // position order is key order, which makes ties resolve to the lower key.
 #pragma once
@@ -27,12 +31,16 @@ namespace hisa {
 
 constexpr int kTokTileM = 128;
 constexpr int kTokJobs = 4;
-constexpr int kTokAcc = 4;
-constexpr int kTokScorerWarps = 4;
-constexpr int kTokSelectWarps = 8;
-constexpr int kTokScorerBase = 3;                 // first scorer warp
-constexpr int kTokSelectBase = 32 * (kTokScorerBase + kTokScorerWarps);
+constexpr int kTokAcc = 8;                        // TMEM accumulators (multiple of the issuer count)
+constexpr int kTokIssuers = 2;                    // MMA issuer warps 1..kTokIssuers
+constexpr int kTokTmaWarp = 1 + kTokIssuers;
+constexpr int kTokScorerBase = kTokTmaWarp + 1;   // first scorer warp
+constexpr int kTokScorerWarps = 4;                // per group; one warp per TMEM lane quarter
+constexpr int kTokScoreGroups = 2;
+constexpr int kTokSelectWarps = 4;
+constexpr int kTokSelectBase = 32 * (kTokScorerBase + kTokScorerWarps * kTokScoreGroups);
 constexpr int kTokThreads = kTokSelectBase + 32 * kTokSelectWarps;
+constexpr int kTokBinCap = 256;                   // boundary-bin buffer of the selector
 constexpr int kTokMaxBlocks = 256;                // top_m limit
 constexpr int kTokMaxBitmapWords = 256;           // blocks per sequence limit / 32
 
@@ -55,6 +63,7 @@ struct alignas(16) TokJob {
   int64_t row;
   int b, n, nblk, ntiles;
   float qsc;
+  uint32_t kmin, kmax, nvalid;     // filled by the scorers for the selector
   alignas(16) float w[64];
   int blk[kTokMaxBlocks];
 };
@@ -69,6 +78,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, const TokenParams p) {
   using namespace sm100;
   using SelGrp = WarpRange<kTokSelectBase, 32 * kTokSelectWarps, 2>;
+  static_assert(kTokAcc % kTokIssuers == 0 && kTokAcc % kTokScoreGroups == 0, "tile ownership");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int row_bytes = p.d * Elem<DT>::bytes;
@@ -83,7 +93,10 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
   TokJob* jobs = reinterpret_cast<TokJob*>(cand + 2 * p.max_cand);            // [kTokJobs]
   SelectSmem* sel = reinterpret_cast<SelectSmem*>(jobs + kTokJobs);
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(sel + 1);                     // [kTokMaxBitmapWords]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uintptr_t>(bitmap + kTokMaxBitmapWords) + 7 & ~uintptr_t(7));
+  uint32_t* bin_key = bitmap + kTokMaxBitmapWords;                             // [kTokBinCap]
+  int32_t* bin_pos = reinterpret_cast<int32_t*>(bin_key + kTokBinCap);         // [kTokBinCap]
+  uint32_t* bin_count = reinterpret_cast<uint32_t*>(bin_pos + kTokBinCap);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uintptr_t>(bin_count + 1) + 7 & ~uintptr_t(7));
   uint64_t* k_full = bars;
   uint64_t* k_empty = k_full + p.stages;
   uint64_t* q_full = k_empty + p.stages;          // [2]
@@ -94,8 +107,8 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
   uint64_t* job_empty = job_full + kTokJobs;      // [kTokJobs]
   uint64_t* cand_full = job_empty + kTokJobs;     // [2]
   uint64_t* cand_empty = cand_full + 2;           // [2]
-  uint64_t* drain = cand_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = cand_empty + 2;                // [kTokIssuers]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + kTokIssuers);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* sel_ok = abort_flag + 1;
 
@@ -103,12 +116,12 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(q_full + i, 1); mbar_init(q_empty + i, 1);
-      mbar_init(cand_full + i, kTokScorerWarps); mbar_init(cand_empty + i, 1);
+      mbar_init(q_full + i, 1); mbar_init(q_empty + i, kTokIssuers);
+      mbar_init(cand_full + i, kTokScorerWarps * kTokScoreGroups); mbar_init(cand_empty + i, 1);
     }
     for (int i = 0; i < kTokAcc; ++i) { mbar_init(acc_full + i, 1); mbar_init(acc_empty + i, kTokScorerWarps); }
     for (int i = 0; i < kTokJobs; ++i) { mbar_init(job_full + i, 1); mbar_init(job_empty + i, 1); }
-    mbar_init(drain, 1);
+    for (int i = 0; i < kTokIssuers; ++i) mbar_init(drain + i, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -187,11 +200,14 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
         J.nblk = cnt;
         J.ntiles = (cnt * p.B + kTokTileM - 1) / kTokTileM;
         J.qsc = qsc;
+        J.kmin = 0xFFFFFFFFu;
+        J.kmax = 0u;
+        J.nvalid = 0u;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(job_full + slot);
     }
-  } else if (warp == 2) {
+  } else if (warp == kTokTmaWarp) {
     // ------------------------------------------------------------ TMA issue
     if (lane == 0) {
       int st = 0;
@@ -235,12 +251,13 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
           if (last_qph[i] >= 0) mbar_drain(q_full + i, static_cast<uint32_t>(last_qph[i]));
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp >= 1 && warp <= kTokIssuers) {
+    // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
+      const int me = warp - 1;                        // this issuer takes tiles g with g % kTokIssuers == me
       constexpr uint32_t idesc = instr_desc(kTokTileM, H, DT == DT_BF16 ? 1u : 0u);
       const int ksteps = row_bytes / 32;
-      int st = 0, ab = 0;
+      int st = 0, ab = 0, g = 0;
       uint32_t kph = 0, aph = 0;
       bool ok = true;
       for (int64_t j = 0; ok && j < njobs; ++j) {
@@ -252,32 +269,36 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
         tc_fence_after();
         const uint32_t q_addr = smem_u32(q_buf + qb * q_bytes);
         for (int i = 0; i < ntiles; ++i) {
-          if (!(ok = mbar_wait(acc_empty + ab, aph ^ 1, abort_flag))) break;
-          if (!(ok = mbar_wait(k_full + st, kph, abort_flag))) break;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(k_buf + st * k_bytes);
-          const uint32_t d_tmem = tmem_base + ab * H;
-          for (int ks = 0; ks < ksteps; ++ks) {
-            const int pn = ks >> 2, off = (ks & 3) * 32;
-            mma<DT>(d_tmem, desc_k_sw128(k_addr + pn * (kTokTileM * 128) + off),
-                    desc_k_sw128(q_addr + pn * (H * 128) + off), idesc, ks > 0 ? 1u : 0u);
+          if (g == me) {
+            if (!(ok = mbar_wait(acc_empty + ab, aph ^ 1, abort_flag))) break;
+            if (!(ok = mbar_wait(k_full + st, kph, abort_flag))) break;
+            tc_fence_after();
+            const uint32_t k_addr = smem_u32(k_buf + st * k_bytes);
+            const uint32_t d_tmem = tmem_base + ab * H;
+            for (int ks = 0; ks < ksteps; ++ks) {
+              const int pn = ks >> 2, off = (ks & 3) * 32;
+              mma<DT>(d_tmem, desc_k_sw128(k_addr + pn * (kTokTileM * 128) + off),
+                      desc_k_sw128(q_addr + pn * (H * 128) + off), idesc, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(k_empty + st);
+            mma_commit(acc_full + ab);
           }
-          mma_commit(k_empty + st);
-          mma_commit(acc_full + ab);
+          if (++g == kTokIssuers) g = 0;
           if (++st == p.stages) { st = 0; kph ^= 1; }
           if (++ab == kTokAcc) { ab = 0; aph ^= 1; }
         }
         if (ok) mma_commit(q_empty + qb);
       }
-      mma_commit(drain);
-      mbar_drain(drain, 0);
+      mma_commit(drain + me);
+      mbar_drain(drain + me, 0);
     }
-  } else if (warp >= kTokScorerBase && warp < kTokScorerBase + kTokScorerWarps) {
-    // ------------------------------------------------------------ scorer
+  } else if (warp >= kTokScorerBase && warp < kTokScorerBase + kTokScorerWarps * kTokScoreGroups) {
+    // ------------------------------------------------------------ scorers
+    const int grp = (warp - kTokScorerBase) / kTokScorerWarps;   // takes tiles g with g % groups == grp
     const int quarter = warp & 3;
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     const int bshift = __ffs(p.B) - 1;
-    int ab = 0;
+    int ab = 0, g = 0;
     uint32_t aph = 0;
     bool ok = true;
     for (int64_t j = 0; ok && j < njobs; ++j) {
@@ -289,53 +310,68 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
               mbar_wait(cand_empty + cb, static_cast<uint32_t>(((j >> 1) & 1) ^ 1), abort_flag);
       }
       if (!(ok = __shfl_sync(0xffffffffu, okl, 0) != 0)) break;
-      const TokJob& J = jobs[slot];
+      TokJob& J = jobs[slot];
       const int ntiles = J.ntiles;
       uint32_t* cj = cand + cb * p.max_cand;
-      float ksc = 1.f;
+      uint32_t lo = 0xFFFFFFFFu, hi = 0u, nv = 0u;
       for (int i = 0; i < ntiles; ++i) {
-        if (lane == 0) okl = mbar_wait(acc_full + ab, aph, abort_flag);
-        if (!(ok = __shfl_sync(0xffffffffu, okl, 0) != 0)) break;
-        tc_fence_after();
-        const int c = i * kTokTileM + quarter * 32 + lane;        // candidate position
-        const int slot_b = c >> bshift;
-        const int s = slot_b < J.nblk ? (J.blk[slot_b] << bshift) + (c & (p.B - 1)) : p.L;
-        const bool valid = s < J.n;
-        if (DT == DT_E4M3 && valid) ksc = __ldg(p.k_scale + static_cast<int64_t>(J.b) * p.L + s);
-        float acc = 0.f;
-        if (H >= 32) {
-          // all TMEM loads of the row first, one wait, then four independent
-          // accumulation chains over float4 weight reads
-          uint32_t v[H];
+        if (g == grp) {
+          if (lane == 0) okl = mbar_wait(acc_full + ab, aph, abort_flag);
+          if (!(ok = __shfl_sync(0xffffffffu, okl, 0) != 0)) break;
+          tc_fence_after();
+          const int c = i * kTokTileM + quarter * 32 + lane;        // candidate position
+          const int slot_b = c >> bshift;
+          const int s = slot_b < J.nblk ? (J.blk[slot_b] << bshift) + (c & (p.B - 1)) : p.L;
+          const bool valid = s < J.n;
+          float ksc = 1.f;
+          if (DT == DT_E4M3 && valid) ksc = __ldg(p.k_scale + static_cast<int64_t>(J.b) * p.L + s);
+          float acc = 0.f;
+          if (H >= 32) {
+            // all TMEM loads of the row first, one wait, then four independent
+            // accumulation chains over float4 weight reads
+            uint32_t v[H];
 #pragma unroll
-          for (int c0 = 0; c0 < H; c0 += 32) tmem_ld32(t_lane + ab * H + c0, *reinterpret_cast<uint32_t(*)[32]>(v + c0));
-          tmem_wait_ld();
-          float a4[4] = {0.f, 0.f, 0.f, 0.f};
-          const float4* w4 = reinterpret_cast<const float4*>(J.w);
+            for (int c0 = 0; c0 < H; c0 += 32)
+              tmem_ld32(t_lane + ab * H + c0, *reinterpret_cast<uint32_t(*)[32]>(v + c0));
+            tmem_wait_ld();
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+            const float4* w4 = reinterpret_cast<const float4*>(J.w);
 #pragma unroll
-          for (int e = 0; e < H / 4; ++e) {
-            const float4 wv = w4[e];
-            a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * e + 0]), 0.f), a4[0]);
-            a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * e + 1]), 0.f), a4[1]);
-            a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * e + 2]), 0.f), a4[2]);
-            a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * e + 3]), 0.f), a4[3]);
+            for (int e = 0; e < H / 4; ++e) {
+              const float4 wv = w4[e];
+              a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * e + 0]), 0.f), a4[0]);
+              a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * e + 1]), 0.f), a4[1]);
+              a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * e + 2]), 0.f), a4[2]);
+              a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * e + 3]), 0.f), a4[3]);
+            }
+            acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+          } else {
+            uint32_t v[16];
+            tmem_ld16(t_lane + ab * H, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc = fmaf(J.w[e], fmaxf(__uint_as_float(v[e]), 0.f), acc);
           }
-          acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-        } else {
-          uint32_t v[16];
-          tmem_ld16(t_lane + ab * H, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) acc = fmaf(J.w[e], fmaxf(__uint_as_float(v[e]), 0.f), acc);
+          if (DT == DT_E4M3) acc *= J.qsc * ksc;
+          const uint32_t key = valid ? float_key(acc) : 0u;
+          cj[c] = key;
+          if (valid) { lo = min(lo, key); hi = max(hi, key); ++nv; }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty + ab);
         }
-        if (DT == DT_E4M3) acc *= J.qsc * ksc;
-        cj[c] = valid ? float_key(acc) : 0u;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty + ab);
+        if (++g == kTokScoreGroups) g = 0;
         if (++ab == kTokAcc) { ab = 0; aph ^= 1; }
       }
       if (!ok) break;
+      lo = __reduce_min_sync(0xffffffffu, lo);
+      hi = __reduce_max_sync(0xffffffffu, hi);
+      nv = __reduce_add_sync(0xffffffffu, nv);
+      if (lane == 0 && nv > 0) {
+        atomicMin(&J.kmin, lo);
+        atomicMax(&J.kmax, hi);
+        atomicAdd(&J.nvalid, nv);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(cand_full + cb);
     }
@@ -359,8 +395,15 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
         oi[slot_out] = (J.blk[i >> bshift] << bshift) + (i & (p.B - 1));
         if (os) os[slot_out] = key_float(key);
       };
-      const uint32_t nv = block_topk<decltype(key_at), decltype(emit), SelGrp>(
-          key_at, ncand, static_cast<uint32_t>(p.top_k), emit, *sel);
+      const uint32_t nv = J.nvalid;
+      if (nv <= static_cast<uint32_t>(p.top_k)) {
+        emit_at_least<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, 1u, emit, *sel);
+      } else if (!two_pass_topk<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, static_cast<uint32_t>(p.top_k),
+                                                                         emit, *sel, bin_key, bin_pos, bin_count,
+                                                                         kTokBinCap, J.kmin, J.kmax)) {
+        block_topk_range<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, static_cast<uint32_t>(p.top_k),
+                                                                   emit, *sel, J.kmin, J.kmax, nv);
+      }
       for (int i = static_cast<int>(nv) + stid; i < p.top_k; i += SelGrp::size()) {
         oi[i] = -1;
         if (os) os[i] = -__int_as_float(0x7f800000);
@@ -383,8 +426,8 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
 inline size_t token_smem_bytes(int row_bytes, int H, int stages, int max_cand) {
   return 1024 + 2 * static_cast<size_t>(H) * row_bytes + static_cast<size_t>(stages) * kTokTileM * row_bytes +
          2 * static_cast<size_t>(max_cand) * 4 + kTokJobs * sizeof(TokJob) + sizeof(SelectSmem) +
-         4 * kTokMaxBitmapWords + 8 +
-         8 * (2 * stages + 4 + 2 * kTokAcc + 2 * kTokJobs + 4 + 1) + 16;
+         4 * kTokMaxBitmapWords + 8 * kTokBinCap + 4 + 8 +
+         8 * (2 * stages + 4 + 2 * kTokAcc + 2 * kTokJobs + 4 + kTokIssuers) + 16;
 }
 
 }  // namespace hisa
