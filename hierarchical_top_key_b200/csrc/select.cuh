@@ -359,6 +359,134 @@ __device__ bool two_pass_topk(KeyAt key_at, int n, uint32_t k, Emit emit, Select
   return true;
 }
 
+// Block-wide exclusive prefix sums of two per-thread counts (thread order);
+// totals go to *ta and *tb.
+template <class Grp>
+__device__ __forceinline__ void block_scan2(uint32_t a, uint32_t b, uint32_t* pa, uint32_t* pb, uint32_t* ta,
+                                            uint32_t* tb, SelectSmem& sm) {
+  const int lane = Grp::tid() & 31, wid = Grp::tid() >> 5, nw = Grp::size() >> 5;
+  uint32_t ia = a, ib = b;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t oa = __shfl_up_sync(0xffffffffu, ia, off);
+    const uint32_t ob = __shfl_up_sync(0xffffffffu, ib, off);
+    if (lane >= off) { ia += oa; ib += ob; }
+  }
+  if (lane == 31) { sm.warp_cnt[wid] = ia; sm.hist[wid] = ib; }   // hist is free here: the bins are consumed
+  Grp::sync();
+  uint32_t wa = 0, wb = 0, sa = 0, sb = 0;
+  for (int i = 0; i < nw; ++i) {
+    const uint32_t ca = sm.warp_cnt[i], cb = sm.hist[i];
+    if (i < wid) { wa += ca; wb += cb; }
+    sa += ca;
+    sb += cb;
+  }
+  Grp::sync();
+  *pa = wa + ia - a;
+  *pb = wb + ib - b;
+  *ta = sa;
+  *tb = sb;
+}
+
+// Like two_pass_topk, for keys cheap to read three times (shared memory):
+// thread i owns positions i, i+size, ...; pass 2 only counts, one block scan
+// gives every thread its output offsets, pass 3 writes.  No returning atomics
+// or per-element shuffles.
+template <class KeyAt, class Emit, class Grp>
+__device__ bool scan_topk(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem& sm, uint32_t* buf_key,
+                          int32_t* buf_pos, int cap, uint32_t kmin, uint32_t kmax) {
+  const int lane = Grp::tid() & 31;
+  const int nbins = kDigitBins;
+  const float smin = key_float(kmin), smax = key_float(kmax);
+  float scale = smax > smin ? static_cast<float>(nbins) / (smax - smin) : 0.f;
+  if (!(scale < 1e30f)) scale = 0.f;
+  auto bin_of = [&](uint32_t key) -> uint32_t {
+    const int b = static_cast<int>((key_float(key) - smin) * scale);
+    return static_cast<uint32_t>(min(max(b, 0), nbins - 1));
+  };
+  for (int i = Grp::tid(); i < nbins; i += Grp::size()) sm.hist[i] = 0;
+  Grp::sync();
+  for (int i = Grp::tid(); i < n; i += Grp::size()) {
+    const uint32_t key = key_at(i);
+    if (key != 0u) atomicAdd(&sm.hist[bin_of(key)], 1u);
+  }
+  Grp::sync();
+  uint32_t remaining = k;
+  {
+    const int nt = Grp::size();
+    const int per = nbins >= nt ? nbins / nt : 1;
+    const int top = nbins - 1 - Grp::tid() * per;
+    uint32_t t = 0;
+    for (int j = 0; j < per; ++j)
+      if (top - j >= 0) t += sm.hist[top - j];
+    uint32_t incl = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) sm.warp_cnt[Grp::tid() >> 5] = incl;
+    Grp::sync();
+    uint32_t woff = 0;
+    for (int wi = 0; wi < (Grp::tid() >> 5); ++wi) woff += sm.warp_cnt[wi];
+    incl += woff;
+    const uint32_t excl = incl - t;
+    if (t > 0 && excl < remaining && incl >= remaining) {
+      uint32_t c = excl;
+      for (int j = 0; j < per; ++j) {
+        const uint32_t h = sm.hist[top - j];
+        if (c + h >= remaining) { sm.digit = top - j; sm.above = c; sm.at_digit = h; break; }
+        c += h;
+      }
+    }
+  }
+  Grp::sync();
+  const uint32_t D = sm.digit, above = sm.above, n_eq = sm.at_digit;
+  remaining -= above;
+  const bool take_bin = n_eq == remaining;
+  if (!take_bin && n_eq > static_cast<uint32_t>(cap)) return false;
+  // pass 2: count what this thread emits and buffers
+  uint32_t cg = 0, ce = 0;
+  for (int i = Grp::tid(); i < n; i += Grp::size()) {
+    const uint32_t key = key_at(i);
+    if (key == 0u) continue;
+    const uint32_t b = bin_of(key);
+    cg += (b > D || (take_bin && b == D)) ? 1u : 0u;
+    ce += (!take_bin && b == D) ? 1u : 0u;
+  }
+  uint32_t og, oe, tg, te;
+  block_scan2<Grp>(cg, ce, &og, &oe, &tg, &te, sm);
+  // pass 3: write
+  for (int i = Grp::tid(); i < n; i += Grp::size()) {
+    const uint32_t key = key_at(i);
+    if (key == 0u) continue;
+    const uint32_t b = bin_of(key);
+    if (b > D || (take_bin && b == D)) {
+      emit(og++, i, key);
+    } else if (b == D) {
+      buf_key[oe] = key;
+      buf_pos[oe] = i;
+      ++oe;
+    }
+  }
+  Grp::sync();
+  if (take_bin) return true;
+  // the remaining places among the buffered keys: larger key first, then lower position
+  const int nb = static_cast<int>(n_eq);
+  for (int e = Grp::tid(); e < nb; e += Grp::size()) {
+    const uint32_t ke = buf_key[e];
+    const int pe = buf_pos[e];
+    uint32_t rank = 0;
+    for (int f = 0; f < nb; ++f) {
+      const uint32_t kf = buf_key[f];
+      rank += (kf > ke || (kf == ke && buf_pos[f] < pe)) ? 1u : 0u;
+    }
+    if (rank < remaining) emit(above + rank, pe, ke);
+  }
+  Grp::sync();
+  return true;
+}
+
 constexpr int kTwoPassCap = 4096;
 
 struct TwoPassSmem {

@@ -18,7 +18,7 @@
 //   warps 4..11  scorers, two groups of four on alternate tiles: TMEM ->
 //                weighted ReLU sum -> candidate keys in smem, plus each
 //                job's key range and valid count
-//   warps 12..15 selector: two-pass radix top-k over the candidate keys
+//   warps 12..15 selector: histogram + counting-scan top-k over the candidate keys
 // Rings: job slots (4), q buffers (2), key stages, TMEM accumulators (8 x H
 // columns), candidate buffers (2).  Blocks are sorted ascending so candidate
 // position order is key order, which makes ties resolve to the lower key.
@@ -398,9 +398,9 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
       const uint32_t nv = J.nvalid;
       if (nv <= static_cast<uint32_t>(p.top_k)) {
         emit_at_least<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, 1u, emit, *sel);
-      } else if (!two_pass_topk<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, static_cast<uint32_t>(p.top_k),
-                                                                         emit, *sel, bin_key, bin_pos, bin_count,
-                                                                         kTokBinCap, J.kmin, J.kmax)) {
+      } else if (!scan_topk<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, static_cast<uint32_t>(p.top_k),
+                                                                     emit, *sel, bin_key, bin_pos, kTokBinCap, J.kmin,
+                                                                     J.kmax)) {
         block_topk_range<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, static_cast<uint32_t>(p.top_k),
                                                                    emit, *sel, J.kmin, J.kmax, nv);
       }
