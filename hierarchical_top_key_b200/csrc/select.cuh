@@ -391,32 +391,38 @@ __device__ __forceinline__ void block_scan2(uint32_t a, uint32_t b, uint32_t* pa
 // Like two_pass_topk, for keys cheap to read three times (shared memory):
 // thread i owns positions i, i+size, ...; pass 2 only counts, one block scan
 // gives every thread its output offsets, pass 3 writes.  No returning atomics
-// or per-element shuffles.
+// or per-element shuffles; loops are unrolled four-wide so the loads of four
+// positions are in flight together.  `nbins` (<= kDigitBins) linear bins.
 template <class KeyAt, class Emit, class Grp>
 __device__ bool scan_topk(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem& sm, uint32_t* buf_key,
-                          int32_t* buf_pos, int cap, uint32_t kmin, uint32_t kmax) {
+                          int32_t* buf_pos, int cap, uint32_t kmin, uint32_t kmax, int nbins = kDigitBins) {
   const int lane = Grp::tid() & 31;
-  const int nbins = kDigitBins;
+  const int tid = Grp::tid(), nt = Grp::size();
   const float smin = key_float(kmin), smax = key_float(kmax);
   float scale = smax > smin ? static_cast<float>(nbins) / (smax - smin) : 0.f;
   if (!(scale < 1e30f)) scale = 0.f;
+  const int top_bin = nbins - 1;
   auto bin_of = [&](uint32_t key) -> uint32_t {
-    const int b = static_cast<int>((key_float(key) - smin) * scale);
-    return static_cast<uint32_t>(min(max(b, 0), nbins - 1));
+    return static_cast<uint32_t>(min(__float2int_rz((key_float(key) - smin) * scale), top_bin));
   };
-  for (int i = Grp::tid(); i < nbins; i += Grp::size()) sm.hist[i] = 0;
+  for (int i = tid; i < nbins; i += nt) sm.hist[i] = 0;
   Grp::sync();
-  for (int i = Grp::tid(); i < n; i += Grp::size()) {
-    const uint32_t key = key_at(i);
-    if (key != 0u) atomicAdd(&sm.hist[bin_of(key)], 1u);
+  // pass 1: histogram
+  for (int base = tid; base < n; base += 4 * nt) {
+    uint32_t kv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) kv[u] = base + u * nt < n ? key_at(base + u * nt) : 0u;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (kv[u] != 0u) atomicAdd(&sm.hist[bin_of(kv[u])], 1u);
   }
   Grp::sync();
   uint32_t remaining = k;
   {
-    const int nt = Grp::size();
     const int per = nbins >= nt ? nbins / nt : 1;
-    const int top = nbins - 1 - Grp::tid() * per;
+    const int top = nbins - 1 - tid * per;
     uint32_t t = 0;
+#pragma unroll 8
     for (int j = 0; j < per; ++j)
       if (top - j >= 0) t += sm.hist[top - j];
     uint32_t incl = t;
@@ -425,10 +431,10 @@ __device__ bool scan_topk(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem
       const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
       if (lane >= off) incl += o;
     }
-    if (lane == 31) sm.warp_cnt[Grp::tid() >> 5] = incl;
+    if (lane == 31) sm.warp_cnt[tid >> 5] = incl;
     Grp::sync();
     uint32_t woff = 0;
-    for (int wi = 0; wi < (Grp::tid() >> 5); ++wi) woff += sm.warp_cnt[wi];
+    for (int wi = 0; wi < (tid >> 5); ++wi) woff += sm.warp_cnt[wi];
     incl += woff;
     const uint32_t excl = incl - t;
     if (t > 0 && excl < remaining && incl >= remaining) {
@@ -445,35 +451,46 @@ __device__ bool scan_topk(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem
   remaining -= above;
   const bool take_bin = n_eq == remaining;
   if (!take_bin && n_eq > static_cast<uint32_t>(cap)) return false;
+  const uint32_t gt_floor = take_bin ? D : D + 1;        // bins >= gt_floor are emitted outright
   // pass 2: count what this thread emits and buffers
   uint32_t cg = 0, ce = 0;
-  for (int i = Grp::tid(); i < n; i += Grp::size()) {
-    const uint32_t key = key_at(i);
-    if (key == 0u) continue;
-    const uint32_t b = bin_of(key);
-    cg += (b > D || (take_bin && b == D)) ? 1u : 0u;
-    ce += (!take_bin && b == D) ? 1u : 0u;
+  for (int base = tid; base < n; base += 4 * nt) {
+    uint32_t kv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) kv[u] = base + u * nt < n ? key_at(base + u * nt) : 0u;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (kv[u] == 0u) continue;
+      const uint32_t b = bin_of(kv[u]);
+      cg += b >= gt_floor ? 1u : 0u;
+      ce += b == D && !take_bin ? 1u : 0u;
+    }
   }
   uint32_t og, oe, tg, te;
   block_scan2<Grp>(cg, ce, &og, &oe, &tg, &te, sm);
   // pass 3: write
-  for (int i = Grp::tid(); i < n; i += Grp::size()) {
-    const uint32_t key = key_at(i);
-    if (key == 0u) continue;
-    const uint32_t b = bin_of(key);
-    if (b > D || (take_bin && b == D)) {
-      emit(og++, i, key);
-    } else if (b == D) {
-      buf_key[oe] = key;
-      buf_pos[oe] = i;
-      ++oe;
+  for (int base = tid; base < n; base += 4 * nt) {
+    uint32_t kv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) kv[u] = base + u * nt < n ? key_at(base + u * nt) : 0u;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (kv[u] == 0u) continue;
+      const uint32_t b = bin_of(kv[u]);
+      if (b >= gt_floor) {
+        emit(og++, base + u * nt, kv[u]);
+      } else if (b == D) {
+        buf_key[oe] = kv[u];
+        buf_pos[oe] = base + u * nt;
+        ++oe;
+      }
     }
   }
   Grp::sync();
   if (take_bin) return true;
   // the remaining places among the buffered keys: larger key first, then lower position
   const int nb = static_cast<int>(n_eq);
-  for (int e = Grp::tid(); e < nb; e += Grp::size()) {
+  for (int e = tid; e < nb; e += nt) {
     const uint32_t ke = buf_key[e];
     const int pe = buf_pos[e];
     uint32_t rank = 0;

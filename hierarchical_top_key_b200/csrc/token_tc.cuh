@@ -389,22 +389,49 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
       const int ncand = J.ntiles * kTokTileM;
       int32_t* oi = p.out_idx + J.row * p.top_k;
       float* os = p.out_score ? p.out_score + J.row * p.top_k : nullptr;
-      auto key_at = [&](int i) { return cj[i]; };
       const int bshift = __ffs(p.B) - 1;
+      // indices are staged in shared memory (the selection's histogram space,
+      // free once offsets are known) and written out coalesced; with scores
+      // requested or k above the staging room they go straight to global
+      const bool staged = os == nullptr && p.top_k <= kDigitBins;
+      int32_t* stage = reinterpret_cast<int32_t*>(sel->hist);
+      auto key_at = [&](int i) { return cj[i]; };
       auto emit = [&](uint32_t slot_out, int i, uint32_t key) {
-        oi[slot_out] = (J.blk[i >> bshift] << bshift) + (i & (p.B - 1));
-        if (os) os[slot_out] = key_float(key);
+        const int32_t s_idx = (J.blk[i >> bshift] << bshift) + (i & (p.B - 1));
+        if (staged) {
+          stage[slot_out] = s_idx;
+        } else {
+          oi[slot_out] = s_idx;
+          if (os) os[slot_out] = key_float(key);
+        }
       };
       const uint32_t nv = J.nvalid;
+      uint32_t filled = 0;
       if (nv <= static_cast<uint32_t>(p.top_k)) {
         emit_at_least<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, 1u, emit, *sel);
-      } else if (!scan_topk<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, static_cast<uint32_t>(p.top_k),
+        filled = nv;
+      } else if (scan_topk<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, static_cast<uint32_t>(p.top_k),
                                                                      emit, *sel, bin_key, bin_pos, kTokBinCap, J.kmin,
-                                                                     J.kmax)) {
+                                                                     J.kmax, 1024)) {
+        filled = static_cast<uint32_t>(p.top_k);
+      } else {
         block_topk_range<decltype(key_at), decltype(emit), SelGrp>(key_at, ncand, static_cast<uint32_t>(p.top_k),
                                                                    emit, *sel, J.kmin, J.kmax, nv);
+        filled = static_cast<uint32_t>(p.top_k);
       }
-      for (int i = static_cast<int>(nv) + stid; i < p.top_k; i += SelGrp::size()) {
+      SelGrp::sync();
+      if (staged) {
+        if ((p.top_k & 3) == 0) {
+          const int4* st4 = reinterpret_cast<const int4*>(stage);
+          int4* o4 = reinterpret_cast<int4*>(oi);
+          for (int i = stid; i < static_cast<int>(filled) / 4; i += SelGrp::size()) o4[i] = st4[i];
+          for (int i = (static_cast<int>(filled) & ~3) + stid; i < static_cast<int>(filled); i += SelGrp::size())
+            oi[i] = stage[i];
+        } else {
+          for (int i = stid; i < static_cast<int>(filled); i += SelGrp::size()) oi[i] = stage[i];
+        }
+      }
+      for (int i = static_cast<int>(filled) + stid; i < p.top_k; i += SelGrp::size()) {
         oi[i] = -1;
         if (os) os[i] = -__int_as_float(0x7f800000);
       }
