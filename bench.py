@@ -36,15 +36,16 @@ DEFAULT_WORKLOAD = "prefill_32k"
 FLOP_PER_PAIR_PER_HEAD_DIM = 2          # one multiply-add per (head, feature) per (query, key) pair
 L2_FLUSH_BYTES = 256 << 20               # larger than the 126 MB L2
 
-# DRAM bytes per launch of the refinement kernel from an ncu capture of the
-# same build and workload; None when the kernel changed since the capture.
-NCU_TRAFFIC = {}
+# DRAM bytes (read + write) per launch of the refinement kernel from an ncu
+# capture of the same kernel and workload (see profiles/); a workload missing
+# here reports null.
+NCU_TRAFFIC = {"prefill_32k": 558091776 + 238973440}
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
@@ -102,7 +103,8 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.5)              # let the sampler start before the timed region
         except OSError:
             self.proc = None
         return self

@@ -401,9 +401,15 @@ __device__ bool scan_topk(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem
   const float smin = key_float(kmin), smax = key_float(kmax);
   float scale = smax > smin ? static_cast<float>(nbins) / (smax - smin) : 0.f;
   if (!(scale < 1e30f)) scale = 0.f;
-  const int top_bin = nbins - 1;
+  const uint32_t top_bin = static_cast<uint32_t>(nbins - 1);
+  // bin = nearest integer to (score - smin) * scale, by adding 2^23 and reading
+  // the low mantissa bits (exact for values below 2^22, monotone in the score);
+  // this keeps the float-to-int conversion pipe free
+  const float bias = 8388608.0f - smin * scale;
   auto bin_of = [&](uint32_t key) -> uint32_t {
-    return static_cast<uint32_t>(min(__float2int_rz((key_float(key) - smin) * scale), top_bin));
+    // signed difference: a value rounded just below 2^23 gives -1 -> bin 0
+    const int b = static_cast<int>(__float_as_uint(fmaf(key_float(key), scale, bias)) - 0x4B000000u);
+    return min(static_cast<uint32_t>(max(b, 0)), top_bin);
   };
   for (int i = tid; i < nbins; i += nt) sm.hist[i] = 0;
   Grp::sync();
