@@ -214,6 +214,29 @@ def workload_config(wl, fp8):
             "top_k": wl.top_k, "l2": "flushed between steps (256 MiB write, outside the timed events)"}
 
 
+# ------------------------------------------------------------------ ranks
+
+
+def replica_seed(seed: int, rank: int) -> int:
+    """Each rank runs its own independent replica of the workload."""
+    return seed + rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest of every rank's `x` (the job is as slow as its slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (ms_max / 1000.0)
+
+
 # ------------------------------------------------------------------ our arm
 
 
@@ -234,7 +257,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     wl = synthetic.WORKLOADS[args.workload]
-    inp = synthetic.generate(wl, args.seed + rank)
+    inp = synthetic.generate(wl, replica_seed(args.seed, rank))
     hb.load()
     stream = torch.cuda.current_stream()
     fp8 = args.fp8
@@ -310,12 +333,9 @@ def main():
     step_ms = [a.elapsed_time(b) for a, b in step_evs]
     stage_ms = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(3)] for e in stage_evs])
     ms = float(np.mean(step_ms))
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, world, dev)
     queries = wl.batch * wl.num_queries
-    value = queries * world / (ms_max / 1000.0)
+    value = job_rate(queries, world, ms_max)
 
     # ---- flat DSA indexer on the same inputs
     flat = None
@@ -374,12 +394,9 @@ def main():
             b.record(stream)
             evs.append((a, b))
         barrier()
-        em = float(np.mean([a.elapsed_time(b) for a, b in evs]))
-        et = torch.tensor([em], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(et, op=dist.ReduceOp.MAX)
-        e2e = {"value": queries * world / (float(et.item()) / 1000.0), "unit": "queries/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": float(et.item())}
+        em = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])), world, dev)
+        e2e = {"value": job_rate(queries, world, em), "unit": "queries/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": em}
 
     # ---- roofline of the dominant kernel (the fused refinement stage)
     peaks = load_peaks()

@@ -53,6 +53,7 @@ _SIGS = {
     "dsa_flat_indexer_topk": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t, _P],
     "hisa_workspace_size": [ctypes.c_int32, ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)],
     "hisa_get_status": [_P],
+    "hisa_selftest_wait_timeout": [ctypes.c_uint64, _P],
     "hisa_status_string": [ctypes.c_int],
     "hisa_last_error": [],
 }

@@ -328,6 +328,19 @@ hisa_status check_indexer_ptrs(const hisa_shape* s, const void* q, const float* 
 
 }  // namespace
 
+// Self-test of the bounded-wait path: one thread waits on a barrier that no
+// one arrives at; the wait gives up after `limit_ns` and records the timeout.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sm100::fence_barrier_init();
+    (void)sm100::mbar_wait(&bar, 0, &abort_flag, limit_ns);
+  }
+}
+
 // =================================================================== C ABI
 
 extern "C" {
@@ -345,6 +358,12 @@ const char* hisa_status_string(hisa_status st) {
 }
 
 const char* hisa_last_error(void) { return g_last_error; }
+
+hisa_status hisa_selftest_wait_timeout(uint64_t limit_ns, hisa_stream stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return fail(HISA_ERR_INVALID_ARG, "limit_ns must be in (0, 10 s]");
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return launch_check("selftest_wait_kernel");
+}
 
 hisa_status hisa_get_status(hisa_stream stream) {
   hisa_status e = cuda_check(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)), "stream sync");

@@ -225,6 +225,14 @@ HISA_API hisa_status hisa_workspace_size(int32_t op, const hisa_shape* shape,
  * call); HISA_ERR_CUDA if the synchronisation itself failed. */
 HISA_API hisa_status hisa_get_status(hisa_stream stream);
 
+/* Self-test of failure detection: launches one thread that waits, with the
+ * same bounded wait the tensor-core kernels use, on a barrier that nothing
+ * ever completes; after limit_ns (0 < limit_ns <= 10 s) it gives up and
+ * records HISA_ERR_TIMEOUT in the device status word, which the next
+ * hisa_get_status() returns (and clears).  Faults nothing: the context stays
+ * usable. */
+HISA_API hisa_status hisa_selftest_wait_timeout(uint64_t limit_ns, hisa_stream stream);
+
 /* Static description of a status code. */
 HISA_API const char* hisa_status_string(hisa_status status);
 
