@@ -285,11 +285,10 @@ hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc
   p.nb = static_cast<int>(num_blocks(s));
   p.max_cand = static_cast<int>(ceil_div(static_cast<int64_t>(s->top_m) * s->block_size, kTokTileM) * kTokTileM);
   p.w = w; p.n_visible = nvis; p.block_idx = bidx; p.q_scale = qsc; p.k_scale = ksc; p.out_idx = oi; p.out_score = os;
-  const size_t fixed = token_smem_bytes(rb, H, 0, p.max_cand) + 16 * 8;
-  const size_t kb = static_cast<size_t>(kTokTileM) * rb;
-  if (fixed + 2 * kb > kSmemBudget)
+  if (token_smem_bytes(rb, H, 2, p.max_cand) > kSmemBudget)
     return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size too large for the on-chip candidate buffers");
-  p.stages = static_cast<int>(std::min<size_t>(6, (kSmemBudget - fixed) / kb));
+  p.stages = 2;
+  while (p.stages < 6 && token_smem_bytes(rb, H, p.stages + 1, p.max_cand) <= kSmemBudget) ++p.stages;
   const size_t smem = token_smem_bytes(rb, H, p.stages, p.max_cand);
   CUtensorMap qm, km;
   hisa_status e = tensor_map_2d(&qm, q, s->dtype, static_cast<uint64_t>(p.rows) * H, s->head_dim, H);

@@ -81,6 +81,42 @@ __device__ void emit_at_least(KeyAt key_at, int n, uint32_t T, Emit emit, Select
   Grp::sync();
 }
 
+// The bin holding the k-th place of sm.hist[0, nbins) counted from the top:
+// sets sm.digit, sm.above (elements in higher bins) and sm.at_digit (the
+// bin's count).  Each thread sums a run of bins, one block scan orders the
+// runs, and the thread whose run crosses k walks it.  Ends with a sync.
+template <class Grp>
+__device__ __forceinline__ void bin_search(SelectSmem& sm, int nbins, uint32_t k) {
+  const int tid = Grp::tid(), nt = Grp::size(), lane = tid & 31;
+  const int per = (nbins + nt - 1) / nt;             // every bin belongs to one thread's run
+  const int top = nbins - 1 - tid * per;
+  uint32_t t = 0;
+#pragma unroll 8
+  for (int j = 0; j < per; ++j)
+    if (top - j >= 0) t += sm.hist[top - j];
+  uint32_t incl = t;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) sm.warp_cnt[tid >> 5] = incl;
+  Grp::sync();
+  uint32_t woff = 0;
+  for (int wi = 0; wi < (tid >> 5); ++wi) woff += sm.warp_cnt[wi];
+  incl += woff;
+  const uint32_t excl = incl - t;
+  if (t > 0 && excl < k && incl >= k) {
+    uint32_t c = excl;
+    for (int j = 0; j < per && top - j >= 0; ++j) {
+      const uint32_t h = sm.hist[top - j];
+      if (c + h >= k) { sm.digit = top - j; sm.above = c; sm.at_digit = h; break; }
+      c += h;
+    }
+  }
+  Grp::sync();
+}
+
 // Top-k of the keys at positions [0, n) (key 0 = absent): calls
 // Emit(slot, position, key) exactly once for each slot 0..min(k, valid)-1 and
 // returns the number of valid keys.  Ties at the k-th place go to the lower
@@ -139,38 +175,7 @@ __device__ uint32_t block_topk_range(KeyAt key_at, int n, uint32_t k, Emit emit,
       if (act) atomicAdd(&sm.hist[(key >> shift) & dmask], 1u);
     }
     Grp::sync();
-    {
-      // block-parallel search from the top bin: thread i owns bins
-      // [nbins-1-i*per, nbins-(i+1)*per]; exclusive prefix of the per-thread
-      // sums across the group finds the bin holding the `remaining`-th key
-      const int nt = Grp::size();
-      const int per = nbins >= nt ? nbins / nt : 1;
-      const int top = nbins - 1 - Grp::tid() * per;
-      uint32_t t = 0;
-      for (int j = 0; j < per; ++j)
-        if (top - j >= 0) t += sm.hist[top - j];
-      uint32_t incl = t;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-      }
-      if (lane == 31) sm.warp_cnt[Grp::tid() >> 5] = incl;
-      Grp::sync();
-      uint32_t woff = 0;
-      for (int wi = 0; wi < (Grp::tid() >> 5); ++wi) woff += sm.warp_cnt[wi];
-      incl += woff;
-      const uint32_t excl = incl - t;
-      if (t > 0 && excl < remaining && incl >= remaining) {
-        uint32_t c = excl;
-        for (int j = 0; j < per; ++j) {
-          const uint32_t h = sm.hist[top - j];
-          if (c + h >= remaining) { sm.digit = top - j; sm.above = c; sm.at_digit = h; break; }
-          c += h;
-        }
-      }
-    }
-    Grp::sync();
+    bin_search<Grp>(sm, nbins, remaining);
     prefix |= sm.digit << shift;
     remaining -= sm.above;
     n_eq = sm.at_digit;
@@ -256,35 +261,7 @@ __device__ bool two_pass_topk(KeyAt key_at, int n, uint32_t k, Emit emit, Select
   }
   Grp::sync();
   uint32_t remaining = k;
-  {
-    const int nt = Grp::size();
-    const int per = nbins >= nt ? nbins / nt : 1;
-    const int top = nbins - 1 - Grp::tid() * per;
-    uint32_t t = 0;
-    for (int j = 0; j < per; ++j)
-      if (top - j >= 0) t += sm.hist[top - j];
-    uint32_t incl = t;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
-    }
-    if (lane == 31) sm.warp_cnt[Grp::tid() >> 5] = incl;
-    Grp::sync();
-    uint32_t woff = 0;
-    for (int wi = 0; wi < (Grp::tid() >> 5); ++wi) woff += sm.warp_cnt[wi];
-    incl += woff;
-    const uint32_t excl = incl - t;
-    if (t > 0 && excl < remaining && incl >= remaining) {
-      uint32_t c = excl;
-      for (int j = 0; j < per; ++j) {
-        const uint32_t h = sm.hist[top - j];
-        if (c + h >= remaining) { sm.digit = top - j; sm.above = c; sm.at_digit = h; break; }
-        c += h;
-      }
-    }
-  }
-  Grp::sync();
+  bin_search<Grp>(sm, nbins, remaining);
   const uint32_t D = sm.digit, above = sm.above, n_eq = sm.at_digit;
   remaining -= above;
   Grp::sync();
@@ -424,35 +401,7 @@ __device__ bool scan_topk(KeyAt key_at, int n, uint32_t k, Emit emit, SelectSmem
   }
   Grp::sync();
   uint32_t remaining = k;
-  {
-    const int per = nbins >= nt ? nbins / nt : 1;
-    const int top = nbins - 1 - tid * per;
-    uint32_t t = 0;
-#pragma unroll 8
-    for (int j = 0; j < per; ++j)
-      if (top - j >= 0) t += sm.hist[top - j];
-    uint32_t incl = t;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
-    }
-    if (lane == 31) sm.warp_cnt[tid >> 5] = incl;
-    Grp::sync();
-    uint32_t woff = 0;
-    for (int wi = 0; wi < (tid >> 5); ++wi) woff += sm.warp_cnt[wi];
-    incl += woff;
-    const uint32_t excl = incl - t;
-    if (t > 0 && excl < remaining && incl >= remaining) {
-      uint32_t c = excl;
-      for (int j = 0; j < per; ++j) {
-        const uint32_t h = sm.hist[top - j];
-        if (c + h >= remaining) { sm.digit = top - j; sm.above = c; sm.at_digit = h; break; }
-        c += h;
-      }
-    }
-  }
-  Grp::sync();
+  bin_search<Grp>(sm, nbins, remaining);
   const uint32_t D = sm.digit, above = sm.above, n_eq = sm.at_digit;
   remaining -= above;
   const bool take_bin = n_eq == remaining;

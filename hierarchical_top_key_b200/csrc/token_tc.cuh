@@ -97,8 +97,14 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
   int32_t* bin_pos = reinterpret_cast<int32_t*>(bin_key + kTokBinCap);         // [kTokBinCap]
   uint32_t* bin_count = reinterpret_cast<uint32_t*>(bin_pos + kTokBinCap);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uintptr_t>(bin_count + 1) + 7 & ~uintptr_t(7));
-  uint64_t* k_full = bars;
-  uint64_t* k_empty = k_full + p.stages;
+  // Key stage s holding tile g (the CTA's g-th tile) completes on
+  // k_full[g % kTokIssuers][s]: consecutive tiles of a stage can go to
+  // different issuers, and a barrier waited on by more than one of them could
+  // let a parity wait pass on an older phase; per issuer, each barrier's uses
+  // are in that issuer's own order.  Both sides keep each barrier's phase as
+  // one bit of a register mask.
+  uint64_t* k_full = bars;                               // [kTokIssuers][stages]
+  uint64_t* k_empty = k_full + kTokIssuers * p.stages;   // [stages]
   uint64_t* q_full = k_empty + p.stages;          // [2]
   uint64_t* q_empty = q_full + 2;                 // [2]
   uint64_t* acc_full = q_empty + 2;               // [kTokAcc]
@@ -114,7 +120,8 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < p.stages; ++s) { mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1); }
+    for (int s = 0; s < kTokIssuers * p.stages; ++s) mbar_init(k_full + s, 1);
+    for (int s = 0; s < p.stages; ++s) mbar_init(k_empty + s, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(q_full + i, 1); mbar_init(q_empty + i, kTokIssuers);
       mbar_init(cand_full + i, kTokScorerWarps * kTokScoreGroups); mbar_init(cand_empty + i, 1);
@@ -210,9 +217,9 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
   } else if (warp == kTokTmaWarp) {
     // ------------------------------------------------------------ TMA issue
     if (lane == 0) {
-      int st = 0;
-      uint32_t kph = 0;
-      int8_t last_ph[8];
+      int st = 0, gi = 0;                       // stage, issuer of the next tile
+      uint32_t kph = 0, fph = 0;                // k_empty phase; k_full phases, one bit per barrier
+      int8_t last_ph[8], last_bar[8];          // per stage: the last full barrier armed and its phase
       for (int i = 0; i < 8; ++i) last_ph[i] = -1;
       int8_t last_qph[2] = {-1, -1};
       bool ok = true;
@@ -233,20 +240,25 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
           if (!(ok = mbar_wait(k_empty + st, kph ^ 1, abort_flag))) break;
           const int first = tl * blocks_per_tile;
           const int nblk_t = min(blocks_per_tile, J.nblk - first);
-          mbar_arrive_expect_tx(k_full + st, static_cast<uint32_t>(nblk_t * p.B * row_bytes));
+          const int kfi = gi * p.stages + st;
+          uint64_t* kf = k_full + kfi;
+          mbar_arrive_expect_tx(kf, static_cast<uint32_t>(nblk_t * p.B * row_bytes));
           for (int q = 0; q < nblk_t; ++q) {
             const int krow = kb + J.blk[first + q] * p.B;
             for (int pn = 0; pn < panels; ++pn)
-              tma_load_2d(k_buf + st * k_bytes + pn * (kTokTileM * 128) + q * p.B * 128, &kmap, k_full + st,
+              tma_load_2d(k_buf + st * k_bytes + pn * (kTokTileM * 128) + q * p.B * 128, &kmap, kf,
                           pn * panel_elems, krow);
           }
-          last_ph[st] = static_cast<int8_t>(kph);
+          last_ph[st] = static_cast<int8_t>((fph >> kfi) & 1u);
+          last_bar[st] = static_cast<int8_t>(kfi);
+          fph ^= 1u << kfi;
+          if (++gi == kTokIssuers) gi = 0;
           if (++st == p.stages) { st = 0; kph ^= 1; }
         }
       }
       if (!ok) {   // drain the copies this thread issued before leaving
         for (int i = 0; i < p.stages; ++i)
-          if (last_ph[i] >= 0) mbar_drain(k_full + i, static_cast<uint32_t>(last_ph[i]));
+          if (last_ph[i] >= 0) mbar_drain(k_full + last_bar[i], static_cast<uint32_t>(last_ph[i]));
         for (int i = 0; i < 2; ++i)
           if (last_qph[i] >= 0) mbar_drain(q_full + i, static_cast<uint32_t>(last_qph[i]));
       }
@@ -258,7 +270,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
       constexpr uint32_t idesc = instr_desc(kTokTileM, H, DT == DT_BF16 ? 1u : 0u);
       const int ksteps = row_bytes / 32;
       int st = 0, ab = 0, g = 0;
-      uint32_t kph = 0, aph = 0;
+      uint32_t aph = 0, fph = 0;               // fph: phases of this issuer's k_full barriers, one bit per stage
       bool ok = true;
       for (int64_t j = 0; ok && j < njobs; ++j) {
         const int slot = static_cast<int>(j % kTokJobs);
@@ -271,7 +283,8 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
         for (int i = 0; i < ntiles; ++i) {
           if (g == me) {
             if (!(ok = mbar_wait(acc_empty + ab, aph ^ 1, abort_flag))) break;
-            if (!(ok = mbar_wait(k_full + st, kph, abort_flag))) break;
+            if (!(ok = mbar_wait(k_full + me * p.stages + st, (fph >> st) & 1u, abort_flag))) break;
+            fph ^= 1u << st;
             tc_fence_after();
             const uint32_t k_addr = smem_u32(k_buf + st * k_bytes);
             const uint32_t d_tmem = tmem_base + ab * H;
@@ -284,7 +297,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
             mma_commit(acc_full + ab);
           }
           if (++g == kTokIssuers) g = 0;
-          if (++st == p.stages) { st = 0; kph ^= 1; }
+          if (++st == p.stages) st = 0;
           if (++ab == kTokAcc) { ab = 0; aph ^= 1; }
         }
         if (ok) mma_commit(q_empty + qb);
@@ -329,20 +342,21 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
           if (H >= 32) {
             // all TMEM loads of the row first, one wait, then four independent
             // accumulation chains over float4 weight reads
-            uint32_t v[H];
-#pragma unroll
-            for (int c0 = 0; c0 < H; c0 += 32)
-              tmem_ld32(t_lane + ab * H + c0, *reinterpret_cast<uint32_t(*)[32]>(v + c0));
-            tmem_wait_ld();
             float a4[4] = {0.f, 0.f, 0.f, 0.f};
             const float4* w4 = reinterpret_cast<const float4*>(J.w);
 #pragma unroll
-            for (int e = 0; e < H / 4; ++e) {
-              const float4 wv = w4[e];
-              a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * e + 0]), 0.f), a4[0]);
-              a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * e + 1]), 0.f), a4[1]);
-              a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * e + 2]), 0.f), a4[2]);
-              a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * e + 3]), 0.f), a4[3]);
+            for (int c0 = 0; c0 < H; c0 += 32) {
+              uint32_t v[32];
+              tmem_ld32(t_lane + ab * H + c0, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float4 wv = w4[c0 / 4 + e];
+                a4[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[4 * e + 0]), 0.f), a4[0]);
+                a4[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[4 * e + 1]), 0.f), a4[1]);
+                a4[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[4 * e + 2]), 0.f), a4[2]);
+                a4[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[4 * e + 3]), 0.f), a4[3]);
+              }
             }
             acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
           } else {
@@ -454,7 +468,7 @@ inline size_t token_smem_bytes(int row_bytes, int H, int stages, int max_cand) {
   return 1024 + 2 * static_cast<size_t>(H) * row_bytes + static_cast<size_t>(stages) * kTokTileM * row_bytes +
          2 * static_cast<size_t>(max_cand) * 4 + kTokJobs * sizeof(TokJob) + sizeof(SelectSmem) +
          4 * kTokMaxBitmapWords + 8 * kTokBinCap + 4 + 8 +
-         8 * (2 * stages + 4 + 2 * kTokAcc + 2 * kTokJobs + 4 + kTokIssuers) + 16;
+         8 * ((kTokIssuers + 1) * stages + 4 + 2 * kTokAcc + 2 * kTokJobs + 4 + kTokIssuers) + 16;
 }
 
 }  // namespace hisa
