@@ -43,6 +43,7 @@ class Shape(ctypes.Structure):
 _P = ctypes.c_void_p
 _SIGS = {
     "hisa_pool_blocks": [_P, _P, _P, _P, ctypes.POINTER(Shape), _P],
+    "hisa_pool_blocks_range": [_P, _P, _P, _P, ctypes.POINTER(Shape), ctypes.c_int32, ctypes.c_int32, _P],
     "hisa_compress_keys": [_P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                            ctypes.c_int32, _P],
     "hisa_quantize_e4m3": [_P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _P, _P, _P],
@@ -156,6 +157,24 @@ def hisa_pool_blocks(k: torch.Tensor, block_size: int, k_scale: Optional[torch.T
     _check(load().hisa_pool_blocks(k.data_ptr(), _ptr(k_scale), kpool.data_ptr(), _ptr(kps), ctypes.byref(shape),
                                    _stream()), "hisa_pool_blocks")
     return kpool, kps
+
+
+def hisa_pool_blocks_range(k: torch.Tensor, block_size: int, first_block: int, block_count: int,
+                           kpool: torch.Tensor, k_scale: Optional[torch.Tensor] = None,
+                           kpool_scale: Optional[torch.Tensor] = None) -> None:
+    """Pool blocks [first_block, first_block + block_count) of every sequence into
+    the caller's kpool [batch, nb, d] (and kpool_scale for E4M3) in place."""
+    _need(k, "keys", 3)
+    b, L, d = k.shape
+    nb = -(-L // block_size)
+    if tuple(kpool.shape) != (b, nb, d) or kpool.dtype != k.dtype or not kpool.is_contiguous():
+        raise ValueError("kpool must be a contiguous [batch, ceil(L/B), d] tensor of the keys' dtype")
+    if (k_scale is None) != (kpool_scale is None):
+        raise ValueError("k_scale and kpool_scale go together (E4M3 keys)")
+    shape = Shape(b, L, 1, 1, d, block_size, 1, 1, dtype_code(k))
+    _check(load().hisa_pool_blocks_range(k.data_ptr(), _ptr(k_scale), kpool.data_ptr(), _ptr(kpool_scale),
+                                         ctypes.byref(shape), first_block, block_count, _stream()),
+           "hisa_pool_blocks_range")
 
 
 def hisa_compress_keys(k_raw: torch.Tensor, ratio: int) -> torch.Tensor:

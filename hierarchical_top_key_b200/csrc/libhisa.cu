@@ -393,6 +393,13 @@ hisa_status hisa_workspace_size(int32_t op, const hisa_shape* s, size_t* bytes) 
 hisa_status hisa_pool_blocks(const void* k, const float* k_scale, void* kpool, float* kpool_scale,
                              const hisa_shape* s, hisa_stream stream) {
   if (!s) return fail(HISA_ERR_INVALID_ARG, "shape is NULL");
+  return hisa_pool_blocks_range(k, k_scale, kpool, kpool_scale, s, 0, static_cast<int32_t>(num_blocks(s)), stream);
+}
+
+hisa_status hisa_pool_blocks_range(const void* k, const float* k_scale, void* kpool, float* kpool_scale,
+                                   const hisa_shape* s, int32_t first_block, int32_t block_count, hisa_stream stream) {
+  if (!s) return fail(HISA_ERR_INVALID_ARG, "shape is NULL");
+  if (first_block < 0 || block_count < 0) return fail(HISA_ERR_INVALID_ARG, "first_block and block_count must be >= 0");
   if (s->batch < 1 || s->num_keys < 1 || s->block_size < 1)
     return fail(HISA_ERR_INVALID_ARG, "batch, num_keys, block_size must be >= 1");
   if (s->head_dim != 64 && s->head_dim != 128) return fail(HISA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
@@ -401,23 +408,26 @@ hisa_status hisa_pool_blocks(const void* k, const float* k_scale, void* kpool, f
   if (s->dtype == HISA_E4M3 && (!k_scale || !kpool_scale))
     return fail(HISA_ERR_INVALID_ARG, "E4M3 pooling needs k_scale and kpool_scale");
   const int nb = static_cast<int>(num_blocks(s));
+  const int first = std::min(first_block, nb);
+  const int count = std::min(block_count, nb - first);
+  if (count == 0) return HISA_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t threads_total = static_cast<int64_t>(s->batch) * nb * (s->head_dim * elem_bytes(s->dtype) / 16);
+  const int64_t threads_total = static_cast<int64_t>(s->batch) * count * (s->head_dim * elem_bytes(s->dtype) / 16);
   const int grid = static_cast<int>(std::min<int64_t>(ceil_div(threads_total, 256), 148 * 64));
   const uint8_t* in = static_cast<const uint8_t*>(k);
   uint8_t* out = static_cast<uint8_t*>(kpool);
   switch (s->dtype) {
     case HISA_F32:
       segment_mean_kernel<DT_F32><<<grid, 256, 0, st>>>(in, nullptr, out, nullptr, s->batch, s->num_keys, nb,
-                                                        s->head_dim, s->block_size);
+                                                        s->head_dim, s->block_size, first, count);
       break;
     case HISA_BF16:
       segment_mean_kernel<DT_BF16><<<grid, 256, 0, st>>>(in, nullptr, out, nullptr, s->batch, s->num_keys, nb,
-                                                         s->head_dim, s->block_size);
+                                                         s->head_dim, s->block_size, first, count);
       break;
     case HISA_E4M3:
       segment_mean_kernel<DT_E4M3><<<grid, 256, 0, st>>>(in, k_scale, out, kpool_scale, s->batch, s->num_keys,
-                                                         nb, s->head_dim, s->block_size);
+                                                         nb, s->head_dim, s->block_size, first, count);
       break;
     default: return fail(HISA_ERR_INVALID_ARG, "unknown dtype %d", s->dtype);
   }
@@ -442,10 +452,10 @@ hisa_status hisa_compress_keys(const void* k_raw, void* ck, int32_t batch, int32
   uint8_t* out = static_cast<uint8_t*>(ck);
   if (dtype == HISA_F32)
     segment_mean_kernel<DT_F32><<<grid, 256, 0, st>>>(in, nullptr, out, nullptr, batch, num_raw_keys, n_out,
-                                                      head_dim, ratio);
+                                                      head_dim, ratio, 0, n_out);
   else
     segment_mean_kernel<DT_BF16><<<grid, 256, 0, st>>>(in, nullptr, out, nullptr, batch, num_raw_keys, n_out,
-                                                       head_dim, ratio);
+                                                       head_dim, ratio, 0, n_out);
   return launch_check("segment_mean_kernel (compress)");
 }
 

@@ -19,18 +19,19 @@ template <int DT>
 __global__ void __launch_bounds__(256) segment_mean_kernel(
     const uint8_t* __restrict__ in, const float* __restrict__ in_scale,
     uint8_t* __restrict__ out, float* __restrict__ out_scale,
-    int batch, int n_in, int n_out, int d, int G) {
+    int batch, int n_in, int n_out, int d, int G, int o_first, int o_count) {
   constexpr int VE = Vec16<DT>::n;             // elements per 16-byte vector
   const int vecs = d / VE;                     // threads per output row (power of 2, <= 32)
   const int64_t row_bytes = static_cast<int64_t>(d) * Elem<DT>::bytes;
-  const int64_t total = static_cast<int64_t>(batch) * n_out * vecs;
+  const int64_t total = static_cast<int64_t>(batch) * o_count * vecs;
   for (int64_t g = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; g < ceil_div(total, 32) * 32;
        g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const bool live = g < total;
-    const int64_t orow = live ? g / vecs : 0;            // flattened (b, o)
+    const int64_t lrow = live ? g / vecs : 0;            // flattened (b, o - o_first)
     const int v = static_cast<int>(g % vecs);
-    const int b = static_cast<int>(orow / n_out);
-    const int o = static_cast<int>(orow % n_out);
+    const int b = static_cast<int>(lrow / o_count);
+    const int o = o_first + static_cast<int>(lrow % o_count);
+    const int64_t orow = static_cast<int64_t>(b) * n_out + o;   // output row in [batch, n_out]
     const int r0 = o * G;
     const int r1 = min(r0 + G, n_in);
     double acc[VE];

@@ -107,6 +107,24 @@ HISA_API hisa_status hisa_pool_blocks(const void* k, const float* k_scale, void*
                              hisa_stream stream);
 
 /*
+ * Block pooling of a range of blocks: the rows b in [first_block,
+ * first_block + block_count) (clipped to ceil(num_keys / B)) of every
+ * sequence's kpool (and kpool_scale for E4M3) are written exactly as
+ * hisa_pool_blocks writes them; every other row is left untouched.
+ * The pages pool keys into blocks once per context (HISA abstract) and do not
+ * say how a decoder keeps them; this entry lets it keep the pooled keys as a
+ * cache, pooling a block once when its last key arrives, since the coarse
+ * stage only scores blocks that are complete (the current block is kept
+ * without a score).  Same layouts, ownership and checks as hisa_pool_blocks;
+ * first_block < 0 or block_count < 0 is HISA_ERR_INVALID_ARG, an empty range
+ * returns HISA_OK without a launch.
+ */
+HISA_API hisa_status hisa_pool_blocks_range(const void* k, const float* k_scale, void* kpool,
+                                            float* kpool_scale, const hisa_shape* shape,
+                                            int32_t first_block, int32_t block_count,
+                                            hisa_stream stream);
+
+/*
  * Key compression ("StreamIndex: Memory-Bounded Compressed Sparse Attention
  * via Streaming Top-k", arXiv 2605.02568, abstract: the indexer runs over keys
  * compressed by a fixed ratio, 4 in V4-Flash).  ck[j] = mean of raw keys

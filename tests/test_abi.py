@@ -82,5 +82,9 @@ def test_pointer_validation_returns_before_any_launch(L):
     assert L.hisa_token_score_topk(0x1000, None, 0x2000, 0x3000, None, 0x4000, 0x5000, ctypes.byref(big), 0x6000,
                                    None, None, 0, None) == 2
     assert L.hisa_pool_blocks(None, None, None, None, ctypes.byref(s), None) == 1
+    assert L.hisa_pool_blocks_range(0x1000, None, 0x2000, None, ctypes.byref(s), -1, 1, None) == 1
+    assert L.hisa_pool_blocks_range(0x1000, None, 0x2000, None, ctypes.byref(s), 0, -1, None) == 1
+    # a range past the last block launches nothing (the placeholder pointers are never used)
+    assert L.hisa_pool_blocks_range(0x1000, None, 0x2000, None, ctypes.byref(s), 1 << 20, 4, None) == 0
     assert L.hisa_quantize_e4m3(0x1000, hb.HISA_BF16, 10, 100, 0x2000, 0x3000, None) == 2   # cols % 16
     assert L.hisa_compress_keys(0x1000, 0x2000, 1, 100, 128, 4, hb.HISA_E4M3, None) == 2
