@@ -495,8 +495,20 @@ hisa_status hisa_block_score_topm(const void* q, const float* q_scale, const flo
   for (const RowChunk& c : chunks) {
     e = score_rows(s, q, q_scale, w, kpool, kpool_scale, n_visible, s->block_size, static_cast<int>(nb), c, ws, ld, st);
     if (e != HISA_OK) return e;
-    block_select_kernel<<<static_cast<unsigned>(c.nrows), 512, 0, st>>>(ws, ld, n_visible, c.row0, s->num_keys,
-                                                                        s->block_size, s->top_m, block_idx);
+    const int grid = static_cast<int>(std::min<int64_t>(ceil_div(c.nrows, 8), static_cast<int64_t>(num_sms()) * 8));
+    if (nb <= 32 * 8) {
+      block_select_warp_kernel<8><<<grid, 256, 0, st>>>(ws, ld, n_visible, c.row0, c.nrows, s->num_keys,
+                                                        s->block_size, s->top_m, block_idx);
+    } else if (nb <= 32 * 16) {
+      block_select_warp_kernel<16><<<grid, 256, 0, st>>>(ws, ld, n_visible, c.row0, c.nrows, s->num_keys,
+                                                         s->block_size, s->top_m, block_idx);
+    } else if (nb <= 32 * 32) {
+      block_select_warp_kernel<32><<<grid, 256, 0, st>>>(ws, ld, n_visible, c.row0, c.nrows, s->num_keys,
+                                                         s->block_size, s->top_m, block_idx);
+    } else {
+      block_select_kernel<<<static_cast<unsigned>(c.nrows), 512, 0, st>>>(ws, ld, n_visible, c.row0, s->num_keys,
+                                                                          s->block_size, s->top_m, block_idx);
+    }
     e = launch_check("block_select_kernel");
     if (e != HISA_OK) return e;
   }

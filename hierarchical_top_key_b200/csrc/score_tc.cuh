@@ -12,12 +12,17 @@
 // exists outside TMEM.
 //
 // Persistent, warp-specialised CTA (one per SM):
+//   warp 10     unit set-up: visibility, weights and scales of each work unit
+//               into a ring of four shared-memory slots, ahead of the others
 //   warp 0      TMA producer: q group (one or two buffers) and key tiles (ring)
 //   warp 1      TMEM owner and MMA issuer (one thread)
 //   warps 2..9  epilogue: TMEM -> registers -> weighted ReLU sum -> global
 // Two TMEM accumulators (2 x 256 columns) let the MMA of tile i+1 overlap the
-// epilogue of tile i.  Work units are (query group, chunk of key tiles); the
-// schedule is static and identical in every role.
+// epilogue of tile i.  Work units are (query group, chunk of key tiles) in a
+// static schedule; the set-up warp publishes the non-empty ones in order and
+// ends the ring with an empty unit.  Units with few key tiles (the coarse
+// stage has one or two per query group) are then no longer paced by global
+// loads in the producer, the issuer and the epilogue.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -27,7 +32,18 @@ namespace hisa {
 constexpr int kDenseTileM = 128;
 constexpr int kDenseN = 256;
 constexpr int kDenseEpiWarps = 8;
-constexpr int kDenseThreads = 64 + 32 * kDenseEpiWarps;
+constexpr int kDenseSetupWarp = 2 + kDenseEpiWarps;
+constexpr int kDenseThreads = 32 * (kDenseSetupWarp + 1);
+constexpr int kDenseSlots = 4;
+constexpr int kDenseMaxG = 16;            // queries per group (H >= 16)
+
+// One published work unit.  ntiles == 0 ends the ring.
+struct alignas(16) DenseSlot {
+  int b, t0, nq, tile0, ntiles, pad0, pad1, pad2;
+  int vis[kDenseMaxG];                    // visible key rows of each query of the group
+  float qsc[kDenseMaxG];                  // E4M3 q scales (1 otherwise)
+  float w[kDenseN];                       // [G][H] head weights (0 past the last query)
+};
 
 struct DenseParams {
   int Q, H, d, L;           // L: key rows per sequence (keys, or pooled blocks)
@@ -59,24 +75,8 @@ __device__ __forceinline__ int dense_vis(const DenseParams& p, int n) {
   return max(0, min(v, p.L));
 }
 
-// Unit u: groups in descending order (longest causal prefixes first), chunks
-// of kc_tiles key tiles.  ntiles <= 0 means the unit has no visible key.
-__device__ __forceinline__ DenseUnit dense_unit(const DenseParams& p, int64_t u) {
-  DenseUnit U;
-  const int64_t gi = p.ngroups - 1 - u / p.max_chunks;
-  const int chunk = static_cast<int>(u % p.max_chunks);
-  const int64_t gg = p.gg0 + gi;
-  U.b = static_cast<int>(gg / p.groups_per_seq);
-  const int g = static_cast<int>(gg % p.groups_per_seq);
-  U.t0 = g * p.G;
-  U.nq = min(p.G, p.Q - U.t0);
-  int vmax = 0;
-  for (int j = 0; j < U.nq; ++j) vmax = max(vmax, dense_vis(p, __ldg(p.n_visible + static_cast<int64_t>(U.b) * p.Q + U.t0 + j)));
-  const int tiles = (vmax + kDenseTileM - 1) / kDenseTileM;
-  U.tile0 = chunk * p.kc_tiles;
-  U.ntiles = min(p.kc_tiles, tiles - U.tile0);
-  return U;
-}
+// Unit u of the schedule: groups in descending order (longest causal
+// prefixes first), then chunks of kc_tiles key tiles.
 
 // Snake order over rounds of gridDim.x units balances the causal triangle.
 __device__ __forceinline__ int64_t dense_unit_index(int64_t round) {
@@ -105,13 +105,12 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
   uint64_t* q_empty = q_full + 2;                        // [2]
   uint64_t* acc_full = q_empty + 2;                      // [2]
   uint64_t* acc_empty = acc_full + 2;                    // [2]
-  uint64_t* drain = acc_empty + 2;
+  uint64_t* unit_full = acc_empty + 2;                   // [kDenseSlots]
+  uint64_t* unit_empty = unit_full + kDenseSlots;        // [kDenseSlots]
+  uint64_t* drain = unit_empty + kDenseSlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* w_s = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(tmem_slot + 2) + 15) & ~uintptr_t(15));
-                                                         // [8 warps][G/2 * H] = [4 * G * H], 16-byte aligned
-  float* qsc_s = w_s + 4 * kDenseN;                      // [8 warps][G/2]
-  int* vis_s = reinterpret_cast<int*>(qsc_s + 4 * G);    // [8 warps][G/2]
+  DenseSlot* slots = reinterpret_cast<DenseSlot*>((reinterpret_cast<uintptr_t>(tmem_slot + 2) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -120,6 +119,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
       mbar_init(q_full + i, 1); mbar_init(q_empty + i, 1);
       mbar_init(acc_full + i, 1); mbar_init(acc_empty + i, kDenseEpiWarps);
     }
+    for (int i = 0; i < kDenseSlots; ++i) { mbar_init(unit_full + i, 1); mbar_init(unit_empty + i, kDenseEpiWarps); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -132,7 +132,52 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
   const uint32_t tmem_base = *tmem_slot;
   const int64_t total_units = static_cast<int64_t>(p.ngroups) * p.max_chunks;
 
-  if (warp == 0) {
+  if (warp == kDenseSetupWarp) {
+    // ------------------------------------------------------------ unit set-up
+    int un = 0;
+    bool ok = true;
+    for (int64_t r = 0; ok && r * gridDim.x < total_units; ++r) {
+      const int64_t u = dense_unit_index(r);
+      if (u >= total_units) continue;
+      const int64_t gg = p.gg0 + (p.ngroups - 1 - u / p.max_chunks);
+      const int chunk = static_cast<int>(u % p.max_chunks);
+      const int b = static_cast<int>(gg / p.groups_per_seq);
+      const int t0 = static_cast<int>(gg % p.groups_per_seq) * p.G;
+      const int nq = min(p.G, p.Q - t0);
+      const int64_t qrow0 = static_cast<int64_t>(b) * p.Q + t0;
+      const int vis = lane < nq ? dense_vis(p, __ldg(p.n_visible + qrow0 + lane)) : 0;
+      const int vmax = __reduce_max_sync(0xffffffffu, vis);
+      const int tile0 = chunk * p.kc_tiles;
+      const int ntiles = min(p.kc_tiles, (vmax + kDenseTileM - 1) / kDenseTileM - tile0);
+      if (ntiles <= 0) continue;
+      const int sl = un % kDenseSlots;
+      int okl = 1;
+      if (lane == 0) okl = mbar_wait(unit_empty + sl, ((un / kDenseSlots) & 1) ^ 1, abort_flag) ? 1 : 0;
+      if (!(ok = __shfl_sync(0xffffffffu, okl, 0) != 0)) break;
+      DenseSlot& S = slots[sl];
+      if (lane == 0) { S.b = b; S.t0 = t0; S.nq = nq; S.tile0 = tile0; S.ntiles = ntiles; }
+      if (lane < kDenseMaxG) {
+        S.vis[lane] = vis;
+        S.qsc[lane] = (DT == DT_E4M3 && lane < nq) ? __ldg(p.q_scale + qrow0 + lane) : 1.f;
+      }
+      for (int i = lane; i < G * H; i += 32) {
+        const int j = i / H;
+        S.w[i] = j < nq ? __ldg(p.w + (qrow0 + j) * p.H + (i % H)) : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(unit_full + sl);
+      ++un;
+    }
+    if (ok) {   // the empty unit that ends the ring
+      const int sl = un % kDenseSlots;
+      int okl = 1;
+      if (lane == 0) okl = mbar_wait(unit_empty + sl, ((un / kDenseSlots) & 1) ^ 1, abort_flag) ? 1 : 0;
+      if (__shfl_sync(0xffffffffu, okl, 0) != 0 && lane == 0) {
+        slots[sl].ntiles = 0;
+        mbar_arrive(unit_full + sl);
+      }
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int st = 0;
@@ -142,11 +187,12 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
       for (int s = 0; s < 8; ++s) last_ph[s] = -1;
       int8_t last_qph[2] = {-1, -1};
       bool ok = true;
-      for (int64_t r = 0; ok && r * gridDim.x < total_units; ++r) {
-        const int64_t u = dense_unit_index(r);
-        if (u >= total_units) continue;
-        const DenseUnit U = dense_unit(p, u);
-        if (U.ntiles <= 0) continue;
+      while (ok) {
+        const int sl = un % kDenseSlots;
+        if (!(ok = mbar_wait(unit_full + sl, (un / kDenseSlots) & 1, abort_flag))) break;
+        DenseUnit U;
+        U.b = slots[sl].b; U.t0 = slots[sl].t0; U.tile0 = slots[sl].tile0; U.ntiles = slots[sl].ntiles;
+        if (U.ntiles == 0) break;
         const int qb = un % p.q_bufs;
         if (!(ok = mbar_wait(q_empty + qb, ((un / p.q_bufs) & 1) ^ 1, abort_flag))) break;
         mbar_arrive_expect_tx(q_full + qb, q_bytes);
@@ -181,11 +227,12 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
       uint32_t kph = 0, aph = 0;
       int un = 0;
       bool ok = true;
-      for (int64_t r = 0; ok && r * gridDim.x < total_units; ++r) {
-        const int64_t u = dense_unit_index(r);
-        if (u >= total_units) continue;
-        const DenseUnit U = dense_unit(p, u);
-        if (U.ntiles <= 0) continue;
+      while (ok) {
+        const int sl = un % kDenseSlots;
+        if (!(ok = mbar_wait(unit_full + sl, (un / kDenseSlots) & 1, abort_flag))) break;
+        DenseUnit U;
+        U.ntiles = slots[sl].ntiles;
+        if (U.ntiles == 0) break;
         const int qb = un % p.q_bufs;
         if (!(ok = mbar_wait(q_full + qb, (un / p.q_bufs) & 1, abort_flag))) break;
         tc_fence_after();
@@ -216,35 +263,29 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Each warp stages the weights, visibility and scales of its own queries
-    // (no cross-warp barrier inside the loop, so an abort cannot strand a
-    // warp); lane 0 alone waits on the accumulator barrier.
+    // The unit's weights, visibility and scales come from its slot; lane 0
+    // alone waits on the barriers, and each warp releases the slot when it
+    // is done with the unit.
     const int e = warp - 2;
     const int quarter = warp & 3;                 // TMEM lanes this warp may access
     const int half = e >> 2;                      // which half of the group's queries
     constexpr int QPT = G / 2;                    // queries per thread
-    float* w_w = w_s + e * (QPT * H);
-    float* qsc_w = qsc_s + e * QPT;
-    int* vis_w = vis_s + e * QPT;
     int64_t tc = 0;
+    int un = 0;
     bool ok = true;
-    for (int64_t r = 0; ok && r * gridDim.x < total_units; ++r) {
-      const int64_t u = dense_unit_index(r);
-      if (u >= total_units) continue;
-      const DenseUnit U = dense_unit(p, u);
-      if (U.ntiles <= 0) continue;
+    while (ok) {
+      const int sl = un % kDenseSlots;
+      int okl = 1;
+      if (lane == 0) okl = mbar_wait(unit_full + sl, (un / kDenseSlots) & 1, abort_flag) ? 1 : 0;
+      if (!(ok = __shfl_sync(0xffffffffu, okl, 0) != 0)) break;
+      const DenseSlot& S = slots[sl];
+      DenseUnit U;
+      U.b = S.b; U.t0 = S.t0; U.nq = S.nq; U.tile0 = S.tile0; U.ntiles = S.ntiles;
+      if (U.ntiles == 0) break;
       const int64_t qrow0 = static_cast<int64_t>(U.b) * p.Q + U.t0;
-      __syncwarp();
-      for (int i = lane; i < QPT * H; i += 32) {
-        const int j = half * QPT + i / H;
-        w_w[i] = j < U.nq ? __ldg(p.w + (qrow0 + j) * p.H + (i % H)) : 0.f;
-      }
-      for (int jq = lane; jq < QPT; jq += 32) {
-        const int j = half * QPT + jq;
-        vis_w[jq] = j < U.nq ? dense_vis(p, __ldg(p.n_visible + qrow0 + j)) : 0;
-        qsc_w[jq] = (DT == DT_E4M3 && j < U.nq) ? __ldg(p.q_scale + qrow0 + j) : 1.f;
-      }
-      __syncwarp();
+      const float* w_w = S.w + half * QPT * H;
+      const float* qsc_w = S.qsc + half * QPT;
+      const int* vis_w = S.vis + half * QPT;
       uint32_t kmin[QPT], kmax[QPT];
 #pragma unroll
       for (int jq = 0; jq < QPT; ++jq) { kmin[jq] = 0xFFFFFFFFu; kmax[jq] = 0u; }
@@ -314,6 +355,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
           }
         }
       }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(unit_empty + sl);
+      ++un;
     }
   }
   tc_fence_before();
@@ -327,8 +372,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
 // Bytes of dynamic shared memory the dense kernel needs.
 inline size_t dense_smem_bytes(int row_bytes, int stages, int q_bufs) {
   return 1024 /*alignment slack*/ + q_bufs * static_cast<size_t>(kDenseN) * row_bytes +
-         static_cast<size_t>(stages) * kDenseTileM * row_bytes + 8 * (2 * stages + 9) + 32 + 4 * 4 * kDenseN +
-         2 * 4 * 4 * 64 + 64;
+         static_cast<size_t>(stages) * kDenseTileM * row_bytes + 8 * (2 * stages + 9 + 2 * kDenseSlots) + 8 + 16 +
+         kDenseSlots * sizeof(DenseSlot);
 }
 
 }  // namespace hisa

@@ -533,4 +533,71 @@ __global__ void __launch_bounds__(512) block_select_kernel(
   block_topk(key_at, c, static_cast<uint32_t>(top_m - 1), emit, sm);
 }
 
+// The same selection with one warp per row, for rows of at most 32 * KPL
+// block scores: each lane keeps its KPL keys (positions lane, lane + 32, ...)
+// in registers; the (m-1)-th largest key T is found bit by bit from the top,
+// each step counting the keys >= the candidate value across the warp; keys
+// above T are emitted by ballot, then the lowest positions among the keys
+// equal to T fill the remaining places.
+template <int KPL>
+__global__ void __launch_bounds__(256) block_select_warp_kernel(
+    const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n_visible, int64_t row0,
+    int64_t nrows, int L, int block_size, int top_m, int32_t* __restrict__ out_idx) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t lr = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5; lr < nrows; lr += warps) {
+    const int64_t r = row0 + lr;
+    const float* row = scores + lr * ld;
+    const int n = max(0, min(__ldg(n_visible + r), L));
+    const int c = n > 0 ? (n - 1) / block_size : -1;
+    int32_t* oi = out_idx + r * top_m;
+    if (c + 1 <= top_m) {                    // every visible block (or none)
+      for (int i = lane; i < top_m; i += 32) oi[i] = i <= c ? i : -1;
+      continue;
+    }
+    if (lane == 0) oi[0] = c;
+    const uint32_t k = static_cast<uint32_t>(top_m - 1);
+    if (k == 0) continue;
+    uint32_t key[KPL];
+    uint32_t kmax = 0u, kmin = 0xFFFFFFFFu;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      const int i = lane + 32 * j;
+      key[j] = i < c ? float_key(__ldg(row + i)) : 0u;
+      if (i < c) { kmax = max(kmax, key[j]); kmin = min(kmin, key[j]); }
+    }
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    // bits above the highest one where kmin and kmax differ are common to all keys
+    const int top_bit = kmin == kmax ? -1 : 31 - __clz(kmin ^ kmax);
+    uint32_t T = top_bit < 0 ? kmax : (kmax & ~((2u << top_bit) - 1u));
+    for (int bit = top_bit; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      uint32_t cnt = 0;
+#pragma unroll
+      for (int j = 0; j < KPL; ++j) cnt += key[j] >= cand ? 1u : 0u;
+      if (__reduce_add_sync(0xffffffffu, cnt) >= k) T = cand;
+    }
+    // T is the k-th largest key: emit the keys above it, then the lowest
+    // positions among those equal to it
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t base = 1;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      const uint32_t ball = __ballot_sync(0xffffffffu, key[j] > T);
+      if (key[j] > T) oi[base + __popc(ball & lt)] = lane + 32 * j;
+      base += __popc(ball);
+    }
+    const uint32_t need = k + 1 - base;      // places left for keys equal to T
+    uint32_t seen = 0;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+      const uint32_t ball = __ballot_sync(0xffffffffu, key[j] == T && key[j] != 0u);
+      const uint32_t rank = seen + __popc(ball & lt);
+      if (key[j] == T && key[j] != 0u && rank < need) oi[base + rank] = lane + 32 * j;
+      seen += __popc(ball);
+    }
+  }
+}
+
 }  // namespace hisa
