@@ -285,6 +285,109 @@ class HisaIndexer:
         return (idx, sc, blocks) if return_blocks else (idx, sc)
 
 
+    def from_host(self, q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, n_visible: torch.Tensor,
+                  out: torch.Tensor, chunks: int = 16, device=None) -> torch.Tensor:
+        """The indexer on inputs in (pinned) host memory, writing the indices into
+        the host tensor `out` [batch, Q, top_k] int32.
+
+        The work is cut into `chunks` pieces (query ranges of a single sequence,
+        or ranges of sequences) run as a pipeline on three streams: the copy of
+        piece i+1 in, the kernels of piece i and the copy of piece i-1 out
+        overlap.  A piece copies only the keys its queries see that earlier
+        pieces did not, and pools only the blocks those keys complete (the
+        coarse stage scores complete blocks only).  Returns `out`; the caller's
+        current stream waits for the last copy, so events recorded on it
+        bracket the whole call.  bf16 / fp32 inputs, keys already in the
+        indexer's key space."""
+        for t, name, nd in ((q, "q", 4), (w, "w", 3), (k, "keys", 3), (n_visible, "n_visible", 2),
+                            (out, "out", 3)):
+            if t.is_cuda or not t.is_contiguous() or t.dim() != nd:
+                raise ValueError(f"{name} must be a contiguous host tensor with {nd} dims")
+        b, Q, H, d = q.shape
+        L = k.shape[1]
+        B, m, kk = self.block_size, self.top_m, self.top_k
+        if tuple(out.shape) != (b, Q, kk) or out.dtype != torch.int32:
+            raise ValueError("out must be an int32 [batch, Q, top_k] host tensor")
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        lib = load()
+        dt = dtype_code(q)
+        nb = -(-L // B)
+        nv_host = n_visible.numpy()
+        # pieces: query ranges of one sequence, or ranges of whole sequences
+        if b == 1:
+            bounds = [(0, 1, (Q * i) // chunks, (Q * (i + 1)) // chunks) for i in range(chunks)]
+        else:
+            bounds = [((b * i) // chunks, (b * (i + 1)) // chunks, 0, Q) for i in range(chunks)]
+        bounds = [x for x in bounds if x[1] > x[0] and x[3] > x[2]]
+        rows_max = max((s1 - s0) * (t1 - t0) for s0, s1, t0, t1 in bounds)
+        qd = torch.empty_like(q, device=dev)
+        wd = torch.empty_like(w, device=dev)
+        kd = torch.empty_like(k, device=dev)
+        nvd = torch.empty_like(n_visible, device=dev)
+        kpool = torch.empty((b, nb, d), dtype=k.dtype, device=dev)
+        blocks = torch.empty((b, Q, m), dtype=torch.int32, device=dev)
+        idx = torch.empty((b, Q, kk), dtype=torch.int32, device=dev)
+        wshape = Shape(rows_max, L, 1, H, d, B, m, 1, dt)
+        ws = _workspace(workspace_size(OP_BLOCK, wshape), dev)
+        cur = torch.cuda.current_stream(dev)
+        s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        start = torch.cuda.Event()
+        start.record(cur)
+        s_in.wait_event(start)
+        esz_q, esz_k = q.element_size(), k.element_size()
+        keys_in = [0] * b          # keys already copied, per sequence
+        pooled = [0] * b           # blocks already pooled, per sequence
+        for s0, s1, t0, t1 in bounds:
+            nseq, nq = s1 - s0, t1 - t0
+            # keys and blocks this piece needs beyond the earlier pieces
+            n_hi = int(min(L, max(1, nv_host[s0:s1, t0:t1].max())))
+            with torch.cuda.stream(s_in):
+                for sq in range(s0, s1):
+                    if n_hi > keys_in[sq]:
+                        kd[sq, keys_in[sq]:n_hi].copy_(k[sq, keys_in[sq]:n_hi], non_blocking=True)
+                        keys_in[sq] = n_hi
+                qd[s0:s1, t0:t1].copy_(q[s0:s1, t0:t1], non_blocking=True)
+                wd[s0:s1, t0:t1].copy_(w[s0:s1, t0:t1], non_blocking=True)
+                nvd[s0:s1, t0:t1].copy_(n_visible[s0:s1, t0:t1], non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(s_in)
+            s_run.wait_event(ready)
+            with torch.cuda.stream(s_run):
+                st = s_run.cuda_stream
+                c_hi = (n_hi - 1) // B        # blocks below the last visible one are complete
+                for sq in range(s0, s1):
+                    if c_hi > pooled[sq]:
+                        shp = Shape(1, L, 1, 1, d, B, 1, 1, dt)
+                        _check(lib.hisa_pool_blocks_range(kd[sq].data_ptr(), None, kpool[sq].data_ptr(), None,
+                                                          ctypes.byref(shp), pooled[sq], c_hi - pooled[sq], st),
+                               "hisa_pool_blocks_range")
+                        pooled[sq] = c_hi
+                shp = Shape(nseq, L, nq, H, d, B, m, kk, dt)
+                if b == 1:
+                    qp = qd[0, t0].data_ptr(); wp = wd[0, t0].data_ptr(); nvp = nvd[0, t0:].data_ptr()
+                    bp = blocks[0, t0].data_ptr(); ip = idx[0, t0].data_ptr()
+                    kp, kpp = kd.data_ptr(), kpool.data_ptr()
+                else:
+                    qp, wp, nvp = qd[s0].data_ptr(), wd[s0].data_ptr(), nvd[s0].data_ptr()
+                    bp, ip = blocks[s0].data_ptr(), idx[s0].data_ptr()
+                    kp, kpp = kd[s0].data_ptr(), kpool[s0].data_ptr()
+                _check(lib.hisa_block_score_topm(qp, None, wp, kpp, None, nvp, ctypes.byref(shp), bp,
+                                                 ws.data_ptr(), ws.numel(), st), "hisa_block_score_topm")
+                _check(lib.hisa_token_score_topk(qp, None, wp, kp, None, nvp, bp, ctypes.byref(shp), ip, None,
+                                                 None, 0, st), "hisa_token_score_topk")
+                fin = torch.cuda.Event()
+                fin.record(s_run)
+            s_out.wait_event(fin)
+            with torch.cuda.stream(s_out):
+                out[s0:s1, t0:t1].copy_(idx[s0:s1, t0:t1], non_blocking=True)
+        last = torch.cuda.Event()
+        last.record(s_out)
+        # the device buffers were allocated on the current stream, which now
+        # waits for the last copy: freeing them on return is ordered after it
+        cur.wait_event(last)
+        return out
+
+
 def to_device_inputs(inputs, device="cuda", fp8: bool = False, compress: bool = True):
     """Upload one synthetic draw (``synthetic.Inputs``) in its storage dtype.
 
