@@ -360,6 +360,30 @@ def main():
         flat_flops = FLOP_PER_PAIR_PER_HEAD_DIM * wl.heads * wl.head_dim * float(np.minimum(nvis, wl.num_keys).sum())
         flat = {"ms_per_layer": fm, "queries_per_s": queries / (fm / 1000.0),
                 "hisa_speedup": fm / ms, "score_tflops": flat_flops / (fm / 1000.0) / 1e12}
+        # the sampled-threshold flat path (same result, smaller workspace), for comparison
+        try:
+            ws_s = torch.empty(max(16, hb.workspace_size(hb.OP_FLAT_SAMPLED, shape)), dtype=torch.uint8, device=dev)
+        except hb.HisaError:
+            ws_s = None
+        if ws_s is not None:
+            hb.dsa_flat_indexer_topk_sampled(q, w, k_static, nv, top_k=wl.top_k, q_scale=qs, k_scale=ks_static,
+                                             workspace=ws_s)
+            barrier()
+            sms_ = []
+            for i in range(max(1, min(args.steps, 5))):
+                flush.zero_()
+                a, b = ev(), ev()
+                a.record(stream)
+                hb.dsa_flat_indexer_topk_sampled(q, w, k_static, nv, top_k=wl.top_k, q_scale=qs, k_scale=ks_static,
+                                                 workspace=ws_s)
+                b.record(stream)
+                sms_.append((a, b))
+            barrier()
+            hb.get_status()
+            flat["sampled_ms_per_layer"] = float(np.mean([a.elapsed_time(b) for a, b in sms_]))
+            flat["sampled_workspace_bytes"] = int(ws_s.numel())
+            flat["workspace_bytes"] = int(ws_flat.numel())
+            del ws_s
 
     # ---- decode with the pooled keys kept between steps: each step pools only
     # the block its new key completes (the coarse stage scores complete blocks)

@@ -23,7 +23,7 @@ import torch
 from . import build as _build
 
 HISA_F32, HISA_BF16, HISA_E4M3 = 0, 1, 2
-OP_BLOCK, OP_TOKEN, OP_FLAT = 1, 2, 3
+OP_BLOCK, OP_TOKEN, OP_FLAT, OP_FLAT_SAMPLED = 1, 2, 3, 4
 STATUS = {0: "HISA_OK", 1: "HISA_ERR_INVALID_ARG", 2: "HISA_ERR_UNSUPPORTED", 3: "HISA_ERR_WORKSPACE",
           4: "HISA_ERR_CUDA", 5: "HISA_ERR_TIMEOUT"}
 
@@ -52,6 +52,7 @@ _SIGS = {
     "hisa_token_score_topk": [_P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t,
                               _P],
     "dsa_flat_indexer_topk": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t, _P],
+    "dsa_flat_indexer_topk_sampled": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t, _P],
     "hisa_workspace_size": [ctypes.c_int32, ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)],
     "hisa_get_status": [_P],
     "hisa_selftest_wait_timeout": [ctypes.c_uint64, _P],
@@ -260,6 +261,22 @@ def dsa_flat_indexer_topk(q, w, k, n_visible, *, top_k: int, q_scale=None, k_sca
     _check(load().dsa_flat_indexer_topk(q.data_ptr(), _ptr(q_scale), w.data_ptr(), k.data_ptr(), _ptr(k_scale),
                                         n_visible.data_ptr(), ctypes.byref(shape), idx.data_ptr(), _ptr(sc),
                                         ws.data_ptr(), ws.numel(), _stream()), "dsa_flat_indexer_topk")
+    return idx, sc
+
+
+def dsa_flat_indexer_topk_sampled(q, w, k, n_visible, *, top_k: int, q_scale=None, k_scale=None,
+                                  want_scores: bool = False, workspace: Optional[torch.Tensor] = None):
+    """Flat DSA indexer through the sampled-threshold path (same result, less
+    workspace): (topk_idx [batch, Q, top_k] int32, scores or None)."""
+    shape = make_shape(q, k, 1, 1, top_k)
+    b, Q = q.shape[:2]
+    idx = torch.empty((b, Q, top_k), dtype=torch.int32, device=q.device)
+    sc = torch.empty((b, Q, top_k), dtype=torch.float32, device=q.device) if want_scores else None
+    ws = workspace if workspace is not None else _workspace(workspace_size(OP_FLAT_SAMPLED, shape), q.device)
+    _check(load().dsa_flat_indexer_topk_sampled(q.data_ptr(), _ptr(q_scale), w.data_ptr(), k.data_ptr(),
+                                                _ptr(k_scale), n_visible.data_ptr(), ctypes.byref(shape),
+                                                idx.data_ptr(), _ptr(sc), ws.data_ptr(), ws.numel(), _stream()),
+           "dsa_flat_indexer_topk_sampled")
     return idx, sc
 
 

@@ -6,6 +6,7 @@
 #include <cstring>
 #include <cstdarg>
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 #include <vector>
 
@@ -17,6 +18,7 @@
 #include "score_simt.cuh"
 #include "score_tc.cuh"
 #include "token_tc.cuh"
+#include "flat_lite.cuh"
 
 using namespace hisa;
 
@@ -112,7 +114,7 @@ int num_sms() {
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 
 hisa_status tensor_map_2d(CUtensorMap* map, const void* base, int dtype, uint64_t rows, uint64_t cols,
-                          uint32_t box_rows) {
+                          uint32_t box_rows, uint64_t row_stride_elems = 0) {
   if (!g_encode_tiled) {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -124,7 +126,7 @@ hisa_status tensor_map_2d(CUtensorMap* map, const void* base, int dtype, uint64_
   const int es = elem_bytes(dtype);
   const CUtensorMapDataType ty = dtype == HISA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * es};
+  cuuint64_t strides[1] = {(row_stride_elems ? row_stride_elems : cols) * es};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode_tiled(map, ty, 2, const_cast<void*>(base), dims, strides, box, estr,
@@ -213,6 +215,32 @@ hisa_status dense_tc_h(const hisa_shape* s, const CUtensorMap& qm, const CUtenso
 }
 
 // Score rows of one chunk: out[(b*Q+t) - row0][s] for the visible keys.
+// Tensor-core scoring of one row chunk against every stride-th key (stride >=
+// 1), writing score rows (out, ld) or, with `thresh`, compacted pairs.
+hisa_status score_rows_tc_mode(const hisa_shape* s, const void* q, const float* qsc, const float* w,
+                               const void* keys, const float* ksc, const int32_t* nvis, int stride,
+                               const RowChunk& c, float* out, int64_t ld, const uint32_t* thresh, uint2* pairs,
+                               uint32_t* counts, int cap, cudaStream_t st) {
+  CUtensorMap qm, km;
+  const int Lv = s->num_keys / stride;                 // key rows per sequence in the strided view
+  hisa_status e = tensor_map_2d(&qm, q, s->dtype, static_cast<uint64_t>(rows_of(s)) * s->heads, s->head_dim, kDenseN);
+  if (e != HISA_OK) return e;
+  e = tensor_map_2d(&km, keys, s->dtype, static_cast<uint64_t>(s->batch) * Lv, s->head_dim, kDenseTileM,
+                    static_cast<uint64_t>(stride) * s->head_dim);
+  if (e != HISA_OK) return e;
+  DenseParams p{};
+  p.Q = s->num_queries; p.H = s->heads; p.d = s->head_dim; p.L = Lv;
+  p.G = kDenseN / s->heads;
+  p.groups_per_seq = static_cast<int>(ceil_div(s->num_queries, p.G));
+  p.block_div = 0;
+  p.vis_stride = stride;
+  p.gg0 = c.gg0; p.ngroups = c.ngroups; p.row0 = c.row0;
+  p.w = w; p.n_visible = nvis; p.q_scale = qsc; p.k_scale = ksc; p.out = out; p.ld = ld; p.minmax = nullptr;
+  p.ksc_ld = s->num_keys; p.ksc_step = stride;
+  p.thresh = thresh; p.pairs = pairs; p.counts = counts; p.cap = cap;
+  return s->dtype == HISA_BF16 ? dense_tc_h<DT_BF16>(s, qm, km, p, st) : dense_tc_h<DT_E4M3>(s, qm, km, p, st);
+}
+
 hisa_status score_rows(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* keys,
                        const float* ksc, const int32_t* nvis, int block_div, int L, const RowChunk& c, float* out,
                        int64_t ld, cudaStream_t st, uint32_t* minmax = nullptr) {
@@ -229,6 +257,7 @@ hisa_status score_rows(const hisa_shape* s, const void* q, const float* qsc, con
     p.block_div = block_div;
     p.gg0 = c.gg0; p.ngroups = c.ngroups; p.row0 = c.row0;
     p.w = w; p.n_visible = nvis; p.q_scale = qsc; p.k_scale = ksc; p.out = out; p.ld = ld; p.minmax = minmax;
+    p.ksc_ld = L; p.ksc_step = 1;
     return s->dtype == HISA_BF16 ? dense_tc_h<DT_BF16>(s, qm, km, p, st) : dense_tc_h<DT_E4M3>(s, qm, km, p, st);
   }
   switch (s->dtype) {
@@ -315,6 +344,115 @@ hisa_status token_tc_h(const hisa_shape* s, const void* q, const float* qsc, con
   }
 }
 
+// ------------------------------------------------------------ flat top-k without score rows
+
+struct LitePlan {
+  int stride;        // every stride-th key is sampled
+  int r_target;      // the threshold is the r_target-th largest sample score
+  int cap;           // pairs kept per query
+  int64_t sld;       // sample scores per row (padded)
+  int fb_ctas;       // CTAs (scratch rows) of the fallback
+  size_t fixed;      // workspace bytes independent of the chunk: counter + fallback scratch
+  size_t per_row;    // workspace bytes per row
+};
+
+// The sampled-threshold flat path applies to tensor-core shapes whose key
+// count the sample stride divides and whose pair buffer would be smaller
+// than the visible prefix; r_target and cap put the chance that fewer than k
+// or more than cap keys pass the threshold several standard deviations out
+// under uniform sampling (a miss only costs the fallback).
+bool lite_plan(const hisa_shape* s, LitePlan* lp) {
+  if (!dense_tc_ok(s)) return false;
+  const int L = s->num_keys, k = s->top_k;
+  int stride = 16;
+  while (L / stride > 4096) stride *= 2;
+  if (L % stride != 0 || L / stride < 1) return false;
+  const double kr = static_cast<double>(k) / stride;
+  const int r = static_cast<int>(std::ceil(kr + 6.0 * std::sqrt(kr))) + 2;
+  int cap = static_cast<int>(std::ceil(r * static_cast<double>(stride) + 8.0 * stride * std::sqrt(static_cast<double>(r))));
+  cap = (cap + 63) / 64 * 64;
+  if (cap > 8192 || cap >= L) return false;
+  lp->stride = stride;
+  lp->r_target = r;
+  lp->cap = cap;
+  lp->sld = pad4(L / stride);
+  lp->fb_ctas = std::min(num_sms(), 32);
+  lp->fixed = 256 + static_cast<size_t>(lp->fb_ctas) * L * 4 + 16;   // + alignment of the pair buffer
+  lp->per_row = static_cast<size_t>(lp->sld) * 4 + 12 + static_cast<size_t>(cap) * 8;
+  return true;
+}
+
+template <int DT>
+hisa_status launch_flat_fallback(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* k,
+                                 const float* ksc, const int32_t* nvis, int64_t row0, const uint32_t* fail_count,
+                                 const int32_t* fail_rows, float* scratch, int fb_ctas, int32_t* oi, float* os,
+                                 cudaStream_t st) {
+  auto run = [&](auto kern, size_t smem) {
+    hisa_status e = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    static_cast<int>(smem)), "flat_fallback attribute");
+    if (e != HISA_OK) return e;
+    kern<<<fb_ctas, kSimtThreads, smem, st>>>(static_cast<const uint8_t*>(q), qsc, w, static_cast<const uint8_t*>(k),
+                                              ksc, nvis, row0, s->num_queries, s->heads, s->head_dim, s->num_keys,
+                                              s->top_k, fail_count, fail_rows, scratch, oi, os);
+    return launch_check("flat_fallback_kernel");
+  };
+  if (s->heads <= 16) return run(flat_fallback_kernel<DT, 16>, SimtTile<DT, 16>::smem_bytes(s->head_dim));
+  return run(flat_fallback_kernel<DT, 64>, SimtTile<DT, 64>::smem_bytes(s->head_dim));
+}
+
+hisa_status flat_lite(const hisa_shape* s, const LitePlan& lp, const void* q, const float* qsc, const float* w,
+                      const void* k, const float* ksc, const int32_t* nvis, int32_t* oi, float* os, void* workspace,
+                      size_t ws_bytes, cudaStream_t st) {
+  const int64_t rows = rows_of(s);
+  const int64_t cap_rows = static_cast<int64_t>((ws_bytes - lp.fixed) / lp.per_row);
+  std::vector<RowChunk> chunks;
+  hisa_status e = plan_chunks(s, dense_group(s), std::min<int64_t>(rows, cap_rows), chunks);
+  if (e != HISA_OK) return e;
+  int64_t R = 0;
+  for (const RowChunk& c : chunks) R = std::max(R, c.nrows);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint32_t* fail_count = reinterpret_cast<uint32_t*>(base);
+  float* scratch = reinterpret_cast<float*>(base + 256);
+  uint8_t* p = base + lp.fixed;
+  float* sample = reinterpret_cast<float*>(p);                      p += static_cast<size_t>(R) * lp.sld * 4;
+  uint32_t* thresh = reinterpret_cast<uint32_t*>(p);                p += static_cast<size_t>(R) * 4;
+  uint32_t* counts = reinterpret_cast<uint32_t*>(p);                p += static_cast<size_t>(R) * 4;
+  int32_t* fail_rows = reinterpret_cast<int32_t*>(p);               p += static_cast<size_t>(R) * 4;
+  uint2* pairs = reinterpret_cast<uint2*>((reinterpret_cast<uintptr_t>(p) + 7) & ~uintptr_t(7));
+  const int sms = num_sms();
+  for (const RowChunk& c : chunks) {
+    e = cuda_check(cudaMemsetAsync(counts, 0, static_cast<size_t>(c.nrows) * 4, st), "clear pair counts");
+    if (e != HISA_OK) return e;
+    e = cuda_check(cudaMemsetAsync(fail_count, 0, 4, st), "clear fallback count");
+    if (e != HISA_OK) return e;
+    e = score_rows_tc_mode(s, q, qsc, w, k, ksc, nvis, lp.stride, c, sample, lp.sld, nullptr, nullptr, nullptr, 0, st);
+    if (e != HISA_OK) return e;
+    const unsigned tgrid = static_cast<unsigned>(std::min<int64_t>(c.nrows, static_cast<int64_t>(sms) * 16));
+    flat_thresh_kernel<32><<<tgrid, 128, 0, st>>>(sample, lp.sld, nvis, c.row0, c.nrows, s->num_keys, lp.stride, lp.cap,
+                                                  lp.r_target, thresh);
+    e = launch_check("flat_thresh_kernel");
+    if (e != HISA_OK) return e;
+    e = score_rows_tc_mode(s, q, qsc, w, k, ksc, nvis, 1, c, nullptr, 0, thresh, pairs, counts, lp.cap, st);
+    if (e != HISA_OK) return e;
+    const unsigned sgrid = static_cast<unsigned>(std::min<int64_t>(c.nrows, static_cast<int64_t>(sms) * 8));
+    if (lp.cap <= 256 * 16)
+      flat_pairs_select_kernel<16><<<sgrid, 256, 0, st>>>(pairs, counts, lp.cap, nvis, c.row0, c.nrows, s->num_keys,
+                                                          s->top_k, oi, os, fail_count, fail_rows);
+    else
+      flat_pairs_select_kernel<32><<<sgrid, 256, 0, st>>>(pairs, counts, lp.cap, nvis, c.row0, c.nrows, s->num_keys,
+                                                          s->top_k, oi, os, fail_count, fail_rows);
+    e = launch_check("flat_pairs_select_kernel");
+    if (e != HISA_OK) return e;
+    e = s->dtype == HISA_BF16
+            ? launch_flat_fallback<DT_BF16>(s, q, qsc, w, k, ksc, nvis, c.row0, fail_count, fail_rows, scratch,
+                                            lp.fb_ctas, oi, os, st)
+            : launch_flat_fallback<DT_E4M3>(s, q, qsc, w, k, ksc, nvis, c.row0, fail_count, fail_rows, scratch,
+                                            lp.fb_ctas, oi, os, st);
+    if (e != HISA_OK) return e;
+  }
+  return HISA_OK;
+}
+
 hisa_status check_indexer_ptrs(const hisa_shape* s, const void* q, const float* q_scale, const float* w,
                                const void* k, const float* k_scale, const int32_t* n_visible) {
   if (!q || !w || !k || !n_visible) return fail(HISA_ERR_INVALID_ARG, "q, w, keys and n_visible must be non-NULL");
@@ -380,12 +518,18 @@ hisa_status hisa_get_status(hisa_stream stream) {
 
 hisa_status hisa_workspace_size(int32_t op, const hisa_shape* s, size_t* bytes) {
   if (!bytes) return fail(HISA_ERR_INVALID_ARG, "bytes is NULL");
-  hisa_status e = check_shape(s, op != HISA_OP_FLAT_TOPK);
+  hisa_status e = check_shape(s, op != HISA_OP_FLAT_TOPK && op != HISA_OP_FLAT_TOPK_SAMPLED);
   if (e != HISA_OK) return e;
   switch (op) {
     case HISA_OP_FLAT_TOPK: *bytes = static_cast<size_t>(rows_of(s) * (pad4(s->num_keys) * 4 + 8)); return HISA_OK;
     case HISA_OP_BLOCK_SCORE_TOPM: *bytes = static_cast<size_t>(rows_of(s) * pad4(num_blocks(s)) * 4); return HISA_OK;
     case HISA_OP_TOKEN_SCORE_TOPK: *bytes = 0; return HISA_OK;
+    case HISA_OP_FLAT_TOPK_SAMPLED: {
+      LitePlan lp;
+      if (!lite_plan(s, &lp)) return fail(HISA_ERR_UNSUPPORTED, "shape not supported by the sampled flat top-k");
+      *bytes = lp.fixed + lp.per_row * static_cast<size_t>(rows_of(s));
+      return HISA_OK;
+    }
   }
   return fail(HISA_ERR_INVALID_ARG, "unknown op %d", op);
 }
@@ -584,6 +728,27 @@ hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale, const flo
     if (e != HISA_OK) return e;
   }
   return HISA_OK;
+}
+
+hisa_status dsa_flat_indexer_topk_sampled(const void* q, const float* q_scale, const float* w, const void* k,
+                                          const float* k_scale, const int32_t* n_visible, const hisa_shape* s,
+                                          int32_t* topk_idx, float* topk_score, void* workspace, size_t ws_bytes,
+                                          hisa_stream stream) {
+  hisa_status e = check_shape(s, false);
+  if (e != HISA_OK) return e;
+  e = check_indexer_ptrs(s, q, q_scale, w, k, k_scale, n_visible);
+  if (e != HISA_OK) return e;
+  if (!topk_idx || !aligned4(topk_idx)) return fail(HISA_ERR_INVALID_ARG, "topk_idx must be non-NULL, 4-byte aligned");
+  LitePlan lp;
+  if (!lite_plan(s, &lp))
+    return fail(HISA_ERR_UNSUPPORTED, "sampled flat top-k needs a tensor-core shape, num_keys divisible by the "
+                                      "sample stride and top_k small enough for the pair buffer");
+  if (!workspace || !aligned16(workspace)) return fail(HISA_ERR_WORKSPACE, "workspace must be non-NULL, 16-byte aligned");
+  if (ws_bytes < lp.fixed + lp.per_row * dense_group(s))
+    return fail(HISA_ERR_WORKSPACE, "workspace holds fewer than one query group (%zu bytes needed)",
+                lp.fixed + lp.per_row * dense_group(s));
+  return flat_lite(s, lp, q, q_scale, w, k, k_scale, n_visible, topk_idx, topk_score, workspace, ws_bytes,
+                   reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

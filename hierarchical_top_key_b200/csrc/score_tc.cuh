@@ -42,6 +42,7 @@ struct alignas(16) DenseSlot {
   int b, t0, nq, tile0, ntiles, pad0, pad1, pad2;
   int vis[kDenseMaxG];                    // visible key rows of each query of the group
   float qsc[kDenseMaxG];                  // E4M3 q scales (1 otherwise)
+  uint32_t thr[kDenseMaxG];               // compaction thresholds (ordering keys)
   float w[kDenseN];                       // [G][H] head weights (0 past the last query)
 };
 
@@ -50,6 +51,7 @@ struct DenseParams {
   int G;                    // queries per group (kDenseN / H)
   int groups_per_seq;
   int block_div;            // 0: flat (vis = n); > 0: coarse (vis = (n-1)/block_div)
+  int vis_stride;           // > 1: the key rows are every vis_stride-th key (vis = ceil(n / vis_stride))
   int kc_tiles;             // key tiles per work unit
   int max_chunks;           // units per group
   int stages;               // key-tile ring depth (<= 8)
@@ -64,6 +66,16 @@ struct DenseParams {
   float* out;
   int64_t ld;
   uint32_t* minmax;         // nullable: per output row, (min, max) ordering key written
+  int64_t ksc_ld;           // E4M3 key scales: key row s of sequence b has scale k_scale[b*ksc_ld + s*ksc_step]
+  int ksc_step;
+  // Compaction (thresh != nullptr): instead of score rows, each output row r
+  // receives the (key row, ordering key) pairs whose key is >= thresh[r],
+  // appended at pairs[r*cap ...] in any order; counts[r] counts them all
+  // (beyond cap the pairs are dropped but still counted).
+  const uint32_t* thresh;
+  uint2* pairs;
+  uint32_t* counts;
+  int cap;
 };
 
 struct DenseUnit {
@@ -72,6 +84,7 @@ struct DenseUnit {
 
 __device__ __forceinline__ int dense_vis(const DenseParams& p, int n) {
   int v = p.block_div > 0 ? (n > 0 ? (n - 1) / p.block_div : 0) : n;
+  if (p.vis_stride > 1) v = n > 0 ? (n + p.vis_stride - 1) / p.vis_stride : 0;
   return max(0, min(v, p.L));
 }
 
@@ -159,6 +172,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
       if (lane < kDenseMaxG) {
         S.vis[lane] = vis;
         S.qsc[lane] = (DT == DT_E4M3 && lane < nq) ? __ldg(p.q_scale + qrow0 + lane) : 1.f;
+        S.thr[lane] = (p.thresh != nullptr && lane < nq) ? __ldg(p.thresh + qrow0 + lane - p.row0) : 0u;
       }
       for (int i = lane; i < G * H; i += 32) {
         const int j = i / H;
@@ -286,9 +300,27 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
       const float* w_w = S.w + half * QPT * H;
       const float* qsc_w = S.qsc + half * QPT;
       const int* vis_w = S.vis + half * QPT;
+      const uint32_t* thr_w = S.thr + half * QPT;
       uint32_t kmin[QPT], kmax[QPT];
 #pragma unroll
       for (int jq = 0; jq < QPT; ++jq) { kmin[jq] = 0xFFFFFFFFu; kmax[jq] = 0u; }
+      // compaction: a tile's appends are reserved (lane 0's atomic) while the
+      // tile is scored and written out one tile later, so the atomic's latency
+      // hides behind the next tile's work
+      uint32_t pball[QPT], pkey[QPT], pbase[QPT];
+      int ps = 0;
+#pragma unroll
+      for (int jq = 0; jq < QPT; ++jq) pball[jq] = 0u;
+      auto flush = [&]() {
+#pragma unroll
+        for (int jq = 0; jq < QPT; ++jq) {
+          if (pball[jq] == 0u) continue;
+          const uint32_t slot = __shfl_sync(0xffffffffu, pbase[jq], 0) + __popc(pball[jq] & ((1u << lane) - 1u));
+          if (((pball[jq] >> lane) & 1u) && slot < static_cast<uint32_t>(p.cap))
+            p.pairs[(qrow0 + half * QPT + jq - p.row0) * p.cap + slot] = make_uint2(ps, pkey[jq]);
+          pball[jq] = 0u;
+        }
+      };
       for (int i = 0; i < U.ntiles; ++i, ++tc) {
         const int ab = static_cast<int>(tc & 1);
         int okl = 1;
@@ -298,8 +330,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
         tc_fence_after();
         const int s = (U.tile0 + i) * kDenseTileM + quarter * 32 + lane;
         float ksc = 1.f;
-        if (DT == DT_E4M3 && s < p.L) ksc = __ldg(p.k_scale + static_cast<int64_t>(U.b) * p.L + s);
+        if (DT == DT_E4M3 && s < p.L)
+          ksc = __ldg(p.k_scale + static_cast<int64_t>(U.b) * p.ksc_ld + static_cast<int64_t>(s) * p.ksc_step);
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + ab * kDenseN;
+        uint32_t nball[QPT], nkey[QPT], nbase[QPT];
 #pragma unroll
         for (int jq = 0; jq < QPT; ++jq) {
           const int j = half * QPT + jq;
@@ -331,10 +365,18 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
 #pragma unroll
             for (int c = 0; c < 16; ++c) acc = fmaf(wq[c], fmaxf(__uint_as_float(v[c]), 0.f), acc);
           }
-          if (s < vis_w[jq]) {
-            if (DT == DT_E4M3) acc *= qsc_w[jq] * ksc;
+          if (DT == DT_E4M3) acc *= qsc_w[jq] * ksc;
+          const uint32_t key = float_key(acc);
+          if (p.thresh != nullptr) {
+            // warp-aggregated append of this tile's keys that pass the row's threshold
+            const bool take = s < vis_w[jq] && key >= thr_w[jq] && key != 0u;
+            nball[jq] = __ballot_sync(0xffffffffu, take);
+            nkey[jq] = key;
+            nbase[jq] = (lane == 0 && nball[jq] != 0u)
+                            ? atomicAdd(p.counts + (qrow0 + j - p.row0), static_cast<uint32_t>(__popc(nball[jq])))
+                            : 0u;
+          } else if (s < vis_w[jq]) {
             p.out[(qrow0 + j - p.row0) * p.ld + s] = acc;
-            const uint32_t key = float_key(acc);
             kmin[jq] = min(kmin[jq], key);
             kmax[jq] = max(kmax[jq], key);
           }
@@ -342,7 +384,14 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty + ab);
+        if (p.thresh != nullptr) {
+          flush();          // the previous tile's appends, reserved one tile ago
+#pragma unroll
+          for (int jq = 0; jq < QPT; ++jq) { pball[jq] = nball[jq]; pkey[jq] = nkey[jq]; pbase[jq] = nbase[jq]; }
+          ps = s;
+        }
       }
+      if (p.thresh != nullptr) flush();
       if (ok && p.minmax != nullptr) {
 #pragma unroll
         for (int jq = 0; jq < QPT; ++jq) {

@@ -85,7 +85,8 @@ typedef struct CUstream_st* hisa_stream;
 enum {
   HISA_OP_BLOCK_SCORE_TOPM = 1,
   HISA_OP_TOKEN_SCORE_TOPK = 2,
-  HISA_OP_FLAT_TOPK = 3
+  HISA_OP_FLAT_TOPK = 3,
+  HISA_OP_FLAT_TOPK_SAMPLED = 4
 };
 
 /*
@@ -207,6 +208,32 @@ HISA_API hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale,
                                   const hisa_shape* shape, int32_t* topk_idx,
                                   float* topk_score, void* workspace,
                                   size_t ws_bytes, hisa_stream stream);
+
+/*
+ * The flat indexer's top-k without score rows, after the sampled-range,
+ * write-back-only-promising-candidates scheme of "LITETOPK" (Indexer-TopK
+ * abstract): every 16th key (or sparser, so that at most 4096 are sampled) is
+ * scored; per query the r-th largest sample score is a threshold at or above
+ * which more than k keys lie with overwhelming probability; every key is then
+ * scored and only the (position, score) pairs at or above the threshold are
+ * written back and selected from.  Queries whose estimate misses (fewer than
+ * k pairs, or more than the pair buffer holds) are rescored on CUDA cores.
+ * The result is exactly dsa_flat_indexer_topk's; the workspace per query is
+ * the sample row plus the pair buffer instead of a full score row.
+ * Same arguments, layouts and errors as dsa_flat_indexer_topk; the workspace
+ * holds at least hisa_workspace_size(HISA_OP_FLAT_TOPK_SAMPLED) bytes (less
+ * runs the queries in chunks).  Tensor-core shapes only (bf16 / E4M3, head_dim
+ * x element size of 128 or 256 bytes, H in {16, 32, 64}) whose key count the
+ * sample stride divides and whose pair buffer (at most 8192 pairs) is smaller
+ * than num_keys; other shapes return HISA_ERR_UNSUPPORTED.
+ */
+HISA_API hisa_status dsa_flat_indexer_topk_sampled(const void* q, const float* q_scale,
+                                          const float* w, const void* k,
+                                          const float* k_scale,
+                                          const int32_t* n_visible,
+                                          const hisa_shape* shape, int32_t* topk_idx,
+                                          float* topk_score, void* workspace,
+                                          size_t ws_bytes, hisa_stream stream);
 
 /*
  * hisa_block_score_topm without a caller workspace, for callers that cannot
