@@ -200,6 +200,46 @@ def flat_query(q_t, w_t, keys, n_t: int, top_k: int):
     return pick.astype(np.int64), scores[pick]
 
 
+# ------------------------------------------------------------ three levels
+#
+# Coarse-to-fine over three levels ("LongCat Sparse Attention" abstract,
+# Hierarchical Indexing: a coarse-to-fine scoring scheme that narrows the
+# candidate set step by step), read here as HISA's coarse step applied twice:
+# super-blocks of `group` blocks are pooled from the keys like blocks are, the
+# current super-block plus the best of the fully visible ones are kept, the
+# fully visible blocks inside them are scored with their pooled keys, and the
+# current block plus the best of those go to the token stage.
+
+def candidate_blocks(superblocks: np.ndarray, c_t: int, group: int) -> np.ndarray:
+    """Fully visible blocks (b < c_t) inside the retained super-blocks, ascending."""
+    parts = [np.arange(u * group, min((u + 1) * group, c_t)) for u in sorted(superblocks)]
+    return np.concatenate(parts).astype(np.int64) if parts else np.zeros(0, np.int64)
+
+
+def select_blocks_among(q_t, w_t, kpool, cands: np.ndarray, c_t: int, top_m: int) -> np.ndarray:
+    """Second level: the current block plus the top_m-1 best candidate blocks
+    (every candidate when they fit), ascending; ties go to the lower block."""
+    if c_t < 0:
+        return np.zeros(0, np.int64)
+    if len(cands) + 1 <= top_m:
+        return np.sort(np.concatenate([cands, [c_t]])).astype(np.int64)
+    scores = indexer_scores(q_t, w_t, kpool[cands])
+    kept = cands[top_by_score(scores, top_m - 1)]
+    return np.sort(np.concatenate([kept, [c_t]])).astype(np.int64)
+
+
+def hisa3_query(q_t, w_t, keys, kpool, kpool2, n_t: int, block: int, group: int, top_m2: int,
+                top_m: int, top_k: int):
+    """Three-level indexer for one query -> (super-blocks, blocks, indices, scores).
+    kpool2 holds the pooled super-blocks (block * group keys each)."""
+    sb = select_blocks(q_t, w_t, kpool2, n_t, block * group, top_m2)
+    c = current_block(n_t, block)
+    blocks = select_blocks_among(q_t, w_t, kpool, candidate_blocks(sb, c, group), c, top_m)
+    cand = candidate_keys(blocks, n_t, block)
+    idx, sc = refine_tokens(q_t, w_t, keys, cand, top_k)
+    return sb, blocks, idx, sc
+
+
 def pad_row(values: np.ndarray, width: int, fill) -> np.ndarray:
     out = np.full(width, fill, dtype=np.asarray(values).dtype if len(values) else np.int64)
     out[:len(values)] = values

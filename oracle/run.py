@@ -67,6 +67,22 @@ class Sequence:
         cand = ho.candidate_keys(np.asarray(blocks, np.int64), int(self.n_visible[t]), self.block)
         return ho.refine_tokens(self.q[t], self.w[t], self.keys, cand, top_k or self.top_k)
 
+    def superblocks_pooled(self, group: int) -> np.ndarray:
+        """Pooled super-blocks of `group` blocks (pooled from the keys like blocks)."""
+        cache = self.__dict__.setdefault("_kpool2", {})
+        if group not in cache:
+            if self.fp8:
+                pc, ps = ho.pool_blocks_e4m3(self.k_codes, self.k_scale, self.block * group)
+                cache[group] = ho.dequantize_e4m3_rows(pc, ps)
+            else:
+                cache[group] = ho.pool_blocks(self.keys, self.block * group, self.workload.dtype)
+        return cache[group]
+
+    def hisa3(self, t: int, group: int, top_m2: int, top_m: int | None = None, top_k: int | None = None):
+        return ho.hisa3_query(self.q[t], self.w[t], self.keys, self.kpool, self.superblocks_pooled(group),
+                              int(self.n_visible[t]), self.block, group, top_m2, top_m or self.top_m,
+                              top_k or self.top_k)
+
     def scores(self, t: int, positions) -> np.ndarray:
         """Oracle indexer score of query t at the given key positions."""
         return ho.indexer_scores(self.q[t], self.w[t], self.keys[np.asarray(positions, np.int64)])

@@ -202,6 +202,85 @@ def pin_brute_force_hisa():
         assert set(idx.tolist()) == want, (trial, idx, want)
 
 
+def pin_brute_force_hisa3():
+    """Three levels on tiny inputs: every choice of m2-1 super-blocks, then of
+    m-1 blocks among their fully visible blocks, then of k candidates."""
+    rng = np.random.default_rng(21)
+    for trial in range(60):
+        B, S = int(rng.integers(1, 3)), int(rng.integers(1, 4))
+        L = int(rng.integers(1, 19))
+        H, d = int(rng.integers(1, 3)), int(rng.integers(1, 3))
+        m2, m, k = int(rng.integers(1, 4)), int(rng.integers(1, 5)), int(rng.integers(1, 6))
+        q = rng.integers(-2, 3, (H, d)).astype(np.float64)
+        w = rng.integers(0, 3, H).astype(np.float64)
+        keys = rng.integers(-3, 4, (L, d)).astype(np.float64)
+        nt = int(rng.integers(1, L + 1))
+
+        def pooled(size):
+            nb = -(-L // size)
+            out = np.zeros((nb, d))
+            for b in range(nb):
+                members = list(range(b * size, min((b + 1) * size, L)))
+                for i in range(d):
+                    out[b, i] = sum(keys[s, i] for s in members) / len(members)
+            return out.astype(np.float32).astype(np.float64)
+
+        kp, kp2 = pooled(B), pooled(B * S)
+        c2, c = (nt - 1) // (B * S), (nt - 1) // B
+        if c2 + 1 <= m2:
+            want_sb = set(range(c2 + 1))
+        else:
+            want_sb = _brute_topk(list(_loop_scores(q, w, kp2[:c2])), m2 - 1) | {c2}
+        cands = [b for u in sorted(want_sb) for b in range(u * S, min((u + 1) * S, c))]
+        if len(cands) + 1 <= m:
+            want_blocks = set(cands) | {c}
+        else:
+            bs = _loop_scores(q, w, kp[cands])
+            want_blocks = {cands[i] for i in _brute_topk(list(bs), m - 1)} | {c}
+        sb, blocks, idx, _ = ho.hisa3_query(q, w, keys, kp, kp2, nt, B, S, m2, m, k)
+        assert set(sb.tolist()) == want_sb, (trial, sb, want_sb)
+        assert set(blocks.tolist()) == want_blocks, (trial, blocks, want_blocks)
+        cand = [s for b in sorted(want_blocks) for s in range(b * B, min((b + 1) * B, nt))]
+        tok = _loop_scores(q, w, keys[cand]) if cand else np.zeros(0)
+        assert set(idx.tolist()) == {cand[i] for i in _brute_topk(list(tok), k)}, trial
+
+
+def pin_three_levels_reduce_to_two():
+    """Every super-block kept, or super-blocks of one block with m2 = m: the
+    three-level indexer is HISA exactly."""
+    inp = synthetic.generate(synthetic.small_case(num_keys=700, heads=3, head_dim=8, block_size=16,
+                                                  top_m=5, top_k=40, needles=3))
+    seq = Sequence(inp, 0)
+    for t in range(0, 700, 9):
+        blocks, hi, hs = seq.hisa(t)
+        _, b3, i3, s3 = seq.hisa3(t, group=4, top_m2=1000)
+        assert list(b3) == list(blocks) and list(i3) == list(hi), t
+        np.testing.assert_array_equal(s3, hs)
+        _, b1, i1, _ = seq.hisa3(t, group=1, top_m2=5)
+        assert list(b1) == list(blocks) and list(i1) == list(hi), t
+
+
+def pin_three_levels_structure():
+    """The kept blocks lie in the kept super-blocks, the current block is kept,
+    and every candidate block left out scores no higher than the kept ones."""
+    inp = synthetic.generate("tiny")
+    seq = Sequence(inp, 0)
+    B, S = inp.workload.block_size, 2
+    for t in [0, 1, 63, 64, 200, 511, 700, 1023]:
+        nt = int(seq.n_visible[t])
+        sb, blocks, idx, _ = seq.hisa3(t, group=S, top_m2=3, top_m=3)
+        c = ho.current_block(nt, B)
+        assert c in set(blocks.tolist())
+        assert all(b // S in set(sb.tolist()) for b in blocks.tolist())
+        cands = ho.candidate_blocks(sb, c, S)
+        kept = [b for b in blocks.tolist() if b != c]
+        if len(cands) + 1 > 3 and kept:
+            sc = ho.indexer_scores(seq.q[t], seq.w[t], seq.kpool[cands])
+            low = min(sc[list(cands).index(b)] for b in kept)
+            assert all(sc[i] <= low for i, b in enumerate(cands) if b not in kept), t
+        assert set(idx.tolist()) <= set(ho.candidate_keys(blocks, nt, B).tolist())
+
+
 # ---------------------------------------------------------------- closed forms / special cases
 
 

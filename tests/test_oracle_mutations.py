@@ -69,6 +69,19 @@ def _bf16_via_fp32(x):
     return _orig_bf16(np.asarray(x, np.float64).astype(np.float32).astype(np.float64))
 
 
+def _superblock_leaky(superblocks, c_t, group):
+    # also takes the current block and the partial blocks after it
+    parts = [np.arange(u * group, (u + 1) * group) for u in sorted(superblocks)]
+    return np.concatenate(parts).astype(np.int64) if parts else np.zeros(0, np.int64)
+
+
+def _second_level_unforced(q_t, w_t, kpool, cands, c_t, top_m):
+    if c_t < 0 or len(cands) == 0:
+        return np.zeros(0, np.int64)
+    s = ho.indexer_scores(q_t, w_t, kpool[cands])
+    return np.sort(cands[ho.top_by_score(s, top_m)]).astype(np.int64)
+
+
 _orig_e4m3 = ofp8.e4m3_encode
 _orig_bf16 = ofp8.bf16_round
 
@@ -81,6 +94,8 @@ MUTATIONS = {
     "pool_sum_not_mean": [(ho, "block_means", _block_sums)],
     "block_score_abs": [(ho, "select_blocks", _mean_of_relu_blocks)],
     "causal_leak": [(ho, "candidate_keys", _cand_leaky)],
+    "three_levels_partial_blocks": [(ho, "candidate_blocks", _superblock_leaky)],
+    "three_levels_current_not_forced": [(ho, "select_blocks_among", _second_level_unforced)],
     "e4m3_ties_away": [(ofp8, "e4m3_encode", _e4m3_half_away), (ho, "e4m3_encode", _e4m3_half_away)],
     "bf16_double_rounding": [(ofp8, "bf16_round", _bf16_via_fp32), (ho, "bf16_round", _bf16_via_fp32)],
 }
