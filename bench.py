@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-flat", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--superblock-group", type=int, default=0,
+                    help="also time the three-level indexer with super-blocks of this many blocks")
+    ap.add_argument("--top-m2", type=int, default=8, help="super-blocks kept by the three-level indexer")
     return ap.parse_args()
 
 
@@ -212,6 +215,36 @@ def workload_config(wl, fp8):
             "raw_keys": wl.raw_keys, "queries_per_seq": wl.num_queries, "first_query_pos": wl.first_query_pos,
             "heads": wl.heads, "head_dim": wl.head_dim, "block_size": wl.block_size, "top_m": wl.top_m,
             "top_k": wl.top_k, "l2": "flushed between steps (256 MiB write, outside the timed events)"}
+
+
+def graph_ms(step, steps, flush, stream):
+    """Mean device time of `step` replayed from a CUDA graph (launch-bound
+    decode steps: no host work between the kernels), L2 flushed between
+    replays outside the timed events."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()                                   # warm the allocator on the capture stream
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        step()
+    g.replay()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    del g
+    return ms
 
 
 # ------------------------------------------------------------------ ranks
@@ -412,10 +445,77 @@ def main():
         barrier()
         hb.get_status()
         cm = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in cev])), world, dev)
+        cg = max_over_ranks(graph_ms(cached_step, args.steps, flush, stream), world, dev)
         cached = {"ms_per_layer": cm, "queries_per_s": job_rate(queries, world, cm),
                   "hisa_speedup": (flat["ms_per_layer"] / cm) if flat else None,
+                  "graph_ms_per_layer": cg, "graph_hisa_speedup": (flat["ms_per_layer"] / cg) if flat else None,
                   "what": "pooled keys of complete blocks kept between decode steps; a step pools the one block "
                           "its new key completes, then scores blocks and refines"}
+
+    # ---- three levels: pooled super-blocks -> blocks -> tokens
+    three = None
+    if args.superblock_group > 0 and not fp8 and wl.compress_ratio == 1:
+        G3 = args.superblock_group
+        ix3 = hb.HisaIndexer3(wl.block_size, G3, args.top_m2, wl.top_m, wl.top_k)
+        for _ in range(max(3, args.warmup)):
+            ix3(q, w, k_static, nv)
+        barrier()
+        tev = []
+        for i in range(args.steps):
+            flush.zero_()
+            a, b = ev(), ev()
+            a.record(stream)
+            idx3 = ix3(q, w, k_static, nv)
+            b.record(stream)
+            tev.append((a, b))
+        barrier()
+        hb.get_status()
+        tm = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in tev])), world, dev)
+        # overlap with the two-level and the flat indices on a sample of queries
+        idx2, _ = indexer(q, w, k_static, nv)
+        rows = np.random.default_rng(3).choice(wl.batch * wl.num_queries, min(256, wl.batch * wl.num_queries),
+                                               replace=False)
+        r3 = idx3.reshape(-1, wl.top_k)[torch.as_tensor(rows, device=dev)].cpu().numpy()
+        r2 = idx2.reshape(-1, wl.top_k)[torch.as_tensor(rows, device=dev)].cpu().numpy()
+        iou = lambda x, y: len(set(x[x >= 0]) & set(y[y >= 0])) / max(1, len(set(x[x >= 0]) | set(y[y >= 0])))  # noqa: E731
+        three = {"group": G3, "top_m2": args.top_m2, "ms_per_layer": tm, "queries_per_s": job_rate(queries, world, tm),
+                 "hisa_speedup": (flat["ms_per_layer"] / tm) if flat else None,
+                 "iou_vs_two_level": float(np.mean([iou(r3[i], r2[i]) for i in range(len(rows))]))}
+        if not args.no_flat:
+            fidx, _ = hb.dsa_flat_indexer_topk(q, w, k_static, nv, top_k=wl.top_k, workspace=ws_flat)
+            rf = fidx.reshape(-1, wl.top_k)[torch.as_tensor(rows, device=dev)].cpu().numpy()
+            three["iou_vs_flat"] = float(np.mean([iou(r3[i], rf[i]) for i in range(len(rows))]))
+            three["two_level_iou_vs_flat"] = float(np.mean([iou(r2[i], rf[i]) for i in range(len(rows))]))
+        if wl.num_queries == 1:
+            # decode with both pooled levels cached: a step pools the block and the
+            # super-block its new key completes
+            nb = -(-wl.num_keys // wl.block_size)
+            nb2 = -(-wl.num_keys // (wl.block_size * G3))
+            kc, _ = hb.hisa_pool_blocks(k_static, wl.block_size)
+            kc2, _ = hb.hisa_pool_blocks(k_static, wl.block_size * G3)
+
+            def cached3():
+                hb.hisa_pool_blocks_range(k_static, wl.block_size, nb - 1, 1, kc)
+                hb.hisa_pool_blocks_range(k_static, wl.block_size * G3, nb2 - 1, 1, kc2)
+                return ix3(q, w, k_static, nv, kpool=(kc, None), kpool2=(kc2, None))
+
+            for _ in range(3):
+                cached3()
+            barrier()
+            cev3 = []
+            for i in range(args.steps):
+                flush.zero_()
+                a, b = ev(), ev()
+                a.record(stream)
+                cached3()
+                b.record(stream)
+                cev3.append((a, b))
+            barrier()
+            hb.get_status()
+            three["cached_ms_per_layer"] = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in cev3])),
+                                                          world, dev)
+            three["cached_graph_ms_per_layer"] = max_over_ranks(graph_ms(cached3, args.steps, flush, stream),
+                                                                world, dev)
 
     # ---- end to end through the public API with pinned host buffers
     e2e = None
@@ -492,7 +592,8 @@ def main():
             "config": workload_config(wl, fp8),
             "stages_ms": {"pool": float(np.mean(stage_ms[:, 0])), "block_score_topm": float(np.mean(stage_ms[:, 1])),
                           "token_score_topk": tok_ms},
-            "flat": flat, "pooled_keys_cached": cached, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "flat": flat, "pooled_keys_cached": cached, "three_level": three, "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clocks.summary(), "gpu_launches": launches_per_step * args.steps,
         }
         print(json.dumps(line))

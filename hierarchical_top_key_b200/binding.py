@@ -23,7 +23,7 @@ import torch
 from . import build as _build
 
 HISA_F32, HISA_BF16, HISA_E4M3 = 0, 1, 2
-OP_BLOCK, OP_TOKEN, OP_FLAT, OP_FLAT_SAMPLED = 1, 2, 3, 4
+OP_BLOCK, OP_TOKEN, OP_FLAT, OP_FLAT_SAMPLED, OP_BLOCK_REFINE = 1, 2, 3, 4, 5
 STATUS = {0: "HISA_OK", 1: "HISA_ERR_INVALID_ARG", 2: "HISA_ERR_UNSUPPORTED", 3: "HISA_ERR_WORKSPACE",
           4: "HISA_ERR_CUDA", 5: "HISA_ERR_TIMEOUT"}
 
@@ -48,6 +48,8 @@ _SIGS = {
                            ctypes.c_int32, _P],
     "hisa_quantize_e4m3": [_P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _P, _P, _P],
     "hisa_block_score_topm": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, ctypes.c_size_t, _P],
+    "hisa_block_refine_topm": [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(Shape), _P,
+                               _P, ctypes.c_size_t, _P],
     "hisa_block_score_topm_static": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P],
     "hisa_token_score_topk": [_P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t,
                               _P],
@@ -278,6 +280,47 @@ def dsa_flat_indexer_topk_sampled(q, w, k, n_visible, *, top_k: int, q_scale=Non
                                                 idx.data_ptr(), _ptr(sc), ws.data_ptr(), ws.numel(), _stream()),
            "dsa_flat_indexer_topk_sampled")
     return idx, sc
+
+
+def hisa_block_refine_topm(q, w, kpool, n_visible, superblock_idx, *, num_keys: int, block_size: int, top_m: int,
+                           group: int, q_scale=None, kpool_scale=None, workspace: Optional[torch.Tensor] = None):
+    """Second level of the three-level indexer: block_idx [batch, Q, top_m] int32
+    (current block first, -1 padded) from the retained super-blocks."""
+    b, Q, H, d = q.shape
+    top_m2 = superblock_idx.shape[-1]
+    shape = Shape(b, num_keys, Q, H, d, block_size, top_m, 1, dtype_code(q))
+    _need(superblock_idx, "superblock_idx", 3)
+    out = torch.empty((b, Q, top_m), dtype=torch.int32, device=q.device)
+    ws = workspace if workspace is not None else _workspace(workspace_size(OP_BLOCK_REFINE, shape), q.device)
+    _check(load().hisa_block_refine_topm(q.data_ptr(), _ptr(q_scale), w.data_ptr(), kpool.data_ptr(),
+                                         _ptr(kpool_scale), n_visible.data_ptr(), superblock_idx.data_ptr(), top_m2,
+                                         group, ctypes.byref(shape), out.data_ptr(), ws.data_ptr(), ws.numel(),
+                                         _stream()), "hisa_block_refine_topm")
+    return out
+
+
+class HisaIndexer3:
+    """Three-level indexer for one layer: pooled super-blocks (top_m2 kept) ->
+    blocks inside them (top_m kept) -> tokens (top_k).  Super-blocks are runs
+    of `group` blocks."""
+
+    def __init__(self, block_size: int, group: int, top_m2: int, top_m: int, top_k: int):
+        self.block_size, self.group, self.top_m2 = block_size, group, top_m2
+        self.top_m, self.top_k = top_m, top_k
+
+    def __call__(self, q, w, k, n_visible, q_scale=None, k_scale=None, kpool=None, kpool2=None, return_blocks=False):
+        """kpool / kpool2: (pooled keys, scales) of blocks and super-blocks when
+        the caller keeps them (a decoder's cache); pooled here otherwise."""
+        B, L = self.block_size, k.shape[1]
+        kp, kps = kpool if kpool is not None else hisa_pool_blocks(k, B, k_scale)
+        kp2, kps2 = kpool2 if kpool2 is not None else hisa_pool_blocks(k, B * self.group, k_scale)
+        sb = hisa_block_score_topm(q, w, kp2, n_visible, num_keys=L, block_size=B * self.group, top_m=self.top_m2,
+                                   q_scale=q_scale, kpool_scale=kps2)
+        blocks = hisa_block_refine_topm(q, w, kp, n_visible, sb, num_keys=L, block_size=B, top_m=self.top_m,
+                                        group=self.group, q_scale=q_scale, kpool_scale=kps)
+        idx, _ = hisa_token_score_topk(q, w, k, n_visible, blocks, block_size=B, top_k=self.top_k, q_scale=q_scale,
+                                       k_scale=k_scale)
+        return (idx, sb, blocks) if return_blocks else idx
 
 
 class HisaIndexer:

@@ -524,6 +524,9 @@ hisa_status hisa_workspace_size(int32_t op, const hisa_shape* s, size_t* bytes) 
     case HISA_OP_FLAT_TOPK: *bytes = static_cast<size_t>(rows_of(s) * (pad4(s->num_keys) * 4 + 8)); return HISA_OK;
     case HISA_OP_BLOCK_SCORE_TOPM: *bytes = static_cast<size_t>(rows_of(s) * pad4(num_blocks(s)) * 4); return HISA_OK;
     case HISA_OP_TOKEN_SCORE_TOPK: *bytes = 0; return HISA_OK;
+    case HISA_OP_BLOCK_REFINE_TOPM:
+      *bytes = static_cast<size_t>(pad4(rows_of(s)) * 4 + rows_of(s) * std::max(s->top_m - 1, 1) * 4);
+      return HISA_OK;
     case HISA_OP_FLAT_TOPK_SAMPLED: {
       LitePlan lp;
       if (!lite_plan(s, &lp)) return fail(HISA_ERR_UNSUPPORTED, "shape not supported by the sampled flat top-k");
@@ -560,6 +563,27 @@ hisa_status hisa_pool_blocks_range(const void* k, const float* k_scale, void* kp
   const int grid = static_cast<int>(std::min<int64_t>(ceil_div(threads_total, 256), 148 * 64));
   const uint8_t* in = static_cast<const uint8_t*>(k);
   uint8_t* out = static_cast<uint8_t*>(kpool);
+  if (s->block_size >= 512) {
+    // long groups (super-blocks): one CTA per pooled row, the rows split over its threads
+    const int wgrid = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(s->batch) * count, num_sms() * 8));
+    switch (s->dtype) {
+      case HISA_F32:
+        segment_mean_wide_kernel<DT_F32><<<wgrid, 256, 0, st>>>(in, nullptr, out, nullptr, s->batch, s->num_keys, nb,
+                                                                s->head_dim, s->block_size, first, count);
+        break;
+      case HISA_BF16:
+        segment_mean_wide_kernel<DT_BF16><<<wgrid, 256, 0, st>>>(in, nullptr, out, nullptr, s->batch, s->num_keys,
+                                                                 nb, s->head_dim, s->block_size, first, count);
+        break;
+      case HISA_E4M3:
+        segment_mean_wide_kernel<DT_E4M3><<<wgrid, 256, 0, st>>>(in, k_scale, out, kpool_scale, s->batch,
+                                                                 s->num_keys, nb, s->head_dim, s->block_size, first,
+                                                                 count);
+        break;
+      default: return fail(HISA_ERR_INVALID_ARG, "unknown dtype %d", s->dtype);
+    }
+    return launch_check("segment_mean_wide_kernel");
+  }
   switch (s->dtype) {
     case HISA_F32:
       segment_mean_kernel<DT_F32><<<grid, 256, 0, st>>>(in, nullptr, out, nullptr, s->batch, s->num_keys, nb,
@@ -684,6 +708,49 @@ hisa_status hisa_token_score_topk(const void* q, const float* q_scale, const flo
     case HISA_BF16: return token_simt_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
     default: return token_simt_h<DT_E4M3>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
   }
+}
+
+hisa_status hisa_block_refine_topm(const void* q, const float* q_scale, const float* w, const void* kpool,
+                                   const float* kpool_scale, const int32_t* n_visible,
+                                   const int32_t* superblock_idx, int32_t top_m2, int32_t group,
+                                   const hisa_shape* s, int32_t* block_idx, void* workspace, size_t ws_bytes,
+                                   hisa_stream stream) {
+  hisa_status e = check_shape(s, true);
+  if (e != HISA_OK) return e;
+  if (group < 1 || top_m2 < 1) return fail(HISA_ERR_INVALID_ARG, "group and top_m2 must be >= 1");
+  if (!superblock_idx || !block_idx) return fail(HISA_ERR_INVALID_ARG, "superblock_idx and block_idx must be non-NULL");
+  const int64_t nb = num_blocks(s);
+  // level two is the refinement stage run over the pooled blocks: "keys" are
+  // pooled blocks, its "blocks" are super-blocks of `group` pooled blocks,
+  // visibility is the count of fully visible blocks and k is top_m - 1
+  hisa_shape s2 = *s;
+  s2.num_keys = static_cast<int32_t>(nb);
+  s2.block_size = group;
+  s2.top_m = top_m2;
+  s2.top_k = s->top_m - 1;
+  e = check_indexer_ptrs(s, q, q_scale, w, kpool, kpool_scale, n_visible);
+  if (e != HISA_OK) return e;
+  const int64_t rows = rows_of(s);
+  size_t need = 0;
+  e = hisa_workspace_size(HISA_OP_BLOCK_REFINE_TOPM, s, &need);
+  if (e != HISA_OK) return e;
+  if (!workspace || !aligned16(workspace) || ws_bytes < need)
+    return fail(HISA_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned)", need);
+  int32_t* nvb = static_cast<int32_t*>(workspace);
+  int32_t* sel = nvb + pad4(rows);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int grid = static_cast<int>(std::min<int64_t>(ceil_div(rows, 256), 4096));
+  visible_blocks_kernel<<<grid, 256, 0, st>>>(n_visible, rows, s->num_keys, s->block_size, nvb);
+  e = launch_check("visible_blocks_kernel");
+  if (e != HISA_OK) return e;
+  if (s->top_m > 1) {
+    e = hisa_token_score_topk(q, q_scale, w, kpool, kpool_scale, nvb, superblock_idx, &s2, sel, nullptr, nullptr, 0,
+                              stream);
+    if (e != HISA_OK) return e;
+  }
+  assemble_blocks_kernel<<<grid, 256, 0, st>>>(n_visible, s->top_m > 1 ? sel : nullptr, rows, s->num_keys,
+                                              s->block_size, s->top_m, block_idx);
+  return launch_check("assemble_blocks_kernel");
 }
 
 hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale, const float* w, const void* k,

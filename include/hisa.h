@@ -86,7 +86,8 @@ enum {
   HISA_OP_BLOCK_SCORE_TOPM = 1,
   HISA_OP_TOKEN_SCORE_TOPK = 2,
   HISA_OP_FLAT_TOPK = 3,
-  HISA_OP_FLAT_TOPK_SAMPLED = 4
+  HISA_OP_FLAT_TOPK_SAMPLED = 4,
+  HISA_OP_BLOCK_REFINE_TOPM = 5
 };
 
 /*
@@ -208,6 +209,30 @@ HISA_API hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale,
                                   const hisa_shape* shape, int32_t* topk_idx,
                                   float* topk_score, void* workspace,
                                   size_t ws_bytes, hisa_stream stream);
+
+/*
+ * Three-level indexer, second level ("LongCat Sparse Attention" abstract,
+ * Hierarchical Indexing: coarse-to-fine scoring that narrows the candidate
+ * set step by step; here HISA's coarse step applied twice).  Super-blocks are
+ * runs of `group` blocks (pooled with hisa_pool_blocks at block_size
+ * B * group) and superblock_idx [batch, Q, top_m2] is what
+ * hisa_block_score_topm returns for them (current super-block forced).  For
+ * each query, the fully visible blocks (b < c_t) inside its retained
+ * super-blocks are scored with their pooled keys kpool [batch, ceil(L/B), d]
+ * (+ kpool_scale for E4M3); block_idx [batch, Q, top_m] receives the current
+ * block c_t first, then the top_m-1 best of them by (score desc, block asc),
+ * all of them when they fit, -1 padding.  The shape is the indexer's (block
+ * size B, top_m m).  Workspace: hisa_workspace_size(HISA_OP_BLOCK_REFINE_TOPM)
+ * bytes, 16-byte aligned.  Runs hisa_token_score_topk over the pooled blocks,
+ * so its limits apply with block_size = group, top_m = top_m2 and
+ * top_k = top_m - 1.
+ */
+HISA_API hisa_status hisa_block_refine_topm(const void* q, const float* q_scale, const float* w,
+                                            const void* kpool, const float* kpool_scale,
+                                            const int32_t* n_visible, const int32_t* superblock_idx,
+                                            int32_t top_m2, int32_t group, const hisa_shape* shape,
+                                            int32_t* block_idx, void* workspace, size_t ws_bytes,
+                                            hisa_stream stream);
 
 /*
  * The flat indexer's top-k without score rows, after the sampled-range,

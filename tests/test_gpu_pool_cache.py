@@ -62,3 +62,26 @@ def test_block_range_pooling_builds_the_same_cache(lib, fp8):
             np.testing.assert_array_equal(cache_s[b].cpu().numpy(), seq.kpool_scale)
         else:
             np.testing.assert_array_equal(cache[b].float().cpu().numpy().astype(np.float64), seq.kpool)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_long_groups_pool_like_the_oracle(lib, fp8):
+    """Super-block pooling (groups of 1024 keys, the one-CTA-per-row kernel),
+    including a ragged last group, is the oracle's exact mean."""
+    from hierarchical_top_key_b200 import binding as hb
+    from oracle import hisa_oracle as ho
+    wl = synthetic.small_case(batch=2, num_keys=3000, heads=4, head_dim=128, block_size=64, top_m=3, top_k=40,
+                              dtype="bf16", needles=2, name="pool_long")
+    inp = synthetic.generate(wl)
+    dev = hb.to_device_inputs(inp, fp8=fp8)
+    kp, kps = hb.hisa_pool_blocks(dev["k"], 1024, dev["k_scale"])
+    hb.get_status()
+    for b in range(wl.batch):
+        seq = Sequence(inp, b, fp8=fp8)
+        if fp8:
+            pc, ps = ho.pool_blocks_e4m3(seq.k_codes, seq.k_scale, 1024)
+            np.testing.assert_array_equal(kp[b].cpu().numpy(), pc)
+            np.testing.assert_array_equal(kps[b].cpu().numpy(), ps)
+        else:
+            np.testing.assert_array_equal(kp[b].float().cpu().numpy().astype(np.float64),
+                                          ho.pool_blocks(seq.keys, 1024, "bf16"))
