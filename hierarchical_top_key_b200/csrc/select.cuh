@@ -467,6 +467,135 @@ struct TwoPassSmem {
   uint32_t count;
 };
 
+// two_pass_topk over a 16-byte aligned fp32 row, reading it as float4 and two
+// of them per thread per step: a row of scores is streamed from DRAM, and one
+// 4-byte load in flight per thread leaves the selection latency-bound at a
+// fraction of the bandwidth.  Same contract as two_pass_topk.
+template <class Emit, class Grp>
+__device__ bool two_pass_topk_rows(const float* __restrict__ row, int n, uint32_t k, Emit emit, SelectSmem& sm,
+                                   uint32_t* buf_key, int32_t* buf_pos, uint32_t* buf_count, int cap,
+                                   uint32_t kmin, uint32_t kmax) {
+  const int lane = Grp::tid() & 31, tid = Grp::tid(), nt = Grp::size();
+  const int nbins = kDigitBins;
+  const float smin = key_float(kmin), smax = key_float(kmax);
+  float scale = smax > smin ? static_cast<float>(nbins) / (smax - smin) : 0.f;
+  if (!(scale < 1e30f)) scale = 0.f;
+  // bin = nearest integer to (score - smin) * scale, by adding 2^23 and reading
+  // the low mantissa bits: monotone in the score (so in the ordering key) and
+  // free of the float-to-int conversion; computed from the score itself
+  const float bias = 8388608.0f - smin * scale;
+  const uint32_t top_bin = static_cast<uint32_t>(nbins - 1);
+  auto bin_of = [&](float v) -> uint32_t {
+    const int b = static_cast<int>(__float_as_uint(fmaf(v, scale, bias)) - 0x4B000000u);
+    return min(static_cast<uint32_t>(max(b, 0)), top_bin);
+  };
+  // -0 scores bin like +0 (their ordering keys are equal); scores past n are skipped
+  auto load8 = [&](int p0, float (&v)[8], uint32_t& valid) {
+    valid = 0u;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int p = p0 + 4 * h;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (p + 3 < n) {
+        x = __ldcg(reinterpret_cast<const float4*>(row + p));
+        valid |= 0xFu << (4 * h);
+      } else {
+        if (p < n) { x.x = __ldcg(row + p); valid |= 1u << (4 * h); }
+        if (p + 1 < n) { x.y = __ldcg(row + p + 1); valid |= 2u << (4 * h); }
+        if (p + 2 < n) { x.z = __ldcg(row + p + 2); valid |= 4u << (4 * h); }
+      }
+      v[4 * h + 0] = x.x; v[4 * h + 1] = x.y; v[4 * h + 2] = x.z; v[4 * h + 3] = x.w;
+    }
+  };
+  for (int i = tid; i < nbins; i += nt) sm.hist[i] = 0;
+  if (tid == 0) { *buf_count = 0; sm.n_slots = 0; }
+  Grp::sync();
+  for (int p0 = 8 * tid; p0 < n; p0 += 8 * nt) {
+    float v[8];
+    uint32_t valid;
+    load8(p0, v, valid);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if ((valid >> u) & 1u) atomicAdd(&sm.hist[bin_of(v[u])], 1u);
+  }
+  Grp::sync();
+  uint32_t remaining = k;
+  bin_search<Grp>(sm, nbins, remaining);
+  const uint32_t D = sm.digit, above = sm.above, n_eq = sm.at_digit;
+  remaining -= above;
+  Grp::sync();
+  const bool take_bin = n_eq == remaining;
+  if (!take_bin && n_eq > static_cast<uint32_t>(cap)) return false;
+  const uint32_t gt_floor = take_bin ? D : D + 1;
+  // pass 2: emit keys from the bins above the boundary (or from it too when
+  // all of it is taken) and buffer the boundary bin; most warp-steps find
+  // nothing to do and skip the slot bookkeeping
+  for (int b0 = 0; b0 < n; b0 += 8 * nt) {
+    const int p0 = b0 + 8 * tid;
+    float v[8];
+    uint32_t valid;
+    load8(p0, v, valid);
+    uint32_t gt_mask = 0u, eq_mask = 0u;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t b = bin_of(v[u]);
+      const bool ok = (valid >> u) & 1u;
+      gt_mask |= (ok && b >= gt_floor) ? 1u << u : 0u;
+      eq_mask |= (ok && !take_bin && b == D) ? 1u << u : 0u;
+    }
+    if (__any_sync(0xffffffffu, gt_mask != 0u)) {
+      // this warp's emissions for the step: count, one reservation, prefix
+      const uint32_t cnt = __popc(gt_mask);
+      uint32_t incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      uint32_t base = 0;
+      if (lane == 31) base = atomicAdd(&sm.n_slots, incl);
+      base = __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
+      for (uint32_t m = gt_mask; m; m &= m - 1) {
+        const int u = __ffs(m) - 1;
+        emit(base++, p0 + u, float_key(v[u]));
+      }
+    }
+    if (__any_sync(0xffffffffu, eq_mask != 0u)) {
+      const uint32_t cnt = __popc(eq_mask);
+      uint32_t incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      uint32_t base = 0;
+      if (lane == 31) base = atomicAdd(buf_count, incl);
+      base = __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
+      for (uint32_t m = eq_mask; m; m &= m - 1) {
+        const int u = __ffs(m) - 1;
+        buf_key[base] = float_key(v[u]);
+        buf_pos[base] = p0 + u;
+        ++base;
+      }
+    }
+  }
+  Grp::sync();
+  if (take_bin) return true;
+  const int nb = static_cast<int>(n_eq);
+  for (int e = tid; e < nb; e += nt) {
+    const uint32_t ke = buf_key[e];
+    const int pe = buf_pos[e];
+    uint32_t rank = 0;
+    for (int f = 0; f < nb; ++f) {
+      const uint32_t kf = buf_key[f];
+      rank += (kf > ke || (kf == ke && buf_pos[f] < pe)) ? 1u : 0u;
+    }
+    if (rank < remaining) emit(above + rank, pe, ke);
+  }
+  Grp::sync();
+  return true;
+}
+
 // Flat DSA top-k over fp32 score rows: row r holds scores of keys 0..n_r-1.
 // `minmax` (nullable) holds, per row, the smallest and largest ordering key
 // the scoring kernel wrote; with it the row is read twice (histogram, then
@@ -491,9 +620,15 @@ __global__ void __launch_bounds__(512) flat_select_kernel(
   uint32_t nv = static_cast<uint32_t>(n);
   bool done = false;
   if (minmax != nullptr && n > top_k) {
-    done = two_pass_topk<decltype(key_at), decltype(emit), CtaGroup>(
-        key_at, n, static_cast<uint32_t>(top_k), emit, sm, tp.key, tp.pos, &tp.count, kTwoPassCap,
-        minmax[2 * blockIdx.x], minmax[2 * blockIdx.x + 1]);
+    // vectorised two passes (boundary bins up to 256 keys), then the general
+    // two passes (up to kTwoPassCap), then the radix select
+    done = two_pass_topk_rows<decltype(emit), CtaGroup>(row, n, static_cast<uint32_t>(top_k), emit, sm, tp.key,
+                                                         tp.pos, &tp.count, 256, minmax[2 * blockIdx.x],
+                                                         minmax[2 * blockIdx.x + 1]);
+    if (!done)
+      done = two_pass_topk<decltype(key_at), decltype(emit), CtaGroup>(
+          key_at, n, static_cast<uint32_t>(top_k), emit, sm, tp.key, tp.pos, &tp.count, kTwoPassCap,
+          minmax[2 * blockIdx.x], minmax[2 * blockIdx.x + 1]);
   }
   if (!done) nv = block_topk(key_at, n, static_cast<uint32_t>(top_k), emit, sm);
   for (int i = static_cast<int>(nv) + threadIdx.x; i < top_k; i += blockDim.x) {
