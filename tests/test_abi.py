@@ -52,6 +52,20 @@ def test_workspace_sizes(L):
     assert hb.workspace_size(hb.OP_BLOCK, s) == 6 * 16 * 4           # ceil(1001/64)=16
 
 
+def test_workspace_sizes_of_the_extensions(L):
+    s = _shape()
+    rows = s.batch * s.num_queries
+    # the second level of the three-level indexer: visible-block counts + (m-1) picks per row
+    assert hb.workspace_size(hb.OP_BLOCK_REFINE, s) == rows * 4 + rows * (s.top_m - 1) * 4
+    # the sampled flat top-k: a sample row and a pair buffer per query instead of a score row
+    sampled = hb.workspace_size(hb.OP_FLAT_SAMPLED, s)
+    assert 0 < sampled < hb.workspace_size(hb.OP_FLAT, s) // 2
+    # shapes it does not cover are refused before anything else
+    n = ctypes.c_size_t(0)
+    assert L.hisa_workspace_size(hb.OP_FLAT_SAMPLED, ctypes.byref(_shape(dtype=hb.HISA_F32)), ctypes.byref(n)) == 2
+    assert L.hisa_workspace_size(hb.OP_FLAT_SAMPLED, ctypes.byref(_shape(num_keys=32760)), ctypes.byref(n)) == 2
+
+
 @pytest.mark.parametrize("field,value,status", [
     ("head_dim", 96, 2), ("heads", 65, 2), ("heads", 0, 2), ("batch", 0, 1), ("top_k", 0, 1),
     ("dtype", 7, 1), ("block_size", 0, 1), ("top_m", 0, 1)])
