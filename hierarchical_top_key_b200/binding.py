@@ -246,9 +246,11 @@ def hisa_token_score_topk(q, w, k, n_visible, block_idx, *, block_size: int, top
     b, Q = q.shape[:2]
     idx = torch.empty((b, Q, top_k), dtype=torch.int32, device=q.device)
     sc = torch.empty((b, Q, top_k), dtype=torch.float32, device=q.device) if want_scores else None
+    need = workspace_size(OP_TOKEN, shape)
+    ws = _workspace(need, q.device) if need > 0 else None
     _check(load().hisa_token_score_topk(q.data_ptr(), _ptr(q_scale), w.data_ptr(), k.data_ptr(), _ptr(k_scale),
                                         n_visible.data_ptr(), block_idx.data_ptr(), ctypes.byref(shape),
-                                        idx.data_ptr(), _ptr(sc), None, 0, _stream()), "hisa_token_score_topk")
+                                        idx.data_ptr(), _ptr(sc), _ptr(ws), need, _stream()), "hisa_token_score_topk")
     return idx, sc
 
 

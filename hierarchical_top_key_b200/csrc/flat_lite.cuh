@@ -20,68 +20,6 @@
 
 namespace hisa {
 
-// Sum of one value per thread over a CTA of NT threads; every thread gets it.
-template <int NT>
-__device__ __forceinline__ uint32_t cta_sum(uint32_t v, uint32_t* red) {
-  v = __reduce_add_sync(0xffffffffu, v);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  uint32_t t = 0;
-#pragma unroll
-  for (int i = 0; i < NT / 32; ++i) t += red[i];
-  __syncthreads();
-  return t;
-}
-
-template <int NT>
-__device__ __forceinline__ uint32_t cta_max(uint32_t v, uint32_t* red) {
-  v = __reduce_max_sync(0xffffffffu, v);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  uint32_t t = 0;
-#pragma unroll
-  for (int i = 0; i < NT / 32; ++i) t = max(t, red[i]);
-  __syncthreads();
-  return t;
-}
-
-template <int NT>
-__device__ __forceinline__ uint32_t cta_min(uint32_t v, uint32_t* red) {
-  v = __reduce_min_sync(0xffffffffu, v);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  uint32_t t = 0xFFFFFFFFu;
-#pragma unroll
-  for (int i = 0; i < NT / 32; ++i) t = min(t, red[i]);
-  __syncthreads();
-  return t;
-}
-
-// The r-th largest of the CTA's keys (KPT per thread, 0 = absent; r >= 1 and
-// at most the number of present keys): bit by bit from the highest bit where
-// the smallest and largest keys differ, keeping a bit when at least r keys
-// are >= the value with it set.
-template <int NT, int KPT>
-__device__ uint32_t cta_rth_largest(const uint32_t (&key)[KPT], uint32_t r, uint32_t* red) {
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-#pragma unroll
-  for (int u = 0; u < KPT; ++u)
-    if (key[u] != 0u) { lo = min(lo, key[u]); hi = max(hi, key[u]); }
-  lo = cta_min<NT>(lo, red);
-  hi = cta_max<NT>(hi, red);
-  if (lo >= hi) return hi;
-  const int top = 31 - __clz(lo ^ hi);
-  uint32_t T = hi & ~((2u << top) - 1u);
-  for (int bit = top; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    uint32_t c = 0;
-#pragma unroll
-    for (int u = 0; u < KPT; ++u) c += key[u] >= cand ? 1u : 0u;
-    if (cta_sum<NT>(c, red) >= r) T = cand;
-  }
-  return T;
-}
-
 // Per query: the compaction threshold from its sample scores (row lr of
 // `sample`, sample j = key j*stride).  Queries whose whole visible prefix fits
 // the pair buffer take every key (threshold 1).

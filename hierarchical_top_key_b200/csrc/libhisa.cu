@@ -305,7 +305,7 @@ bool token_tc_ok(const hisa_shape* s) {
 template <int DT, int H>
 hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* k,
                             const float* ksc, const int32_t* nvis, const int32_t* bidx, int32_t* oi, float* os,
-                            cudaStream_t st) {
+                            cudaStream_t st, int parts = 1) {
   const int rb = s->head_dim * Elem<DT>::bytes;
   TokenParams p{};
   p.rows = rows_of(s);
@@ -313,6 +313,7 @@ hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc
   p.top_m = s->top_m; p.top_k = s->top_k;
   p.nb = static_cast<int>(num_blocks(s));
   p.max_cand = static_cast<int>(ceil_div(static_cast<int64_t>(s->top_m) * s->block_size, kTokTileM) * kTokTileM);
+  p.parts = parts;
   p.w = w; p.n_visible = nvis; p.block_idx = bidx; p.q_scale = qsc; p.k_scale = ksc; p.out_idx = oi; p.out_score = os;
   if (token_smem_bytes(rb, H, 2, p.max_cand) > kSmemBudget)
     return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size too large for the on-chip candidate buffers");
@@ -328,7 +329,7 @@ hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc
   e = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
                  "token_tc attribute");
   if (e != HISA_OK) return e;
-  const int grid = static_cast<int>(std::min<int64_t>(p.rows, num_sms()));
+  const int grid = static_cast<int>(std::min<int64_t>(p.rows * parts, num_sms()));
   kern<<<grid, kTokThreads, smem, st>>>(qm, km, p);
   return launch_check("token_tc_kernel");
 }
@@ -336,12 +337,28 @@ hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc
 template <int DT>
 hisa_status token_tc_h(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* k,
                        const float* ksc, const int32_t* nvis, const int32_t* bidx, int32_t* oi, float* os,
-                       cudaStream_t st) {
+                       cudaStream_t st, int parts = 1) {
   switch (s->heads) {
-    case 16: return launch_token_tc<DT, 16>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st);
-    case 32: return launch_token_tc<DT, 32>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st);
-    default: return launch_token_tc<DT, 64>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st);
+    case 16: return launch_token_tc<DT, 16>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st, parts);
+    case 32: return launch_token_tc<DT, 32>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st, parts);
+    default: return launch_token_tc<DT, 64>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st, parts);
   }
+}
+
+// Jobs per query of the tensor-core refinement stage: with few queries (a
+// decode step) each query's retained blocks are split over several CTAs, whose
+// top-k lists are merged exactly afterwards, so that more SMs gather keys.
+int token_parts(const hisa_shape* s) {
+  const int64_t rows = rows_of(s);
+  const int sms = num_sms();
+  if (!token_tc_ok(s) || rows * 2 > sms) return 1;
+  int parts = static_cast<int>(std::min<int64_t>({4, sms / rows, static_cast<int64_t>(s->top_m)}));
+  while (parts > 1 && static_cast<int64_t>(parts) * s->top_k > 8192) --parts;   // merge holds 8192 per row
+  return std::max(parts, 1);
+}
+
+size_t token_split_bytes(const hisa_shape* s, int parts) {
+  return parts > 1 ? static_cast<size_t>(rows_of(s)) * parts * s->top_k * 8 : 0;
 }
 
 // ------------------------------------------------------------ flat top-k without score rows
@@ -523,7 +540,7 @@ hisa_status hisa_workspace_size(int32_t op, const hisa_shape* s, size_t* bytes) 
   switch (op) {
     case HISA_OP_FLAT_TOPK: *bytes = static_cast<size_t>(rows_of(s) * (pad4(s->num_keys) * 4 + 8)); return HISA_OK;
     case HISA_OP_BLOCK_SCORE_TOPM: *bytes = static_cast<size_t>(rows_of(s) * pad4(num_blocks(s)) * 4); return HISA_OK;
-    case HISA_OP_TOKEN_SCORE_TOPK: *bytes = 0; return HISA_OK;
+    case HISA_OP_TOKEN_SCORE_TOPK: *bytes = token_split_bytes(s, token_parts(s)); return HISA_OK;
     case HISA_OP_BLOCK_REFINE_TOPM:
       *bytes = static_cast<size_t>(pad4(rows_of(s)) * 4 + rows_of(s) * std::max(s->top_m - 1, 1) * 4);
       return HISA_OK;
@@ -687,8 +704,6 @@ hisa_status hisa_token_score_topk(const void* q, const float* q_scale, const flo
                                   const float* k_scale, const int32_t* n_visible, const int32_t* block_idx,
                                   const hisa_shape* s, int32_t* topk_idx, float* topk_score, void* workspace,
                                   size_t ws_bytes, hisa_stream stream) {
-  (void)workspace;
-  (void)ws_bytes;
   hisa_status e = check_shape(s, true);
   if (e != HISA_OK) return e;
   e = check_indexer_ptrs(s, q, q_scale, w, k, k_scale, n_visible);
@@ -698,6 +713,26 @@ hisa_status hisa_token_score_topk(const void* q, const float* q_scale, const flo
   if (static_cast<int64_t>(s->top_m) * s->block_size > kMaxCandidates)
     return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size must be <= %d", kMaxCandidates);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int parts = token_parts(s);
+  if (parts > 1 && workspace && aligned16(workspace) && ws_bytes >= token_split_bytes(s, parts)) {
+    // split queries: every part's top-k with scores into the workspace, then the exact merge
+    const int64_t rows = rows_of(s);
+    int32_t* pidx = static_cast<int32_t*>(workspace);
+    float* psc = reinterpret_cast<float*>(pidx + rows * parts * s->top_k);
+    e = s->dtype == HISA_BF16
+            ? token_tc_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, pidx, psc, st, parts)
+            : token_tc_h<DT_E4M3>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, pidx, psc, st, parts);
+    if (e != HISA_OK) return e;
+    const int items = parts * s->top_k;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(rows, num_sms() * 4));
+    if (items <= 256 * 8)
+      merge_parts_kernel<8><<<grid, 256, 0, st>>>(pidx, psc, parts, rows, s->top_k, topk_idx, topk_score);
+    else if (items <= 256 * 16)
+      merge_parts_kernel<16><<<grid, 256, 0, st>>>(pidx, psc, parts, rows, s->top_k, topk_idx, topk_score);
+    else
+      merge_parts_kernel<32><<<grid, 256, 0, st>>>(pidx, psc, parts, rows, s->top_k, topk_idx, topk_score);
+    return launch_check("merge_parts_kernel");
+  }
   if (token_tc_ok(s)) {
     return s->dtype == HISA_BF16
                ? token_tc_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st)

@@ -81,6 +81,68 @@ __device__ void emit_at_least(KeyAt key_at, int n, uint32_t T, Emit emit, Select
   Grp::sync();
 }
 
+// Sum of one value per thread over a CTA of NT threads; every thread gets it.
+template <int NT>
+__device__ __forceinline__ uint32_t cta_sum(uint32_t v, uint32_t* red) {
+  v = __reduce_add_sync(0xffffffffu, v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  uint32_t t = 0;
+#pragma unroll
+  for (int i = 0; i < NT / 32; ++i) t += red[i];
+  __syncthreads();
+  return t;
+}
+
+template <int NT>
+__device__ __forceinline__ uint32_t cta_max(uint32_t v, uint32_t* red) {
+  v = __reduce_max_sync(0xffffffffu, v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  uint32_t t = 0;
+#pragma unroll
+  for (int i = 0; i < NT / 32; ++i) t = max(t, red[i]);
+  __syncthreads();
+  return t;
+}
+
+template <int NT>
+__device__ __forceinline__ uint32_t cta_min(uint32_t v, uint32_t* red) {
+  v = __reduce_min_sync(0xffffffffu, v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  uint32_t t = 0xFFFFFFFFu;
+#pragma unroll
+  for (int i = 0; i < NT / 32; ++i) t = min(t, red[i]);
+  __syncthreads();
+  return t;
+}
+
+// The r-th largest of the CTA's keys (KPT per thread, 0 = absent; r >= 1 and
+// at most the number of present keys): bit by bit from the highest bit where
+// the smallest and largest keys differ, keeping a bit when at least r keys
+// are >= the value with it set.
+template <int NT, int KPT>
+__device__ uint32_t cta_rth_largest(const uint32_t (&key)[KPT], uint32_t r, uint32_t* red) {
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+  for (int u = 0; u < KPT; ++u)
+    if (key[u] != 0u) { lo = min(lo, key[u]); hi = max(hi, key[u]); }
+  lo = cta_min<NT>(lo, red);
+  hi = cta_max<NT>(hi, red);
+  if (lo >= hi) return hi;
+  const int top = 31 - __clz(lo ^ hi);
+  uint32_t T = hi & ~((2u << top) - 1u);
+  for (int bit = top; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    uint32_t c = 0;
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) c += key[u] >= cand ? 1u : 0u;
+    if (cta_sum<NT>(c, red) >= r) T = cand;
+  }
+  return T;
+}
+
 // The bin holding the k-th place of sm.hist[0, nbins) counted from the top:
 // sets sm.digit, sm.above (elements in higher bins) and sm.at_digit (the
 // bin's count).  Each thread sums a run of bins, one block scan orders the
@@ -594,6 +656,82 @@ __device__ bool two_pass_topk_rows(const float* __restrict__ row, int n, uint32_
   }
   Grp::sync();
   return true;
+}
+
+// Top-k of the union of `parts` top-k lists per row (idx -1 = empty slot),
+// by (score desc, index asc): the refinement stage split over several CTAs
+// per query writes each part's own top-k, and since every element of the
+// query's top-k is in its part's top-k, the top-k of the union is exact.
+template <int KPT>
+__global__ void __launch_bounds__(256) merge_parts_kernel(const int32_t* __restrict__ part_idx,
+                                                          const float* __restrict__ part_score, int parts,
+                                                          int64_t rows, int k, int32_t* __restrict__ out_idx,
+                                                          float* __restrict__ out_score) {
+  __shared__ uint32_t red[8];
+  __shared__ uint32_t slot_ctr;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int m_all = parts * k;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const int32_t* pi = part_idx + r * m_all;
+    const float* ps = part_score + r * m_all;
+    uint32_t key[KPT], pos[KPT];
+    uint32_t valid = 0;
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) {
+      const int i = tid + u * 256;
+      const int32_t x = i < m_all ? pi[i] : -1;
+      pos[u] = x >= 0 ? static_cast<uint32_t>(x) : 0xFFFFFFFFu;
+      key[u] = x >= 0 ? max(float_key(ps[i]), 1u) : 0u;
+      valid += x >= 0 ? 1u : 0u;
+    }
+    valid = cta_sum<256>(valid, red);
+    int32_t* oi = out_idx + r * k;
+    float* os = out_score ? out_score + r * k : nullptr;
+    uint32_t T = 0u, P = 0xFFFFFFFFu;
+    if (valid > static_cast<uint32_t>(k)) {
+      T = cta_rth_largest<256, KPT>(key, static_cast<uint32_t>(k), red);
+      uint32_t gt = 0, eq = 0;
+#pragma unroll
+      for (int u = 0; u < KPT; ++u) {
+        gt += key[u] > T ? 1u : 0u;
+        eq += key[u] == T ? 1u : 0u;
+      }
+      gt = cta_sum<256>(gt, red);
+      eq = cta_sum<256>(eq, red);
+      const uint32_t need = static_cast<uint32_t>(k) - gt;
+      if (eq > need) {
+        P = 0u;
+        for (int bit = 30; bit >= 0; --bit) {
+          const uint32_t test = P | ((1u << bit) - 1u);
+          uint32_t cnt = 0;
+#pragma unroll
+          for (int u = 0; u < KPT; ++u) cnt += (key[u] == T && pos[u] <= test) ? 1u : 0u;
+          if (cta_sum<256>(cnt, red) < need) P |= 1u << bit;
+        }
+      }
+    }
+    if (tid == 0) slot_ctr = 0;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < KPT; ++u) {
+      const bool take = key[u] != 0u && (key[u] > T || (key[u] == T && pos[u] <= P));
+      const uint32_t ball = __ballot_sync(0xffffffffu, take);
+      uint32_t base = 0;
+      if (lane == 0 && ball) base = atomicAdd(&slot_ctr, static_cast<uint32_t>(__popc(ball)));
+      base = __shfl_sync(0xffffffffu, base, 0) + __popc(ball & ((1u << lane) - 1u));
+      if (take) {
+        oi[base] = static_cast<int32_t>(pos[u]);
+        if (os) os[base] = ps[tid + u * 256];
+      }
+    }
+    __syncthreads();
+    const uint32_t filled = min(valid, static_cast<uint32_t>(k));
+    for (int i = static_cast<int>(filled) + tid; i < k; i += 256) {
+      oi[i] = -1;
+      if (os) os[i] = -__int_as_float(0x7f800000);
+    }
+    __syncthreads();
+  }
 }
 
 // Flat DSA top-k over fp32 score rows: row r holds scores of keys 0..n_r-1.

@@ -55,12 +55,14 @@ struct TokenParams {
   const int32_t* block_idx;
   const float* q_scale;
   const float* k_scale;
-  int32_t* out_idx;
+  int32_t* out_idx;        // [rows * parts, top_k]
   float* out_score;
+  int parts;                // > 1: each query's retained blocks split over `parts` jobs, each writing its own top-k
 };
 
 struct alignas(16) TokJob {
   int64_t row;
+  int64_t orow;            // output row: row * parts + part
   int b, n, nblk, ntiles;
   float qsc;
   uint32_t kmin, kmax, nvalid;     // filled by the scorers for the selector
@@ -68,9 +70,9 @@ struct alignas(16) TokJob {
   int blk[kTokMaxBlocks];
 };
 
-__device__ __forceinline__ int64_t tok_job_row(const TokenParams& p, int64_t j) {
-  // largest prefixes first
-  return p.rows - 1 - (static_cast<int64_t>(blockIdx.x) + j * gridDim.x);
+__device__ __forceinline__ int64_t tok_job_id(const TokenParams& p, int64_t j) {
+  // largest prefixes first; job id = row * parts + part
+  return p.rows * p.parts - 1 - (static_cast<int64_t>(blockIdx.x) + j * gridDim.x);
 }
 
 template <int DT, int H>
@@ -138,7 +140,8 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int64_t njobs = p.rows > blockIdx.x ? (p.rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int64_t total_jobs = p.rows * p.parts;
+  const int64_t njobs = total_jobs > blockIdx.x ? (total_jobs - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ job set-up
@@ -149,7 +152,9 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
       if (lane == 0) okl = mbar_wait(job_empty + slot, static_cast<uint32_t>(((j / kTokJobs) & 1) ^ 1), abort_flag);
       if (!(ok = __shfl_sync(0xffffffffu, okl, 0) != 0)) break;
       TokJob& J = jobs[slot];
-      const int64_t row = tok_job_row(p, j);
+      const int64_t jid = tok_job_id(p, j);
+      const int64_t row = jid / p.parts;
+      const int part = static_cast<int>(jid % p.parts);
       const int b = static_cast<int>(row / p.Q);
       // every global read of the job at once: visibility, block list, weights
       const int n_raw = __ldg(p.n_visible + row);
@@ -186,7 +191,11 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += o;
       }
-      const int cnt = __shfl_sync(0xffffffffu, incl, 31);
+      const int cnt_all = __shfl_sync(0xffffffffu, incl, 31);
+      // this job's share of the blocks (all of them unless the query is split)
+      const int lo = static_cast<int>((static_cast<int64_t>(cnt_all) * part) / p.parts);
+      const int hi = static_cast<int>((static_cast<int64_t>(cnt_all) * (part + 1)) / p.parts);
+      const int cnt = hi - lo;
       int pos = incl - local;
       for (int i = 0; i < wpl; ++i) {
         const int wi = lane * wpl + i;
@@ -195,13 +204,15 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
         while (bits) {
           const int bit = __ffs(bits) - 1;
           bits &= bits - 1;
-          J.blk[pos++] = (wi << 5) + bit;
+          if (pos >= lo && pos < hi) J.blk[pos - lo] = (wi << 5) + bit;
+          ++pos;
         }
       }
       J.w[lane] = w0;
       J.w[lane + 32] = w1;
       if (lane == 0) {
         J.row = row;
+        J.orow = jid;
         J.b = b;
         J.n = n;
         J.nblk = cnt;
@@ -401,8 +412,8 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
       const TokJob& J = jobs[slot];
       const uint32_t* cj = cand + cb * p.max_cand;
       const int ncand = J.ntiles * kTokTileM;
-      int32_t* oi = p.out_idx + J.row * p.top_k;
-      float* os = p.out_score ? p.out_score + J.row * p.top_k : nullptr;
+      int32_t* oi = p.out_idx + J.orow * p.top_k;
+      float* os = p.out_score ? p.out_score + J.orow * p.top_k : nullptr;
       const int bshift = __ffs(p.B) - 1;
       // indices are staged in shared memory (the selection's histogram space,
       // free once offsets are known) and written out coalesced; with scores

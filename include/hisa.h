@@ -183,6 +183,12 @@ HISA_API hisa_status hisa_block_score_topm(const void* q, const float* q_scale,
  *   topk_idx   [batch, Q, top_k] int32 (output)
  *   topk_score [batch, Q, top_k] fp32 (output, may be NULL; -inf padding)
  * Requires top_m * block_size <= 16384.
+ * Workspace: optional.  hisa_workspace_size(HISA_OP_TOKEN_SCORE_TOPK) is
+ * nonzero for shapes with few queries (at most half the SM count, as in a
+ * decode step); given at least that much (16-byte aligned), each query's
+ * blocks are split over several CTAs and their top-k lists merged exactly,
+ * so more SMs gather keys.  NULL (or less) runs one CTA per query.  The
+ * result is the same either way.
  */
 HISA_API hisa_status hisa_token_score_topk(const void* q, const float* q_scale,
                                   const float* w, const void* k,

@@ -47,6 +47,10 @@ def test_workspace_sizes(L):
     assert hb.workspace_size(hb.OP_FLAT, s) == 32768 * (32768 * 4 + 8)
     assert hb.workspace_size(hb.OP_BLOCK, s) == 32768 * 256 * 4
     assert hb.workspace_size(hb.OP_TOKEN, s) == 0
+    # few queries (a decode step): room for the per-part top-k lists of split queries
+    dec = _shape(batch=64, num_queries=1, num_keys=131072, top_m=64)
+    parts = hb.workspace_size(hb.OP_TOKEN, dec) // (64 * 2048 * 8)
+    assert parts >= 2 and hb.workspace_size(hb.OP_TOKEN, dec) == 64 * parts * 2048 * 8
     s = _shape(num_keys=1001, num_queries=3, batch=2, block_size=64)
     assert hb.workspace_size(hb.OP_FLAT, s) == 6 * (1004 * 4 + 8)    # rows padded to 16 bytes, + row range
     assert hb.workspace_size(hb.OP_BLOCK, s) == 6 * 16 * 4           # ceil(1001/64)=16

@@ -38,6 +38,9 @@ SMALL = {
                    needles=4, name="f32_h4"),
     "batch_tail": dict(batch=3, num_keys=2000, num_queries=40, first_query_pos=1960, heads=64, head_dim=128,
                        block_size=128, top_m=4, top_k=256, dtype="bf16", needles=8, name="batch_tail"),
+    # few queries: the refinement stage splits each query's blocks over several CTAs and merges
+    "few_rows_split": dict(batch=4, num_keys=2000, num_queries=2, first_query_pos=1998, heads=64, head_dim=128,
+                           block_size=64, top_m=8, top_k=100, dtype="bf16", needles=4, name="few_rows_split"),
     "compressed": dict(num_keys=600, compress_ratio=4, num_queries=300, first_query_pos=2100, heads=64,
                        head_dim=128, block_size=64, top_m=4, top_k=96, dtype="bf16", needles=0,
                        name="compressed"),
