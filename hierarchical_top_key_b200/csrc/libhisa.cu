@@ -296,10 +296,15 @@ constexpr size_t kSmemBudget = 232448;   // 227 KB opt-in dynamic shared memory 
 
 bool token_tc_ok(const hisa_shape* s) {
   const int rb = s->head_dim * elem_bytes(s->dtype);
-  return (s->dtype == HISA_BF16 || s->dtype == HISA_E4M3) && (rb == 128 || rb == 256) &&
-         (s->heads == 16 || s->heads == 32 || s->heads == 64) &&
-         (s->block_size == 16 || s->block_size == 32 || s->block_size == 64 || s->block_size == 128) &&
-         s->top_m <= kTokMaxBlocks && num_blocks(s) <= 32 * kTokMaxBitmapWords;
+  if (!((s->dtype == HISA_BF16 || s->dtype == HISA_E4M3) && (rb == 128 || rb == 256) &&
+        (s->heads == 16 || s->heads == 32 || s->heads == 64) &&
+        (s->block_size == 16 || s->block_size == 32 || s->block_size == 64 || s->block_size == 128) &&
+        s->top_m <= kTokMaxBlocks && num_blocks(s) <= 32 * kTokMaxBitmapWords))
+    return false;
+  // the candidate buffers and two key stages must fit in shared memory; larger
+  // m * B go to the CUDA-core kernel
+  const int64_t max_cand = ceil_div(static_cast<int64_t>(s->top_m) * s->block_size, kTokTileM) * kTokTileM;
+  return token_smem_bytes(rb, s->heads, 2, static_cast<int>(max_cand)) <= kSmemBudget;
 }
 
 template <int DT, int H>
