@@ -250,19 +250,15 @@ __global__ void __launch_bounds__(kDenseThreads, 1) dense_score_tc_kernel(
         const int qb = un % p.q_bufs;
         if (!(ok = mbar_wait(q_full + qb, (un / p.q_bufs) & 1, abort_flag))) break;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(q_buf + qb * q_bytes);
+        const uint64_t q_desc = desc_k_sw128(smem_u32(q_buf + qb * q_bytes));
         for (int i = 0; i < U.ntiles; ++i) {
           if (!(ok = mbar_wait(acc_empty + ab, aph ^ 1, abort_flag))) break;
           if (!(ok = mbar_wait(k_full + st, kph, abort_flag))) break;
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(k_buf + st * k_bytes);
+          const uint64_t k_desc = desc_k_sw128(smem_u32(k_buf + st * k_bytes));
           const uint32_t d_tmem = tmem_base + ab * kDenseN;
-          for (int ks = 0; ks < ksteps; ++ks) {
-            const int pn = ks >> 2, off = (ks & 3) * 32;
-            const uint64_t a = desc_k_sw128(k_addr + pn * (kDenseTileM * 128) + off);
-            const uint64_t b = desc_k_sw128(q_addr + pn * (kDenseN * 128) + off);
-            mma<DT>(d_tmem, a, b, idesc, ks > 0 ? 1u : 0u);
-          }
+          if (ksteps == 8) mma_tile_sw128<DT, 8, kDenseTileM, kDenseN>(d_tmem, k_desc, q_desc, idesc);
+          else mma_tile_sw128<DT, 4, kDenseTileM, kDenseN>(d_tmem, k_desc, q_desc, idesc);
           mma_commit(k_empty + st);
           mma_commit(acc_full + ab);
           if (++st == p.stages) { st = 0; kph ^= 1; }

@@ -189,6 +189,22 @@ __device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b
   }
 }
 
+// The KS MMAs over K = KS * 32 bytes of one tile: A is ROWS_A rows and B is
+// ROWS_B rows, both K-major in 128-byte-swizzled panels of 64 bf16 / 128 e4m3
+// columns (a panel holds ROWS * 128 bytes).  A single issuing thread is bound
+// by the latency between its MMA instructions, so the descriptors are the
+// tile's base descriptors plus compile-time offsets: the start-address field
+// holds address / 16 and cannot carry, shared addresses being below 256 KB.
+template <int DT, int KS, int ROWS_A, int ROWS_B>
+__device__ __forceinline__ void mma_tile_sw128(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const uint64_t da = static_cast<uint64_t>((ks >> 2) * (ROWS_A * 128 / 16) + (ks & 3) * 2);
+    const uint64_t db = static_cast<uint64_t>((ks >> 2) * (ROWS_B * 128 / 16) + (ks & 3) * 2);
+    mma<DT>(d_tmem, a_desc + da, b_desc + db, idesc, ks > 0 ? 1u : 0u);
+  }
+}
+
 // Arrive once on `bar` when all previously issued tcgen05 operations of this
 // thread have completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {

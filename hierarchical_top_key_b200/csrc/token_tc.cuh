@@ -290,20 +290,17 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
         const int qb = static_cast<int>(j & 1);
         if (!(ok = mbar_wait(q_full + qb, static_cast<uint32_t>((j >> 1) & 1), abort_flag))) break;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(q_buf + qb * q_bytes);
+        const uint64_t q_desc = desc_k_sw128(smem_u32(q_buf + qb * q_bytes));
         for (int i = 0; i < ntiles; ++i) {
           if (g == me) {
             if (!(ok = mbar_wait(acc_empty + ab, aph ^ 1, abort_flag))) break;
             if (!(ok = mbar_wait(k_full + me * p.stages + st, (fph >> st) & 1u, abort_flag))) break;
             fph ^= 1u << st;
             tc_fence_after();
-            const uint32_t k_addr = smem_u32(k_buf + st * k_bytes);
+            const uint64_t k_desc = desc_k_sw128(smem_u32(k_buf + st * k_bytes));
             const uint32_t d_tmem = tmem_base + ab * H;
-            for (int ks = 0; ks < ksteps; ++ks) {
-              const int pn = ks >> 2, off = (ks & 3) * 32;
-              mma<DT>(d_tmem, desc_k_sw128(k_addr + pn * (kTokTileM * 128) + off),
-                      desc_k_sw128(q_addr + pn * (H * 128) + off), idesc, ks > 0 ? 1u : 0u);
-            }
+            if (ksteps == 8) mma_tile_sw128<DT, 8, kTokTileM, H>(d_tmem, k_desc, q_desc, idesc);
+            else mma_tile_sw128<DT, 4, kTokTileM, H>(d_tmem, k_desc, q_desc, idesc);
             mma_commit(k_empty + st);
             mma_commit(acc_full + ab);
           }
