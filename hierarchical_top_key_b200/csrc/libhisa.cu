@@ -322,8 +322,11 @@ hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc
   p.w = w; p.n_visible = nvis; p.block_idx = bidx; p.q_scale = qsc; p.k_scale = ksc; p.out_idx = oi; p.out_score = os;
   if (token_smem_bytes(rb, H, 2, p.max_cand) > kSmemBudget)
     return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size too large for the on-chip candidate buffers");
+  // key stages: as many as fit, up to 96 KB of tiles in flight (three bf16
+  // tiles of d = 128; a fourth was 3 % slower at 32K keys, measured)
+  const int max_stages = std::max(3, static_cast<int>(98304 / (kTokTileM * rb)));
   p.stages = 2;
-  while (p.stages < 6 && token_smem_bytes(rb, H, p.stages + 1, p.max_cand) <= kSmemBudget) ++p.stages;
+  while (p.stages < max_stages && token_smem_bytes(rb, H, p.stages + 1, p.max_cand) <= kSmemBudget) ++p.stages;
   const size_t smem = token_smem_bytes(rb, H, p.stages, p.max_cand);
   CUtensorMap qm, km;
   hisa_status e = tensor_map_2d(&qm, q, s->dtype, static_cast<uint64_t>(p.rows) * H, s->head_dim, H);
