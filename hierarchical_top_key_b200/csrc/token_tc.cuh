@@ -348,8 +348,8 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
           if (DT == DT_E4M3 && valid) ksc = __ldg(p.k_scale + static_cast<int64_t>(J.b) * p.L + s);
           float acc = 0.f;
           if (H >= 32) {
-            // all TMEM loads of the row first, one wait, then four independent
-            // accumulation chains over float4 weight reads
+            // 32 columns per TMEM load (32 registers live, not 64), four
+            // independent accumulation chains over float4 weight reads
             float a4[4] = {0.f, 0.f, 0.f, 0.f};
             const float4* w4 = reinterpret_cast<const float4*>(J.w);
 #pragma unroll
