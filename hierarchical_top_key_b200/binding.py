@@ -44,6 +44,8 @@ _P = ctypes.c_void_p
 _SIGS = {
     "hisa_pool_blocks": [_P, _P, _P, _P, ctypes.POINTER(Shape), _P],
     "hisa_pool_blocks_range": [_P, _P, _P, _P, ctypes.POINTER(Shape), ctypes.c_int32, ctypes.c_int32, _P],
+    "hisa_pool_blocks_paged": [_P, _P, _P, ctypes.c_int32, _P, _P, ctypes.POINTER(Shape), ctypes.c_int32,
+                               ctypes.c_int32, _P],
     "hisa_compress_keys": [_P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                            ctypes.c_int32, _P],
     "hisa_quantize_e4m3": [_P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _P, _P, _P],
@@ -53,6 +55,8 @@ _SIGS = {
     "hisa_block_score_topm_static": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P],
     "hisa_token_score_topk": [_P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t,
                               _P],
+    "hisa_token_score_topk_paged": [_P, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.POINTER(Shape), _P, _P,
+                                    _P, ctypes.c_size_t, _P],
     "dsa_flat_indexer_topk": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t, _P],
     "dsa_flat_indexer_topk_sampled": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t, _P],
     "hisa_workspace_size": [ctypes.c_int32, ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)],
@@ -251,6 +255,62 @@ def hisa_token_score_topk(q, w, k, n_visible, block_idx, *, block_size: int, top
     _check(load().hisa_token_score_topk(q.data_ptr(), _ptr(q_scale), w.data_ptr(), k.data_ptr(), _ptr(k_scale),
                                         n_visible.data_ptr(), block_idx.data_ptr(), ctypes.byref(shape),
                                         idx.data_ptr(), _ptr(sc), _ptr(ws), need, _stream()), "hisa_token_score_topk")
+    return idx, sc
+
+
+def _check_pages(k_pages, page_table, block_size: int, batch: int, num_keys: int):
+    _need(k_pages, "k_pages", 3)
+    if k_pages.shape[1] != block_size:
+        raise ValueError(f"k_pages {tuple(k_pages.shape)} must be [num_pages, block_size={block_size}, d]")
+    _need(page_table, "page_table", 2)
+    nb = -(-num_keys // block_size)
+    if page_table.dtype != torch.int32 or tuple(page_table.shape) != (batch, nb):
+        raise ValueError(f"page_table must be int32 [batch, ceil(num_keys/B)] = {(batch, nb)}, "
+                         f"got {page_table.dtype} {tuple(page_table.shape)}")
+
+
+def hisa_pool_blocks_paged(k_pages, page_table, *, num_keys: int, first_block: int, block_count: int,
+                           kpool: torch.Tensor, k_page_scale: Optional[torch.Tensor] = None,
+                           kpool_scale: Optional[torch.Tensor] = None) -> None:
+    """hisa_pool_blocks_range over paged keys: k_pages [num_pages, B, d], block j of
+    sequence b in page page_table[b, j]; writes kpool [batch, nb, d] rows in place."""
+    B = k_pages.shape[1] if k_pages.dim() == 3 else 0
+    b = page_table.shape[0] if page_table.dim() == 2 else 0
+    _check_pages(k_pages, page_table, B, b, num_keys)
+    d = k_pages.shape[2]
+    nb = -(-num_keys // B)
+    if tuple(kpool.shape) != (b, nb, d) or kpool.dtype != k_pages.dtype or not kpool.is_contiguous():
+        raise ValueError("kpool must be a contiguous [batch, ceil(num_keys/B), d] tensor of the keys' dtype")
+    if (k_page_scale is None) != (kpool_scale is None):
+        raise ValueError("k_page_scale and kpool_scale go together (E4M3 keys)")
+    shape = Shape(b, num_keys, 1, 1, d, B, 1, 1, dtype_code(k_pages))
+    _check(load().hisa_pool_blocks_paged(k_pages.data_ptr(), _ptr(k_page_scale), page_table.data_ptr(),
+                                         k_pages.shape[0], kpool.data_ptr(), _ptr(kpool_scale), ctypes.byref(shape),
+                                         first_block, block_count, _stream()), "hisa_pool_blocks_paged")
+
+
+def hisa_token_score_topk_paged(q, w, k_pages, page_table, n_visible, block_idx, *, num_keys: int, top_k: int,
+                                q_scale=None, k_page_scale=None, want_scores: bool = False):
+    """Refinement stage over paged keys (layout as hisa_pool_blocks_paged):
+    (topk_idx [batch, Q, top_k] int32, scores or None), equal to
+    hisa_token_score_topk on the same keys stored contiguously."""
+    _need(q, "q", 4)
+    _need(block_idx, "block_idx", 3)
+    b, Q, H, d = q.shape
+    B = k_pages.shape[1] if k_pages.dim() == 3 else 0
+    _check_pages(k_pages, page_table, B, b, num_keys)
+    if k_pages.shape[2] != d or dtype_code(k_pages) != dtype_code(q):
+        raise ValueError("k_pages must match q in head_dim and dtype")
+    shape = Shape(b, num_keys, Q, H, d, B, block_idx.shape[-1], top_k, dtype_code(q))
+    idx = torch.empty((b, Q, top_k), dtype=torch.int32, device=q.device)
+    sc = torch.empty((b, Q, top_k), dtype=torch.float32, device=q.device) if want_scores else None
+    need = workspace_size(OP_TOKEN, shape)
+    ws = _workspace(need, q.device) if need > 0 else None
+    _check(load().hisa_token_score_topk_paged(q.data_ptr(), _ptr(q_scale), w.data_ptr(), k_pages.data_ptr(),
+                                              _ptr(k_page_scale), page_table.data_ptr(), k_pages.shape[0],
+                                              n_visible.data_ptr(), block_idx.data_ptr(), ctypes.byref(shape),
+                                              idx.data_ptr(), _ptr(sc), _ptr(ws), need, _stream()),
+           "hisa_token_score_topk_paged")
     return idx, sc
 
 

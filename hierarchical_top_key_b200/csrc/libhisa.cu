@@ -2,6 +2,7 @@
 // planning and stream-ordered kernel launches.  Every step of the indexers
 // runs in the kernels included below; this file only checks arguments and
 // launches them.
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <cstdarg>
@@ -307,10 +308,17 @@ bool token_tc_ok(const hisa_shape* s) {
   return token_smem_bytes(rb, s->heads, 2, static_cast<int>(max_cand)) <= kSmemBudget;
 }
 
+// Paged keys: block j of sequence b is page table[b * nb + j] of a
+// [count, block_size, head_dim] key array (table NULL: keys contiguous).
+struct KeyPages {
+  const int32_t* table = nullptr;
+  int32_t count = 0;
+};
+
 template <int DT, int H>
 hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* k,
                             const float* ksc, const int32_t* nvis, const int32_t* bidx, int32_t* oi, float* os,
-                            cudaStream_t st, int parts = 1) {
+                            cudaStream_t st, int parts = 1, KeyPages pg = {}) {
   const int rb = s->head_dim * Elem<DT>::bytes;
   TokenParams p{};
   p.rows = rows_of(s);
@@ -319,6 +327,7 @@ hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc
   p.nb = static_cast<int>(num_blocks(s));
   p.max_cand = static_cast<int>(ceil_div(static_cast<int64_t>(s->top_m) * s->block_size, kTokTileM) * kTokTileM);
   p.parts = parts;
+  p.pages = pg.table; p.num_pages = pg.count;
   p.w = w; p.n_visible = nvis; p.block_idx = bidx; p.q_scale = qsc; p.k_scale = ksc; p.out_idx = oi; p.out_score = os;
   if (token_smem_bytes(rb, H, 2, p.max_cand) > kSmemBudget)
     return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size too large for the on-chip candidate buffers");
@@ -331,7 +340,9 @@ hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc
   CUtensorMap qm, km;
   hisa_status e = tensor_map_2d(&qm, q, s->dtype, static_cast<uint64_t>(p.rows) * H, s->head_dim, H);
   if (e != HISA_OK) return e;
-  e = tensor_map_2d(&km, k, s->dtype, static_cast<uint64_t>(s->batch) * s->num_keys, s->head_dim, s->block_size);
+  const uint64_t key_rows = pg.table ? static_cast<uint64_t>(pg.count) * s->block_size
+                                    : static_cast<uint64_t>(s->batch) * s->num_keys;
+  e = tensor_map_2d(&km, k, s->dtype, key_rows, s->head_dim, s->block_size);
   if (e != HISA_OK) return e;
   auto kern = token_tc_kernel<DT, H>;
   e = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
@@ -345,11 +356,11 @@ hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc
 template <int DT>
 hisa_status token_tc_h(const hisa_shape* s, const void* q, const float* qsc, const float* w, const void* k,
                        const float* ksc, const int32_t* nvis, const int32_t* bidx, int32_t* oi, float* os,
-                       cudaStream_t st, int parts = 1) {
+                       cudaStream_t st, int parts = 1, KeyPages pg = {}) {
   switch (s->heads) {
-    case 16: return launch_token_tc<DT, 16>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st, parts);
-    case 32: return launch_token_tc<DT, 32>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st, parts);
-    default: return launch_token_tc<DT, 64>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st, parts);
+    case 16: return launch_token_tc<DT, 16>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st, parts, pg);
+    case 32: return launch_token_tc<DT, 32>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st, parts, pg);
+    default: return launch_token_tc<DT, 64>(s, q, qsc, w, k, ksc, nvis, bidx, oi, os, st, parts, pg);
   }
 }
 
@@ -487,6 +498,50 @@ hisa_status check_indexer_ptrs(const hisa_shape* s, const void* q, const float* 
     return fail(HISA_ERR_INVALID_ARG, "E4M3 inputs need q_scale and k_scale");
   return HISA_OK;
 }
+
+// The refinement stage after argument checks: split queries with the merge,
+// the tensor-core kernel, or (contiguous keys only) the CUDA-core kernel.
+hisa_status token_score_topk_checked(const void* q, const float* q_scale, const float* w, const void* k,
+                                     const float* k_scale, const int32_t* n_visible, const int32_t* block_idx,
+                                     const hisa_shape* s, int32_t* topk_idx, float* topk_score, void* workspace,
+                                     size_t ws_bytes, hisa_stream stream, KeyPages pg) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int parts = token_parts(s);
+  if (parts > 1 && workspace && aligned16(workspace) && ws_bytes >= token_split_bytes(s, parts)) {
+    // split queries: every part's top-k with scores into the workspace, then the exact merge
+    const int64_t rows = rows_of(s);
+    int32_t* pidx = static_cast<int32_t*>(workspace);
+    float* psc = reinterpret_cast<float*>(pidx + rows * parts * s->top_k);
+    hisa_status e = s->dtype == HISA_BF16
+            ? token_tc_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, pidx, psc, st, parts, pg)
+            : token_tc_h<DT_E4M3>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, pidx, psc, st, parts, pg);
+    if (e != HISA_OK) return e;
+    const int items = parts * s->top_k;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(rows, num_sms() * 4));
+    if (items <= 256 * 8)
+      merge_parts_kernel<8><<<grid, 256, 0, st>>>(pidx, psc, parts, rows, s->top_k, topk_idx, topk_score);
+    else if (items <= 256 * 16)
+      merge_parts_kernel<16><<<grid, 256, 0, st>>>(pidx, psc, parts, rows, s->top_k, topk_idx, topk_score);
+    else
+      merge_parts_kernel<32><<<grid, 256, 0, st>>>(pidx, psc, parts, rows, s->top_k, topk_idx, topk_score);
+    return launch_check("merge_parts_kernel");
+  }
+  if (token_tc_ok(s)) {
+    return s->dtype == HISA_BF16
+               ? token_tc_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st, 1, pg)
+               : token_tc_h<DT_E4M3>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st, 1, pg);
+  }
+  if (pg.table)
+    return fail(HISA_ERR_UNSUPPORTED,
+                "paged keys need a tensor-core shape: bf16 or E4M3, head_dim * bytes 128 or 256, H 16/32/64, "
+                "B 16..128, top_m * B within the on-chip candidate buffers");
+  switch (s->dtype) {
+    case HISA_F32: return token_simt_h<DT_F32>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
+    case HISA_BF16: return token_simt_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
+    default: return token_simt_h<DT_E4M3>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
+  }
+}
+
 
 }  // namespace
 
@@ -720,37 +775,73 @@ hisa_status hisa_token_score_topk(const void* q, const float* q_scale, const flo
   if (s->top_m > kMaxTopM) return fail(HISA_ERR_UNSUPPORTED, "top_m must be <= %d", kMaxTopM);
   if (static_cast<int64_t>(s->top_m) * s->block_size > kMaxCandidates)
     return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size must be <= %d", kMaxCandidates);
+  return token_score_topk_checked(q, q_scale, w, k, k_scale, n_visible, block_idx, s, topk_idx, topk_score,
+                                  workspace, ws_bytes, stream, KeyPages{});
+}
+
+hisa_status hisa_token_score_topk_paged(const void* q, const float* q_scale, const float* w, const void* k_pages,
+                                        const float* k_page_scale, const int32_t* page_table, int32_t num_pages,
+                                        const int32_t* n_visible, const int32_t* block_idx, const hisa_shape* s,
+                                        int32_t* topk_idx, float* topk_score, void* workspace, size_t ws_bytes,
+                                        hisa_stream stream) {
+  hisa_status e = check_shape(s, true);
+  if (e != HISA_OK) return e;
+  e = check_indexer_ptrs(s, q, q_scale, w, k_pages, k_page_scale, n_visible);
+  if (e != HISA_OK) return e;
+  if (!block_idx || !topk_idx) return fail(HISA_ERR_INVALID_ARG, "block_idx and topk_idx must be non-NULL");
+  if (!page_table || !aligned4(page_table)) return fail(HISA_ERR_INVALID_ARG, "page_table must be non-NULL and 4-byte aligned");
+  if (num_pages < 1) return fail(HISA_ERR_INVALID_ARG, "num_pages must be >= 1");
+  if (static_cast<int64_t>(num_pages) * s->block_size > INT32_MAX)
+    return fail(HISA_ERR_UNSUPPORTED, "num_pages * block_size must fit in int32");
+  if (s->top_m > kMaxTopM) return fail(HISA_ERR_UNSUPPORTED, "top_m must be <= %d", kMaxTopM);
+  if (static_cast<int64_t>(s->top_m) * s->block_size > kMaxCandidates)
+    return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size must be <= %d", kMaxCandidates);
+  return token_score_topk_checked(q, q_scale, w, k_pages, k_page_scale, n_visible, block_idx, s, topk_idx,
+                                  topk_score, workspace, ws_bytes, stream, KeyPages{page_table, num_pages});
+}
+
+hisa_status hisa_pool_blocks_paged(const void* k_pages, const float* k_page_scale, const int32_t* page_table,
+                                   int32_t num_pages, void* kpool, float* kpool_scale, const hisa_shape* s,
+                                   int32_t first_block, int32_t block_count, hisa_stream stream) {
+  if (!s) return fail(HISA_ERR_INVALID_ARG, "shape is NULL");
+  if (first_block < 0 || block_count < 0) return fail(HISA_ERR_INVALID_ARG, "first_block and block_count must be >= 0");
+  if (s->batch < 1 || s->num_keys < 1 || s->block_size < 1)
+    return fail(HISA_ERR_INVALID_ARG, "batch, num_keys, block_size must be >= 1");
+  if (s->head_dim != 64 && s->head_dim != 128) return fail(HISA_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (!k_pages || !kpool || !aligned16(k_pages) || !aligned16(kpool))
+    return fail(HISA_ERR_INVALID_ARG, "k_pages and kpool must be non-NULL and 16-byte aligned");
+  if (!page_table || !aligned4(page_table)) return fail(HISA_ERR_INVALID_ARG, "page_table must be non-NULL and 4-byte aligned");
+  if (num_pages < 1) return fail(HISA_ERR_INVALID_ARG, "num_pages must be >= 1");
+  if (s->dtype == HISA_E4M3 && (!k_page_scale || !kpool_scale))
+    return fail(HISA_ERR_INVALID_ARG, "E4M3 pooling needs k_page_scale and kpool_scale");
+  const int nb = static_cast<int>(num_blocks(s));
+  const int first = std::min(first_block, nb);
+  const int count = std::min(block_count, nb - first);
+  if (count == 0) return HISA_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int parts = token_parts(s);
-  if (parts > 1 && workspace && aligned16(workspace) && ws_bytes >= token_split_bytes(s, parts)) {
-    // split queries: every part's top-k with scores into the workspace, then the exact merge
-    const int64_t rows = rows_of(s);
-    int32_t* pidx = static_cast<int32_t*>(workspace);
-    float* psc = reinterpret_cast<float*>(pidx + rows * parts * s->top_k);
-    e = s->dtype == HISA_BF16
-            ? token_tc_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, pidx, psc, st, parts)
-            : token_tc_h<DT_E4M3>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, pidx, psc, st, parts);
-    if (e != HISA_OK) return e;
-    const int items = parts * s->top_k;
-    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(rows, num_sms() * 4));
-    if (items <= 256 * 8)
-      merge_parts_kernel<8><<<grid, 256, 0, st>>>(pidx, psc, parts, rows, s->top_k, topk_idx, topk_score);
-    else if (items <= 256 * 16)
-      merge_parts_kernel<16><<<grid, 256, 0, st>>>(pidx, psc, parts, rows, s->top_k, topk_idx, topk_score);
-    else
-      merge_parts_kernel<32><<<grid, 256, 0, st>>>(pidx, psc, parts, rows, s->top_k, topk_idx, topk_score);
-    return launch_check("merge_parts_kernel");
-  }
-  if (token_tc_ok(s)) {
-    return s->dtype == HISA_BF16
-               ? token_tc_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st)
-               : token_tc_h<DT_E4M3>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
-  }
+  const int64_t threads_total = static_cast<int64_t>(s->batch) * count * (s->head_dim * elem_bytes(s->dtype) / 16);
+  const int grid = static_cast<int>(std::min<int64_t>(ceil_div(threads_total, 256), 148 * 64));
+  const uint8_t* in = static_cast<const uint8_t*>(k_pages);
+  uint8_t* out = static_cast<uint8_t*>(kpool);
   switch (s->dtype) {
-    case HISA_F32: return token_simt_h<DT_F32>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
-    case HISA_BF16: return token_simt_h<DT_BF16>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
-    default: return token_simt_h<DT_E4M3>(s, q, q_scale, w, k, k_scale, n_visible, block_idx, topk_idx, topk_score, st);
+    case HISA_F32:
+      paged_block_mean_kernel<DT_F32><<<grid, 256, 0, st>>>(in, nullptr, page_table, num_pages, out, nullptr,
+                                                            s->batch, s->num_keys, nb, s->head_dim, s->block_size,
+                                                            first, count);
+      break;
+    case HISA_BF16:
+      paged_block_mean_kernel<DT_BF16><<<grid, 256, 0, st>>>(in, nullptr, page_table, num_pages, out, nullptr,
+                                                             s->batch, s->num_keys, nb, s->head_dim, s->block_size,
+                                                             first, count);
+      break;
+    case HISA_E4M3:
+      paged_block_mean_kernel<DT_E4M3><<<grid, 256, 0, st>>>(in, k_page_scale, page_table, num_pages, out,
+                                                             kpool_scale, s->batch, s->num_keys, nb, s->head_dim,
+                                                             s->block_size, first, count);
+      break;
+    default: return fail(HISA_ERR_INVALID_ARG, "unknown dtype %d", s->dtype);
   }
+  return launch_check("paged_block_mean_kernel");
 }
 
 hisa_status hisa_block_refine_topm(const void* q, const float* q_scale, const float* w, const void* kpool,

@@ -104,6 +104,63 @@ __global__ void __launch_bounds__(256) segment_mean_kernel(
   }
 }
 
+// Block means over paged keys: block o of sequence b is page pages[b * n_out + o]
+// of `in` ([num_pages, G, d], scales [num_pages, G]); its first
+// min(G, n_in - o * G) rows are keys.  Same arithmetic and rounding as
+// segment_mean_kernel.  A page entry outside [0, num_pages) leaves the output
+// row untouched and records HISA_ERR_INVALID_ARG in the status word.
+template <int DT>
+__global__ void __launch_bounds__(256) paged_block_mean_kernel(
+    const uint8_t* __restrict__ in, const float* __restrict__ in_scale, const int32_t* __restrict__ pages,
+    int num_pages, uint8_t* __restrict__ out, float* __restrict__ out_scale,
+    int batch, int n_in, int n_out, int d, int G, int o_first, int o_count) {
+  constexpr int VE = Vec16<DT>::n;
+  const int vecs = d / VE;
+  const int64_t row_bytes = static_cast<int64_t>(d) * Elem<DT>::bytes;
+  const int64_t total = static_cast<int64_t>(batch) * o_count * vecs;
+  for (int64_t g = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; g < ceil_div(total, 32) * 32;
+       g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const bool live = g < total;
+    const int64_t lrow = live ? g / vecs : 0;
+    const int v = static_cast<int>(g % vecs);
+    const int b = static_cast<int>(lrow / o_count);
+    const int o = o_first + static_cast<int>(lrow % o_count);
+    const int64_t orow = static_cast<int64_t>(b) * n_out + o;
+    const int nrows = max(0, min(G, n_in - o * G));
+    bool ok = live;
+    int pg = 0;
+    if (live) {
+      pg = __ldg(pages + orow);
+      if (pg < 0 || pg >= num_pages) {
+        ok = false;
+        if (v == 0) record_status(HISA_ERR_INVALID_ARG);
+      }
+    }
+    double acc[VE];
+#pragma unroll
+    for (int e = 0; e < VE; ++e) acc[e] = 0.0;
+    if (ok) {
+      const uint8_t* base = in + static_cast<int64_t>(pg) * G * row_bytes + v * 16;
+#pragma unroll 4
+      for (int r = 0; r < nrows; ++r) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(base + r * row_bytes));
+        float f[VE];
+        Vec16<DT>::unpack(raw, f);
+        if (DT == DT_E4M3) {
+          const double sc = static_cast<double>(__ldg(in_scale + static_cast<int64_t>(pg) * G + r));
+#pragma unroll
+          for (int e = 0; e < VE; ++e) acc[e] += static_cast<double>(f[e]) * sc;
+        } else {
+#pragma unroll
+          for (int e = 0; e < VE; ++e) acc[e] += static_cast<double>(f[e]);
+        }
+      }
+    }
+    write_mean<DT>(acc, static_cast<double>(max(nrows, 1)), out + orow * row_bytes + v * 16,
+                   out_scale ? out_scale + orow : nullptr, v, vecs, ok);
+  }
+}
+
 // The same means with one CTA per output row, for long groups (few output
 // rows of many keys): the group's rows are split over `parts` threads per
 // column vector, and the fp64 partial sums are added in a fixed order (the

@@ -58,6 +58,8 @@ struct TokenParams {
   int32_t* out_idx;        // [rows * parts, top_k]
   float* out_score;
   int parts;                // > 1: each query's retained blocks split over `parts` jobs, each writing its own top-k
+  const int32_t* pages;     // non-NULL: block j of sequence b is page pages[b * nb + j] of the keys ([num_pages, B, d])
+  int num_pages;
 };
 
 struct alignas(16) TokJob {
@@ -68,6 +70,7 @@ struct alignas(16) TokJob {
   uint32_t kmin, kmax, nvalid;     // filled by the scorers for the selector
   alignas(16) float w[64];
   int blk[kTokMaxBlocks];
+  int page[kTokMaxBlocks];         // with paged keys: the page of blk[i]
 };
 
 __device__ __forceinline__ int64_t tok_job_id(const TokenParams& p, int64_t j) {
@@ -176,8 +179,17 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
       for (int wi = lane; wi < nwords; wi += 32) bitmap[wi] = 0u;
       __syncwarp();
 #pragma unroll
-      for (int k = 0; k < KW; ++k)
-        if (x[k] >= 0 && x[k] < nvis_blocks) atomicOr(bitmap + (x[k] >> 5), 1u << (x[k] & 31));
+      for (int k = 0; k < KW; ++k) {
+        bool keep = x[k] >= 0 && x[k] < nvis_blocks;
+        if (keep && p.pages) {   // a block whose page entry is out of range is dropped and reported
+          const int pg = __ldg(p.pages + static_cast<int64_t>(b) * p.nb + x[k]);
+          if (pg < 0 || pg >= p.num_pages) {
+            keep = false;
+            record_status(HISA_ERR_INVALID_ARG);
+          }
+        }
+        if (keep) atomicOr(bitmap + (x[k] >> 5), 1u << (x[k] & 31));
+      }
       __syncwarp();
       const int wpl = (nwords + 31) >> 5;                        // words per lane, in order
       int local = 0;
@@ -204,7 +216,10 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
         while (bits) {
           const int bit = __ffs(bits) - 1;
           bits &= bits - 1;
-          if (pos >= lo && pos < hi) J.blk[pos - lo] = (wi << 5) + bit;
+          if (pos >= lo && pos < hi) {
+            J.blk[pos - lo] = (wi << 5) + bit;
+            if (p.pages) J.page[pos - lo] = __ldg(p.pages + static_cast<int64_t>(b) * p.nb + (wi << 5) + bit);
+          }
           ++pos;
         }
       }
@@ -255,7 +270,7 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
           uint64_t* kf = k_full + kfi;
           mbar_arrive_expect_tx(kf, static_cast<uint32_t>(nblk_t * p.B * row_bytes));
           for (int q = 0; q < nblk_t; ++q) {
-            const int krow = kb + J.blk[first + q] * p.B;
+            const int krow = p.pages ? J.page[first + q] * p.B : kb + J.blk[first + q] * p.B;
             for (int pn = 0; pn < panels; ++pn)
               tma_load_2d(k_buf + st * k_bytes + pn * (kTokTileM * 128) + q * p.B * 128, &kmap, kf,
                           pn * panel_elems, krow);
@@ -345,7 +360,9 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
           const int s = slot_b < J.nblk ? (J.blk[slot_b] << bshift) + (c & (p.B - 1)) : p.L;
           const bool valid = s < J.n;
           float ksc = 1.f;
-          if (DT == DT_E4M3 && valid) ksc = __ldg(p.k_scale + static_cast<int64_t>(J.b) * p.L + s);
+          if (DT == DT_E4M3 && valid)
+            ksc = __ldg(p.k_scale + (p.pages ? static_cast<int64_t>(J.page[slot_b]) * p.B + (c & (p.B - 1))
+                                             : static_cast<int64_t>(J.b) * p.L + s));
           float acc = 0.f;
           if (H >= 32) {
             // 32 columns per TMEM load (32 registers live, not 64), four

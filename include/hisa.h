@@ -127,6 +127,30 @@ HISA_API hisa_status hisa_pool_blocks_range(const void* k, const float* k_scale,
                                             hisa_stream stream);
 
 /*
+ * Paged keys.  The pages leave the decoder's key storage open; a serving
+ * cache keeps each sequence's keys in fixed-size pages that it allocates as
+ * the sequence grows.  Here one page holds one HISA block:
+ *   k_pages       [num_pages, B, d] in shape->dtype (B = shape->block_size)
+ *   k_page_scale  [num_pages, B] fp32 (E4M3 only)
+ *   page_table    [batch, ceil(L/B)] int32: block j of sequence b (its keys
+ *                 j*B .. j*B+B-1) is page page_table[b * ceil(L/B) + j]
+ * L = shape->num_keys is the longest sequence the table covers; pages past a
+ * sequence's length are never read.  The results equal those of the
+ * contiguous entries on the keys the pages hold.  An entry that is read and
+ * lies outside [0, num_pages) is not dereferenced: the block is skipped and
+ * the device status word reports HISA_ERR_INVALID_ARG (hisa_get_status).
+ *
+ * hisa_pool_blocks_paged: hisa_pool_blocks_range over paged keys; block j's
+ * mean is over its first min(B, L - j*B) rows.  Same outputs, ownership and
+ * checks; page_table must be non-NULL and 4-byte aligned, num_pages >= 1.
+ */
+HISA_API hisa_status hisa_pool_blocks_paged(const void* k_pages, const float* k_page_scale,
+                                            const int32_t* page_table, int32_t num_pages,
+                                            void* kpool, float* kpool_scale,
+                                            const hisa_shape* shape, int32_t first_block,
+                                            int32_t block_count, hisa_stream stream);
+
+/*
  * Key compression ("StreamIndex: Memory-Bounded Compressed Sparse Attention
  * via Streaming Top-k", arXiv 2605.02568, abstract: the indexer runs over keys
  * compressed by a fixed ratio, 4 in V4-Flash).  ck[j] = mean of raw keys
@@ -198,6 +222,25 @@ HISA_API hisa_status hisa_token_score_topk(const void* q, const float* q_scale,
                                   const hisa_shape* shape, int32_t* topk_idx,
                                   float* topk_score, void* workspace,
                                   size_t ws_bytes, hisa_stream stream);
+
+/*
+ * hisa_token_score_topk over paged keys (layout as for
+ * hisa_pool_blocks_paged): the TMA tile load of a retained block reads its
+ * page.  Same result, outputs and workspace rule as hisa_token_score_topk.
+ * Tensor-core shapes only (bf16 or E4M3, head_dim * bytes 128 or 256,
+ * H 16, 32 or 64, B 16..128, top_m * B within the on-chip candidate
+ * buffers); others return HISA_ERR_UNSUPPORTED.  num_pages * B must fit in
+ * int32.
+ */
+HISA_API hisa_status hisa_token_score_topk_paged(const void* q, const float* q_scale,
+                                                 const float* w, const void* k_pages,
+                                                 const float* k_page_scale,
+                                                 const int32_t* page_table, int32_t num_pages,
+                                                 const int32_t* n_visible,
+                                                 const int32_t* block_idx,
+                                                 const hisa_shape* shape, int32_t* topk_idx,
+                                                 float* topk_score, void* workspace,
+                                                 size_t ws_bytes, hisa_stream stream);
 
 /*
  * Flat DSA indexer (the comparison path; HISA abstract: the flat scan of

@@ -106,3 +106,30 @@ def test_pointer_validation_returns_before_any_launch(L):
     assert L.hisa_pool_blocks_range(0x1000, None, 0x2000, None, ctypes.byref(s), 1 << 20, 4, None) == 0
     assert L.hisa_quantize_e4m3(0x1000, hb.HISA_BF16, 10, 100, 0x2000, 0x3000, None) == 2   # cols % 16
     assert L.hisa_compress_keys(0x1000, 0x2000, 1, 100, 128, 4, hb.HISA_E4M3, None) == 2
+
+
+def test_paged_entries_validate_on_the_host(L):
+    s = _shape()
+    P = ctypes.c_int32
+    # refinement over paged keys: no page table, no pages, a page range past int32 rows
+    assert L.hisa_token_score_topk_paged(0x1000, None, 0x2000, 0x3000, None, None, 8, 0x4000, 0x5000,
+                                         ctypes.byref(s), 0x6000, None, None, 0, None) == 1
+    assert L.hisa_token_score_topk_paged(0x1000, None, 0x2000, 0x3000, None, 0x7000, 0, 0x4000, 0x5000,
+                                         ctypes.byref(s), 0x6000, None, None, 0, None) == 1
+    assert L.hisa_token_score_topk_paged(0x1000, None, 0x2000, 0x3000, None, 0x7000, P(1 << 30), 0x4000, 0x5000,
+                                         ctypes.byref(s), 0x6000, None, None, 0, None) == 2
+    # E4M3 pages without their scales
+    s8 = _shape(dtype=hb.HISA_E4M3)
+    assert L.hisa_token_score_topk_paged(0x1000, 0x1100, 0x2000, 0x3000, None, 0x7000, 8, 0x4000, 0x5000,
+                                         ctypes.byref(s8), 0x6000, None, None, 0, None) == 1
+    # shapes the tensor-core kernel does not take have no paged path (fp32 runs on CUDA cores)
+    s32 = _shape(dtype=hb.HISA_F32, heads=4, head_dim=64, block_size=64, top_m=4, top_k=128)
+    assert L.hisa_token_score_topk_paged(0x1000, None, 0x2000, 0x3000, None, 0x7000, 8, 0x4000, 0x5000,
+                                         ctypes.byref(s32), 0x6000, None, None, 0, None) == 2
+    # pooling over paged keys
+    assert L.hisa_pool_blocks_paged(0x1000, None, None, 8, 0x2000, None, ctypes.byref(s), 0, 1, None) == 1
+    assert L.hisa_pool_blocks_paged(0x1000, None, 0x7000, 0, 0x2000, None, ctypes.byref(s), 0, 1, None) == 1
+    assert L.hisa_pool_blocks_paged(0x1000, None, 0x7000, 8, 0x2000, None, ctypes.byref(s), -1, 1, None) == 1
+    assert L.hisa_pool_blocks_paged(0x1000, None, 0x7000, 8, 0x2000, None, ctypes.byref(s8), 0, 1, None) == 1
+    # an empty range launches nothing
+    assert L.hisa_pool_blocks_paged(0x1000, None, 0x7000, 8, 0x2000, None, ctypes.byref(s), 1 << 20, 4, None) == 0
