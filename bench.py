@@ -451,6 +451,32 @@ def main():
                   "graph_ms_per_layer": cg, "graph_hisa_speedup": (flat["ms_per_layer"] / cg) if flat else None,
                   "what": "pooled keys of complete blocks kept between decode steps; a step pools the one block "
                           "its new key completes, then scores blocks and refines"}
+        if wl.num_keys % wl.block_size == 0:
+            # the same step over paged keys: one page per block, pages shuffled
+            bsz = k_static.shape[0]
+            gen = torch.Generator(device="cpu").manual_seed(7)
+            perm = torch.randperm(bsz * nb, generator=gen).to(torch.int32).to(k_static.device)
+            table = perm.view(bsz, nb).contiguous()
+            pages = torch.empty((bsz * nb, wl.block_size, wl.head_dim), dtype=k_static.dtype, device=k_static.device)
+            pages[perm.long()] = k_static.view(bsz * nb, wl.block_size, wl.head_dim)
+            pcache = kcache.clone()
+
+            def paged_step():
+                hb.hisa_pool_blocks_paged(pages, table, num_keys=k_static.shape[1], first_block=nb - 1,
+                                          block_count=1, kpool=pcache)
+                blocks = hb.hisa_block_score_topm(q, w, pcache, nv, num_keys=k_static.shape[1],
+                                                  block_size=wl.block_size, top_m=wl.top_m, workspace=ws_block)
+                return hb.hisa_token_score_topk_paged(q, w, pages, table, nv, blocks, num_keys=k_static.shape[1],
+                                                      top_k=wl.top_k)
+
+            for _ in range(max(3, args.warmup)):
+                paged_step()
+            same = bool(torch.equal(torch.sort(paged_step()[0], dim=-1)[0], torch.sort(cached_step()[0], dim=-1)[0]))
+            hb.get_status()
+            cached["paged_graph_ms_per_layer"] = max_over_ranks(graph_ms(paged_step, args.steps, flush, stream),
+                                                                world, dev)
+            cached["paged_matches_contiguous"] = same
+            del pages, pcache
 
     # ---- three levels: pooled super-blocks -> blocks -> tokens
     three = None
