@@ -37,9 +37,11 @@ FLOP_PER_PAIR_PER_HEAD_DIM = 2          # one multiply-add per (head, feature) p
 L2_FLUSH_BYTES = 256 << 20               # larger than the 126 MB L2
 
 # DRAM bytes (read + write) per launch of the refinement kernel from an ncu
-# capture of the same kernel and workload (see profiles/); a workload missing
-# here reports null.
-NCU_TRAFFIC = {"prefill_32k": 558115456 + 238302336}
+# capture of the same kernel build and workload (see profiles/); a workload
+# missing here reports null.  Empty: the kernel gained paged-key support after
+# the last capture (796,417,792 B per launch at prefill_32k), so that figure
+# no longer describes the kernel the bench times.
+NCU_TRAFFIC = {}
 
 
 def parse():
