@@ -5,10 +5,10 @@
  * What is computed.  "HISA: Efficient Hierarchical Indexing for Fine-Grained
  * Sparse Attention" (arXiv 2603.28458, abstract): the DSA indexer scores every
  * key of a query's prefix and keeps the top-k keys; HISA replaces that flat
- * scan with (1) a coarse stage that scores pooled block representations and
+ * scan with (1) a coarse stage that scores one pooled key per block and
  * keeps the best blocks, and (2) a refinement stage that runs the original
- * indexer only on the keys of the kept blocks, returning the same per-query
- * set of k token indices that the downstream sparse attention consumes.  The
+ * indexer only on the keys of the kept blocks, returning for each query the
+ * same kind of k-index set that the downstream sparse attention consumes.  The
  * indexer score used by every entry point is
  *
  *     I[t,s] = sum_h w[t,h] * ReLU(q[t,h,:] . k[s,:])

@@ -8,11 +8,11 @@ path never calls it, and it shares no code with the CUDA path.
 Sources.  The method is described in the abstract of "HISA: Efficient
 Hierarchical Indexing for Fine-Grained Sparse Attention" (arXiv 2603.28458),
 reproduced on several of the pages: DSA's lightweight indexer scores every key
-of the prefix for every query and keeps a top-k subset; HISA first scores
-pooled block representations and keeps the best blocks, then runs the original
-indexer only on the keys of the retained blocks, returning the same per-query
-set of k token indices (the same page's claim list states that the output is a
-per-query set of k token indices).  Key compression by a ratio of 4 and the
+of the prefix for every query and keeps a top-k subset; HISA first scores one
+pooled key per block and keeps the best blocks, then runs the original indexer
+only on the keys of the kept blocks, returning for each query a set of k token
+indices (the claim list of one page states that the output has the same
+structure as DSA's).  Key compression by a ratio of 4 and the
 rule that the [queries, heads, keys] score tensor must never be materialised
 come from the abstract of "StreamIndex: Memory-Bounded Compressed Sparse
 Attention via Streaming Top-k" (arXiv 2605.02568).
@@ -109,7 +109,7 @@ def block_means(keys: np.ndarray, block: int) -> np.ndarray:
 
 
 def pool_blocks(keys: np.ndarray, block: int, dtype: str) -> np.ndarray:
-    """HISA pooled block representations for bf16/fp32 keys: the mean of each
+    """HISA's pooled block keys for bf16/fp32 keys: the mean of each
     block, rounded once to the key dtype."""
     return round_storage(block_means(keys, block), dtype)
 

@@ -18,6 +18,7 @@ import torch
 
 from oracle import hisa_oracle as ho
 from oracle import ofp8
+from oracle import sparse_attention as sa
 from oracle.run import Sequence
 from hierarchical_top_key_b200 import synthetic
 
@@ -409,6 +410,83 @@ def pin_tiny_workload_invariants():
         fi, _ = seq.flat(int(t))
         found_needles += int(s in set(fi.tolist()))
     assert found_needles >= len(inp.needle_pos[0]) - 1, found_needles
+
+
+
+# ---------------------------------------------------------------- attention over the selected keys
+
+
+def _attn_case(seed=3, H=3, L=9, dk=5, dv=4):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((H, dk)), rng.standard_normal((L, dk)), rng.standard_normal((L, dv)),
+            float(1.0 / np.sqrt(dk)))
+
+
+def pin_sparse_attention_brute_force():
+    """Tiny inputs by explicit loops over a Python set of positions."""
+    import math
+    q, k, v, scale = _attn_case()
+    for row in ([4], [0, 3, 8], [8, -1, 2, 2, -1, 5], [-1, -1], list(range(9))):
+        o, lse = sa.sparse_attention_query(q, k, v, row, scale)
+        sel = sorted({i for i in row if i >= 0})
+        for h in range(q.shape[0]):
+            if not sel:
+                assert lse[h] == -math.inf and not np.any(o[h])
+                continue
+            logits = [scale * sum(q[h, i] * k[s, i] for i in range(k.shape[1])) for s in sel]
+            z = sum(math.exp(x) for x in logits)
+            assert abs(lse[h] - math.log(z)) < 1e-12
+            for c in range(v.shape[1]):
+                want = sum(math.exp(x) / z * v[s, c] for x, s in zip(logits, sel))
+                assert abs(o[h, c] - want) < 1e-12, (row, h, c)
+
+
+def pin_sparse_attention_closed_forms():
+    q, k, v, scale = _attn_case(seed=5)
+    # one selected key: its value row, whatever the query
+    o, lse = sa.sparse_attention_query(q, k, v, [6, -1, 6], scale)
+    np.testing.assert_array_equal(o, np.broadcast_to(v[6], o.shape))
+    np.testing.assert_allclose(lse, scale * (q @ k[6]), rtol=0, atol=1e-14)
+    # a zero query weighs every selected key equally: the mean value row, lse = log |S|
+    sel = [1, 4, 4, 7, -1]
+    o, lse = sa.sparse_attention_query(np.zeros_like(q), k, v, sel, scale)
+    np.testing.assert_allclose(o, np.broadcast_to(v[[1, 4, 7]].mean(axis=0), o.shape), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse, np.log(3.0), rtol=0, atol=1e-14)
+    # affine maps of the values pass through (the weights sum to one)
+    o1, _ = sa.sparse_attention_query(q, k, v, [0, 2, 5, 8], scale)
+    o2, _ = sa.sparse_attention_query(q, k, 3.0 * v - 2.0, [0, 2, 5, 8], scale)
+    np.testing.assert_allclose(o2, 3.0 * o1 - 2.0, rtol=1e-13, atol=1e-13)
+
+
+def pin_sparse_attention_dense_special_case():
+    """Every key selected is plain attention: torch's scaled_dot_product_attention
+    in float64 (keys and values shared by the heads), causal and not; the lse
+    is scipy's logsumexp of the selected logits."""
+    from scipy.special import logsumexp
+    q, k, v, scale = _attn_case(seed=7, H=4, L=11, dk=6, dv=3)
+    Q = k.shape[0]
+    qs = np.random.default_rng(8).standard_normal((Q, q.shape[0], q.shape[1]))
+    tq = torch.from_numpy(qs).permute(1, 0, 2)[None]                  # [1, H, Q, dk]
+    tk = torch.from_numpy(k)[None, None].expand(1, q.shape[0], -1, -1)
+    tv = torch.from_numpy(v)[None, None].expand(1, q.shape[0], -1, -1)
+    for causal in (False, True):
+        want = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale)
+        want = want[0].permute(1, 0, 2).numpy()                        # [Q, H, dv]
+        idx = np.array([[s if (s <= t or not causal) else -1 for s in range(Q)] for t in range(Q)])
+        o, lse = sa.sparse_attention(qs, k, v, idx, scale)
+        np.testing.assert_allclose(o, want, rtol=1e-12, atol=1e-13)
+        for t in range(Q):
+            n = t + 1 if causal else Q
+            np.testing.assert_allclose(lse[t], logsumexp(scale * qs[t] @ k[:n].T, axis=1), rtol=1e-13, atol=1e-13)
+
+
+def pin_sparse_attention_is_a_function_of_the_set():
+    q, k, v, scale = _attn_case(seed=9)
+    base = sa.sparse_attention_query(q, k, v, [2, 5, 7], scale)
+    for row in ([7, 5, 2], [5, -1, 2, 7, 7], [-1, 2, 2, 5, -1, 7, 5]):
+        got = sa.sparse_attention_query(q, k, v, row, scale)
+        np.testing.assert_array_equal(got[0], base[0])
+        np.testing.assert_array_equal(got[1], base[1])
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -6,6 +6,7 @@ import pytest
 import oracle_pins
 from oracle import hisa_oracle as ho
 from oracle import ofp8
+from oracle import sparse_attention as sa
 
 
 def _no_relu(q_t, w_t, keys):
@@ -82,6 +83,41 @@ def _second_level_unforced(q_t, w_t, kpool, cands, c_t, top_m):
     return np.sort(cands[ho.top_by_score(s, top_m)]).astype(np.int64)
 
 
+def _padding_as_position(idx_row):
+    return np.unique(np.asarray(idx_row, np.int64))          # -1 reads the last key
+
+
+def _repeats_counted(idx_row):
+    r = np.asarray(idx_row, np.int64)
+    return np.sort(r[r >= 0])                                 # a repeated index weighs twice
+
+
+_orig_attn = sa.sparse_attention_query
+
+
+def _softmax_over_heads(q_t, keys, values, idx_row, scale):
+    s = sa.selected_positions(idx_row)
+    if s.size == 0:
+        return _orig_attn(q_t, keys, values, idx_row, scale)
+    logits = scale * (np.asarray(q_t, np.float64) @ np.asarray(keys, np.float64)[s].T)
+    e = np.exp(logits - logits.max(axis=0, keepdims=True))
+    p = e / e.sum(axis=0, keepdims=True)
+    return p @ np.asarray(values, np.float64)[s], np.log(np.exp(logits).sum(axis=1))
+
+
+def _scale_dropped(q_t, keys, values, idx_row, scale):
+    return _orig_attn(q_t, keys, values, idx_row, 1.0)
+
+
+def _lse_without_max(q_t, keys, values, idx_row, scale):
+    o, lse = _orig_attn(q_t, keys, values, idx_row, scale)
+    s = sa.selected_positions(idx_row)
+    if s.size:
+        lg = scale * (np.asarray(q_t, np.float64) @ np.asarray(keys, np.float64)[s].T)
+        lse = lse - lg.max(axis=1)
+    return o, lse
+
+
 _orig_e4m3 = ofp8.e4m3_encode
 _orig_bf16 = ofp8.bf16_round
 
@@ -98,6 +134,11 @@ MUTATIONS = {
     "three_levels_current_not_forced": [(ho, "select_blocks_among", _second_level_unforced)],
     "e4m3_ties_away": [(ofp8, "e4m3_encode", _e4m3_half_away), (ho, "e4m3_encode", _e4m3_half_away)],
     "bf16_double_rounding": [(ofp8, "bf16_round", _bf16_via_fp32), (ho, "bf16_round", _bf16_via_fp32)],
+    "attention_padding_as_position": [(sa, "selected_positions", _padding_as_position)],
+    "attention_repeats_counted": [(sa, "selected_positions", _repeats_counted)],
+    "attention_softmax_over_heads": [(sa, "sparse_attention_query", _softmax_over_heads)],
+    "attention_scale_dropped": [(sa, "sparse_attention_query", _scale_dropped)],
+    "attention_lse_without_max": [(sa, "sparse_attention_query", _lse_without_max)],
 }
 
 
