@@ -143,6 +143,16 @@ def dequantize_e4m3_rows(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
     return e4m3_decode(codes) * np.asarray(scale, np.float64)[..., None]
 
 
+def quantize_q_tokens(q: np.ndarray):
+    """E4M3 q with one scale per query token, taken over all H*d values of the
+    token (reading R10 of the task's per-token FP8 variant).
+    q [Q, H, d] -> (codes uint8 [Q, H, d], scale f32 [Q])."""
+    q = np.asarray(q)
+    Qn, H, d = q.shape
+    codes, scale = quantize_e4m3_rows(q.reshape(Qn, H * d).astype(np.float32))
+    return codes.reshape(Qn, H, d), scale
+
+
 def pool_blocks_e4m3(codes: np.ndarray, scale: np.ndarray, block: int):
     """Pooled blocks for E4M3 keys: the float64 mean of the dequantised keys of
     each block, rounded to float32, then re-quantised per block."""

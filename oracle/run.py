@@ -33,11 +33,11 @@ class Sequence:
         self.n_visible = inputs.n_visible[b].astype(np.int64)
         if fp8:
             Qn, H, d = q.shape
-            qc, qs = ho.quantize_e4m3_rows(q.reshape(Qn, H * d).astype(np.float32))
+            qc, qs = ho.quantize_q_tokens(q)
             kc, ks = ho.quantize_e4m3_rows(keys.astype(np.float32))
-            self.q_codes, self.q_scale = qc.reshape(Qn, H, d), qs
+            self.q_codes, self.q_scale = qc, qs
             self.k_codes, self.k_scale = kc, ks
-            q = ho.dequantize_e4m3_rows(qc, qs).reshape(Qn, H, d)
+            q = ho.dequantize_e4m3_rows(qc.reshape(Qn, H * d), qs).reshape(Qn, H, d)
             keys = ho.dequantize_e4m3_rows(kc, ks)
             pc, ps = ho.pool_blocks_e4m3(kc, ks, self.block)
             self.kpool_codes, self.kpool_scale = pc, ps

@@ -81,6 +81,46 @@ def pin_golden_bf16():
     np.testing.assert_array_equal(ofp8.bf16_round(xs), np.array([c["bf16"] for c in g["cases"]]))
 
 
+def _f32_from_bits(hexes):
+    return np.array([int(h, 16) for h in hexes], np.uint32).view(np.float32)
+
+
+def pin_golden_pool_e4m3():
+    """Pooled E4M3 keys: exact mean of the dequantised keys, rounded to fp32,
+    re-quantised per block with the fp32 decision (hand-worked cases)."""
+    g = _load("pool_e4m3.json")
+    for c in g["pool_cases"]:
+        codes = np.array(c["codes"], np.uint8)
+        scale = _f32_from_bits(c["scale_bits"])
+        pc, ps = ho.pool_blocks_e4m3(codes, scale, c["block_size"])
+        np.testing.assert_array_equal(pc, np.array(c["pooled_codes"], np.uint8), err_msg=c["name"])
+        np.testing.assert_array_equal(np.asarray(ps, np.float32).view(np.uint32),
+                                      _f32_from_bits(c["pooled_scale_bits"]).view(np.uint32), err_msg=c["name"])
+
+
+def pin_golden_q_token_scale():
+    """The oracle's E4M3 view of a sequence quantises q with one scale per
+    token over all heads (hand-worked case, through run.Sequence)."""
+    g = _load("pool_e4m3.json")
+    for c in g["q_token_cases"]:
+        q = np.array(c["q"], np.float32)
+        Qn, H, d = q.shape
+        wl = synthetic.small_case(num_keys=4, num_queries=Qn, first_query_pos=4 - Qn, heads=H, head_dim=d,
+                                  block_size=2, top_m=1, top_k=1, dtype="f32", needles=0, name="q_token_golden")
+        keys = np.ones((1, 4, d), np.float32)
+        pos = np.arange(4 - Qn, 4, dtype=np.int64)[None]
+        inp = synthetic.Inputs(wl, q[None], keys, np.ones((1, Qn, H), np.float32), pos,
+                               synthetic.visible_keys(pos, 1), np.zeros((1, 0), np.int64), np.zeros((1, 0), np.int64))
+        seq = Sequence(inp, 0, fp8=True)
+        np.testing.assert_array_equal(seq.q_codes, np.array(c["q_codes"], np.uint8), err_msg=c["name"])
+        np.testing.assert_array_equal(np.asarray(seq.q_scale, np.float32).view(np.uint32),
+                                      _f32_from_bits(c["q_scale_bits"]).view(np.uint32), err_msg=c["name"])
+        # the oracle scores with the dequantised values code * token scale
+        deq = ofp8.e4m3_decode(np.array(c["q_codes"], np.uint8)) * \
+            _f32_from_bits(c["q_scale_bits"]).astype(np.float64)[:, None, None]
+        np.testing.assert_array_equal(seq.q, deq, err_msg=c["name"])
+
+
 # ---------------------------------------------------------------- library special cases
 
 

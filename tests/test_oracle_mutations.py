@@ -118,6 +118,39 @@ def _lse_without_max(q_t, keys, values, idx_row, scale):
     return o, lse
 
 
+def _pool_e4m3_ratio_in_fp64(codes, scale, block):
+    # scale and quotient kept in float64: no fp32 decision
+    means = ho.block_means(ho.dequantize_e4m3_rows(codes, scale), block)
+    amax = np.abs(means).max(axis=1)
+    s = np.where(amax > 0, amax / 448.0, 1.0)
+    return ofp8.e4m3_encode(means / s[:, None]), s.astype(np.float32)
+
+
+def _pool_e4m3_mean_unrounded(codes, scale, block):
+    # fp32 scale, but the float64 mean is divided before any fp32 rounding
+    means = ho.block_means(ho.dequantize_e4m3_rows(codes, scale), block)
+    amax = np.abs(means.astype(np.float32)).max(axis=1)
+    s = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    return ofp8.e4m3_encode((means / s[:, None].astype(np.float64)).astype(np.float32)), s
+
+
+def _pool_e4m3_scale_from_keys(codes, scale, block):
+    # block scale from the absmax of the block's dequantised keys, not of their mean
+    deq = ho.dequantize_e4m3_rows(codes, scale)
+    means = ho.block_means(deq, block).astype(np.float32)
+    nb = means.shape[0]
+    amax = np.array([np.abs(deq[b * block:(b + 1) * block]).max() for b in range(nb)], np.float32)
+    s = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    return ofp8.e4m3_encode((means / s[:, None]).astype(np.float32)), s
+
+
+def _q_scale_per_head(q):
+    q = np.asarray(q)
+    Qn, H, d = q.shape
+    codes, scale = ho.quantize_e4m3_rows(q.reshape(Qn * H, d).astype(np.float32))
+    return codes.reshape(Qn, H, d), scale.reshape(Qn, H).max(axis=1)
+
+
 _orig_e4m3 = ofp8.e4m3_encode
 _orig_bf16 = ofp8.bf16_round
 
@@ -134,6 +167,10 @@ MUTATIONS = {
     "three_levels_current_not_forced": [(ho, "select_blocks_among", _second_level_unforced)],
     "e4m3_ties_away": [(ofp8, "e4m3_encode", _e4m3_half_away), (ho, "e4m3_encode", _e4m3_half_away)],
     "bf16_double_rounding": [(ofp8, "bf16_round", _bf16_via_fp32), (ho, "bf16_round", _bf16_via_fp32)],
+    "e4m3_pool_quotient_in_fp64": [(ho, "pool_blocks_e4m3", _pool_e4m3_ratio_in_fp64)],
+    "e4m3_pool_mean_not_rounded_to_fp32": [(ho, "pool_blocks_e4m3", _pool_e4m3_mean_unrounded)],
+    "e4m3_pool_scale_from_keys": [(ho, "pool_blocks_e4m3", _pool_e4m3_scale_from_keys)],
+    "e4m3_q_scale_per_head": [(ho, "quantize_q_tokens", _q_scale_per_head)],
     "attention_padding_as_position": [(sa, "selected_positions", _padding_as_position)],
     "attention_repeats_counted": [(sa, "selected_positions", _repeats_counted)],
     "attention_softmax_over_heads": [(sa, "sparse_attention_query", _softmax_over_heads)],
