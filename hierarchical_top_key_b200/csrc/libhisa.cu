@@ -8,7 +8,6 @@
 #include <cstdarg>
 #include <algorithm>
 #include <cmath>
-#include <mutex>
 #include <vector>
 
 #include <cudaTypedefs.h>
@@ -971,25 +970,14 @@ constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB of fp32 blo
 // cudaGetSymbolAddress below.
 static __device__ __align__(256) float g_static_block_scores[kStaticScratchBytes / sizeof(float)];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_static_mu;
-void* g_static_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device, resolved once
-// per device with that device current.
+// Device address of the scratch array on the current device.  Looked up on
+// every call (the lookup allocates nothing), so an address never outlives the
+// context it was taken in, e.g. across a cudaDeviceReset.
 hisa_status static_scratch(float** out) {
-  int dev = 0;
-  hisa_status e = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  void* p = nullptr;
+  hisa_status e = cuda_check(cudaGetSymbolAddress(&p, g_static_block_scores), "cudaGetSymbolAddress(block-score scratch)");
   if (e != HISA_OK) return e;
-  if (dev < 0 || dev >= kMaxDevices) return fail(HISA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  std::lock_guard<std::mutex> lock(g_static_mu);
-  if (g_static_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cuda_check(cudaGetSymbolAddress(&p, g_static_block_scores), "cudaGetSymbolAddress(block-score scratch)");
-    if (e != HISA_OK) return e;
-    g_static_ptr[dev] = p;
-  }
-  *out = static_cast<float*>(g_static_ptr[dev]);
+  *out = static_cast<float*>(p);
   return HISA_OK;
 }
 

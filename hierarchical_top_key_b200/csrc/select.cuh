@@ -1,13 +1,22 @@
 // select.cuh - block-wide exact top-k selection on order-preserving uint32
-// keys (radix select, 8 bits per pass), ties resolved to the lower position.
+// keys, ties resolved to the lower position.  Key 0 marks an absent element
+// and is never emitted.  Keys are read through a functor, so the same code
+// serves rows in global memory (flat scores, block scores) and candidate
+// buffers in shared memory (the fused refinement stage).
 //
-// The selection finds the key T of the k-th largest element by four
-// histogram passes (one digit each, most significant first), then emits every
-// element with key > T (in any order) and the lowest-positioned elements with
-// key == T, which fill the remaining slots.  Key 0 marks an absent element and
-// is never emitted.  Keys are read through a functor, so the same code serves
-// rows in global memory (flat scores, block scores) and candidate buffers in
-// shared memory (the fused refinement stage).
+// Two selectors, tried in this order where the caller has the row's key range:
+//  - linear bins (scan_topk, two_pass_topk, two_pass_topk_rows): a histogram
+//    of up to 2048 equal-width bins over [kmin, kmax], a block-parallel search
+//    for the bin holding the k-th place, one counting pass and a block scan,
+//    then one write pass; the members of the boundary bin are gathered into a
+//    small buffer and ranked exactly.  Returns false when that bin overflows
+//    its buffer, and the caller falls back to
+//  - radix select (block_topk_range, block_topk): digits of 11 bits, most
+//    significant first, over only the bits in which kmin and kmax differ, so
+//    the number of histogram passes varies with the row (at most three for 32
+//    bits); it finds the key T of the k-th largest element, then emits every
+//    element with key > T in any order and the lowest-positioned elements with
+//    key == T into the remaining slots.
 #pragma once
 #include "common.cuh"
 

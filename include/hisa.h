@@ -321,8 +321,9 @@ HISA_API hisa_status dsa_flat_indexer_topk_sampled(const void* q, const float* q
  *    Shapes with batch*Q*round_up(ceil(L/B), 4)*4 bytes above 16 MiB return
  *    HISA_ERR_WORKSPACE without launching anything.
  *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
- *    The first call on each device looks up the array's device address on the
- *    current device (cudaGetSymbolAddress); make that first call before any
+ *    Each call looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress, which allocates nothing); the first call on a
+ *    device may load the library's device code there, so make it before any
  *    stream capture.
  *  - All calls share the array and it keeps the last call's contents (nothing
  *    in it needs to start cleared).  Calls that overlap on the GPU, on

@@ -133,3 +133,17 @@ def test_paged_entries_validate_on_the_host(L):
     assert L.hisa_pool_blocks_paged(0x1000, None, 0x7000, 8, 0x2000, None, ctypes.byref(s8), 0, 1, None) == 1
     # an empty range launches nothing
     assert L.hisa_pool_blocks_paged(0x1000, None, 0x7000, 8, 0x2000, None, ctypes.byref(s), 1 << 20, 4, None) == 0
+
+
+def test_static_scratch_refuses_oversized_shape(L):
+    """hisa_block_score_topm_static keeps the block scores in a built-in 16 MiB
+    array; a shape whose scores need more is refused on the host, before any
+    CUDA call (without a GPU an accepted shape would fail at the first CUDA
+    call instead, so the placeholder pointers are never used either way)."""
+    cap = 16 << 20
+    nb = 256                                   # 32768 keys in blocks of 128
+    rows = 2 * cap // (nb * 4)                 # twice the array's capacity
+    s = _shape(num_queries=rows, num_keys=32768, block_size=128)
+    st = L.hisa_block_score_topm_static(0x1000, None, 0x2000, 0x3000, None, 0x4000, ctypes.byref(s), 0x5000, None)
+    assert st == 3
+    assert b"16777216" in L.hisa_last_error()
