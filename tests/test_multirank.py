@@ -1,9 +1,13 @@
 """The multi-GPU host logic of the benchmark on CPU: two gloo ranks.
 
-Every rank runs an independent replica (its own seed, no data-path
-collective); the only exchange is the max-over-ranks reduction of the step
-time, and the job's throughput counts every rank's queries over that time.
-The reference arm runs on rank 0 alone."""
+--split sequences: every rank runs its own sequences of the job (its own
+seed, no data-path collective); the only exchange is the max-over-ranks
+reduction of the step time, and the job's throughput counts every rank's
+queries over that time.  --split queries: one workload is split over the
+ranks by causal work and the shards' index rows are assembled with one
+all-gather; here each rank runs the CPU oracle on its shard, and the
+assembled result must equal the one-process oracle result.  The reference
+arm runs on rank 0 alone."""
 import os
 import socket
 import subprocess
@@ -54,6 +58,75 @@ def test_two_rank_replicas_reduce_max_time():
     from hierarchical_top_key_b200 import synthetic
     wl = synthetic.WORKLOADS["tiny"]
     np.testing.assert_allclose(res[0][3], wl.batch * wl.num_queries * 2 / 2e-3)
+
+
+def _oracle_rows(inp, t0, t1):
+    from oracle.run import Sequence
+    from oracle import hisa_oracle as ho
+    wl = inp.workload
+    seq = Sequence(inp, 0)
+    rows = np.full((t1 - t0, wl.top_k), -1, np.int32)
+    for i, t in enumerate(range(t0, t1)):
+        _, idx, _ = seq.hisa(t)
+        rows[i] = ho.pad_row(idx, wl.top_k, -1)
+    return rows
+
+
+def _split_rank_main(rank, world, port, out):
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    from hierarchical_top_key_b200 import partition, synthetic
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        wl = synthetic.WORKLOADS["tiny"]
+        inp = synthetic.generate(wl, 0, batch=1)                 # one job: every rank draws the same inputs
+        shards = partition.shard_job(inp.n_visible, wl.block_size, wl.top_m, world)
+        s = shards[rank]
+        mine = torch.from_numpy(_oracle_rows(inp, s.t0, s.t1))[None]
+        full = bench.gather_shards(mine, shards, wl.batch, wl.num_queries, wl.top_k, world)
+        out[rank] = (full.numpy(), [(x.t0, x.t1) for x in shards],
+                     partition.shard_work(inp.n_visible, wl.block_size, wl.top_m, shards))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_query_split_reassembles_the_one_rank_result():
+    from hierarchical_top_key_b200 import partition, synthetic
+    world = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_split_rank_main, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
+        res = dict(out)
+    wl = synthetic.WORKLOADS["tiny"]
+    inp = synthetic.generate(wl, 0, batch=1)
+    whole = _oracle_rows(inp, 0, wl.num_queries)[None]
+    for r in range(world):
+        np.testing.assert_array_equal(res[r][0], whole)          # every rank holds the assembled [1, Q, k]
+    ranges = res[0][1]
+    assert ranges[0][0] == 0 and ranges[-1][1] == wl.num_queries
+    assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))  # contiguous, disjoint, covering
+    # balanced by causal work, not by count: each shard within one query's work of an equal share
+    work = partition.query_work(inp.n_visible, wl.block_size, wl.top_m)
+    for w_r in res[0][2]:
+        assert w_r <= work.sum() / world + work.max()
+    assert ranges[0][1] - ranges[0][0] > wl.num_queries // world  # early queries are cheaper
+
+
+def test_sequence_split_keeps_whole_sequences():
+    from hierarchical_top_key_b200 import partition
+    nv = np.full((64, 1), 131072, np.int32)
+    nv[::3] = 4096                                               # uneven sequences
+    for world in (1, 2, 3, 8):
+        shards = partition.shard_job(nv, 128, 64, world)
+        assert [s.seq0 for s in shards][0] == 0 and shards[-1].seq1 == 64
+        assert all(a.seq1 == b.seq0 for a, b in zip(shards, shards[1:]))
+        assert all(s.t0 == 0 and s.t1 == 1 for s in shards)
+        work = partition.query_work(nv, 128, 64).sum(axis=1)
+        for w_r in partition.shard_work(nv, 128, 64, shards):
+            assert w_r <= work.sum() / world + work.max()
 
 
 def test_reference_arm_runs_on_rank_zero_only():
