@@ -23,7 +23,7 @@ import torch
 from . import build as _build
 
 HISA_F32, HISA_BF16, HISA_E4M3 = 0, 1, 2
-OP_BLOCK, OP_TOKEN, OP_FLAT, OP_FLAT_SAMPLED, OP_BLOCK_REFINE = 1, 2, 3, 4, 5
+OP_BLOCK, OP_TOKEN, OP_FLAT, OP_FLAT_SAMPLED, OP_BLOCK_REFINE, OP_FROM_HOST = 1, 2, 3, 4, 5, 6
 STATUS = {0: "HISA_OK", 1: "HISA_ERR_INVALID_ARG", 2: "HISA_ERR_UNSUPPORTED", 3: "HISA_ERR_WORKSPACE",
           4: "HISA_ERR_CUDA", 5: "HISA_ERR_TIMEOUT"}
 
@@ -59,6 +59,9 @@ _SIGS = {
                                     _P, ctypes.c_size_t, _P],
     "dsa_flat_indexer_topk": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t, _P],
     "dsa_flat_indexer_topk_sampled": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, _P, _P, ctypes.c_size_t, _P],
+    "hisa_indexer_from_host": [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Shape), _P, ctypes.c_int32, _P,
+                               ctypes.c_size_t, _P],
+    "hisa_sparse_attention": [_P, _P, _P] + [ctypes.c_int32] * 7 + [ctypes.c_float, _P, _P, _P],
     "hisa_workspace_size": [ctypes.c_int32, ctypes.POINTER(Shape), ctypes.POINTER(ctypes.c_size_t)],
     "hisa_get_status": [_P],
     "hisa_selftest_wait_timeout": [ctypes.c_uint64, _P],
@@ -241,8 +244,19 @@ def hisa_block_score_topm_static(q, w, kpool, n_visible, *, num_keys: int, block
     return out
 
 
+def _token_workspace(shape, device, workspace):
+    """The refinement stage's optional workspace: the caller's, or one sized
+    by hisa_workspace_size (None when the shape has no use for one)."""
+    need = workspace_size(OP_TOKEN, shape)
+    if need == 0:
+        return None, 0
+    if workspace is not None and workspace.numel() >= need:
+        return workspace, workspace.numel()
+    return _workspace(need, device), need
+
+
 def hisa_token_score_topk(q, w, k, n_visible, block_idx, *, block_size: int, top_k: int, q_scale=None,
-                          k_scale=None, want_scores: bool = False):
+                          k_scale=None, want_scores: bool = False, workspace: Optional[torch.Tensor] = None):
     """Refinement stage: (topk_idx [batch, Q, top_k] int32, scores or None)."""
     top_m = block_idx.shape[-1]
     shape = make_shape(q, k, block_size, top_m, top_k)
@@ -250,11 +264,11 @@ def hisa_token_score_topk(q, w, k, n_visible, block_idx, *, block_size: int, top
     b, Q = q.shape[:2]
     idx = torch.empty((b, Q, top_k), dtype=torch.int32, device=q.device)
     sc = torch.empty((b, Q, top_k), dtype=torch.float32, device=q.device) if want_scores else None
-    need = workspace_size(OP_TOKEN, shape)
-    ws = _workspace(need, q.device) if need > 0 else None
+    ws, nbytes = _token_workspace(shape, q.device, workspace)
     _check(load().hisa_token_score_topk(q.data_ptr(), _ptr(q_scale), w.data_ptr(), k.data_ptr(), _ptr(k_scale),
                                         n_visible.data_ptr(), block_idx.data_ptr(), ctypes.byref(shape),
-                                        idx.data_ptr(), _ptr(sc), _ptr(ws), need, _stream()), "hisa_token_score_topk")
+                                        idx.data_ptr(), _ptr(sc), _ptr(ws), nbytes, _stream()),
+           "hisa_token_score_topk")
     return idx, sc
 
 
@@ -290,7 +304,8 @@ def hisa_pool_blocks_paged(k_pages, page_table, *, num_keys: int, first_block: i
 
 
 def hisa_token_score_topk_paged(q, w, k_pages, page_table, n_visible, block_idx, *, num_keys: int, top_k: int,
-                                q_scale=None, k_page_scale=None, want_scores: bool = False):
+                                q_scale=None, k_page_scale=None, want_scores: bool = False,
+                                workspace: Optional[torch.Tensor] = None):
     """Refinement stage over paged keys (layout as hisa_pool_blocks_paged):
     (topk_idx [batch, Q, top_k] int32, scores or None), equal to
     hisa_token_score_topk on the same keys stored contiguously."""
@@ -304,12 +319,11 @@ def hisa_token_score_topk_paged(q, w, k_pages, page_table, n_visible, block_idx,
     shape = Shape(b, num_keys, Q, H, d, B, block_idx.shape[-1], top_k, dtype_code(q))
     idx = torch.empty((b, Q, top_k), dtype=torch.int32, device=q.device)
     sc = torch.empty((b, Q, top_k), dtype=torch.float32, device=q.device) if want_scores else None
-    need = workspace_size(OP_TOKEN, shape)
-    ws = _workspace(need, q.device) if need > 0 else None
+    ws, nbytes = _token_workspace(shape, q.device, workspace)
     _check(load().hisa_token_score_topk_paged(q.data_ptr(), _ptr(q_scale), w.data_ptr(), k_pages.data_ptr(),
                                               _ptr(k_page_scale), page_table.data_ptr(), k_pages.shape[0],
                                               n_visible.data_ptr(), block_idx.data_ptr(), ctypes.byref(shape),
-                                              idx.data_ptr(), _ptr(sc), _ptr(ws), need, _stream()),
+                                              idx.data_ptr(), _ptr(sc), _ptr(ws), nbytes, _stream()),
            "hisa_token_score_topk_paged")
     return idx, sc
 
@@ -342,6 +356,27 @@ def dsa_flat_indexer_topk_sampled(q, w, k, n_visible, *, top_k: int, q_scale=Non
                                                 idx.data_ptr(), _ptr(sc), ws.data_ptr(), ws.numel(), _stream()),
            "dsa_flat_indexer_topk_sampled")
     return idx, sc
+
+
+def hisa_sparse_attention(q, kv, idx, *, scale: float, d_v: int = 512):
+    """Attention over the selected keys (latent KV shared by the heads, value =
+    the first d_v features): q [batch, Q, H, d_qk] bf16, kv [batch, L, d_qk]
+    bf16, idx [batch, Q, top_k] int32 -> (o [batch, Q, H, d_v] bf16,
+    lse [batch, Q, H] fp32)."""
+    _need(q, "q", 4)
+    _need(kv, "kv", 3)
+    _need(idx, "idx", 3)
+    b, Q, H, dqk = q.shape
+    if kv.shape[0] != b or kv.shape[2] != dqk or idx.shape[:2] != (b, Q) or idx.dtype != torch.int32:
+        raise ValueError("kv must be [batch, L, d_qk] and idx int32 [batch, Q, top_k]")
+    if q.dtype != torch.bfloat16 or kv.dtype != torch.bfloat16:
+        raise TypeError("q and kv must be bfloat16")
+    o = torch.empty((b, Q, H, d_v), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((b, Q, H), dtype=torch.float32, device=q.device)
+    _check(load().hisa_sparse_attention(q.data_ptr(), kv.data_ptr(), idx.data_ptr(), b, Q, kv.shape[1], H, dqk,
+                                        d_v, idx.shape[2], float(scale), o.data_ptr(), lse.data_ptr(), _stream()),
+           "hisa_sparse_attention")
+    return o, lse
 
 
 def hisa_block_refine_topm(q, w, kpool, n_visible, superblock_idx, *, num_keys: int, block_size: int, top_m: int,
@@ -393,6 +428,7 @@ class HisaIndexer:
     def __init__(self, block_size: int, top_m: int, top_k: int):
         self.block_size, self.top_m, self.top_k = block_size, top_m, top_k
         self._ws = None
+        self._host_ws = None
 
     def __call__(self, q, w, k, n_visible, q_scale=None, k_scale=None, want_scores=False, return_blocks=False):
         kpool, kps = hisa_pool_blocks(k, self.block_size, k_scale)
@@ -408,105 +444,40 @@ class HisaIndexer:
 
 
     def from_host(self, q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, n_visible: torch.Tensor,
-                  out: torch.Tensor, chunks: int = 16, device=None) -> torch.Tensor:
+                  out: torch.Tensor, chunks: int = 16, device=None, q_scale: Optional[torch.Tensor] = None,
+                  k_scale: Optional[torch.Tensor] = None) -> torch.Tensor:
         """The indexer on inputs in (pinned) host memory, writing the indices into
-        the host tensor `out` [batch, Q, top_k] int32.
-
-        The work is cut into `chunks` pieces (query ranges of a single sequence,
-        or ranges of sequences) run as a pipeline on three streams: the copy of
-        piece i+1 in, the kernels of piece i and the copy of piece i-1 out
-        overlap.  A piece copies only the keys its queries see that earlier
-        pieces did not, and pools only the blocks those keys complete (the
-        coarse stage scores complete blocks only).  Returns `out`; the caller's
+        the host tensor `out` [batch, Q, top_k] int32, through the C entry point
+        hisa_indexer_from_host (copies in, kernels and copies out pipelined over
+        `chunks` pieces on the library's streams).  The device workspace is
+        allocated here, once per shape, and kept.  Returns `out`; the caller's
         current stream waits for the last copy, so events recorded on it
-        bracket the whole call.  bf16 / fp32 inputs, keys already in the
-        indexer's key space."""
+        bracket the whole call."""
         for t, name, nd in ((q, "q", 4), (w, "w", 3), (k, "keys", 3), (n_visible, "n_visible", 2),
                             (out, "out", 3)):
             if t.is_cuda or not t.is_contiguous() or t.dim() != nd:
                 raise ValueError(f"{name} must be a contiguous host tensor with {nd} dims")
+        for t, name in ((q_scale, "q_scale"), (k_scale, "k_scale")):
+            if t is not None and (t.is_cuda or not t.is_contiguous()):
+                raise ValueError(f"{name} must be a contiguous host tensor")
         b, Q, H, d = q.shape
-        L = k.shape[1]
-        B, m, kk = self.block_size, self.top_m, self.top_k
-        if tuple(out.shape) != (b, Q, kk) or out.dtype != torch.int32:
+        if tuple(out.shape) != (b, Q, self.top_k) or out.dtype != torch.int32:
             raise ValueError("out must be an int32 [batch, Q, top_k] host tensor")
+        if n_visible.dtype != torch.int32 or tuple(n_visible.shape) != (b, Q):
+            raise ValueError("n_visible must be int32 [batch, Q]")
+        if k.shape[0] != b or k.shape[2] != d or dtype_code(k) != dtype_code(q):
+            raise ValueError("keys must be [batch, L, d] in q's dtype")
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-        lib = load()
-        dt = dtype_code(q)
-        nb = -(-L // B)
-        nv_host = n_visible.numpy()
-        # pieces: query ranges of one sequence, or ranges of whole sequences
-        if b == 1:
-            bounds = [(0, 1, (Q * i) // chunks, (Q * (i + 1)) // chunks) for i in range(chunks)]
-        else:
-            bounds = [((b * i) // chunks, (b * (i + 1)) // chunks, 0, Q) for i in range(chunks)]
-        bounds = [x for x in bounds if x[1] > x[0] and x[3] > x[2]]
-        rows_max = max((s1 - s0) * (t1 - t0) for s0, s1, t0, t1 in bounds)
-        qd = torch.empty_like(q, device=dev)
-        wd = torch.empty_like(w, device=dev)
-        kd = torch.empty_like(k, device=dev)
-        nvd = torch.empty_like(n_visible, device=dev)
-        kpool = torch.empty((b, nb, d), dtype=k.dtype, device=dev)
-        blocks = torch.empty((b, Q, m), dtype=torch.int32, device=dev)
-        idx = torch.empty((b, Q, kk), dtype=torch.int32, device=dev)
-        wshape = Shape(rows_max, L, 1, H, d, B, m, 1, dt)
-        ws = _workspace(workspace_size(OP_BLOCK, wshape), dev)
-        cur = torch.cuda.current_stream(dev)
-        s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
-        start = torch.cuda.Event()
-        start.record(cur)
-        s_in.wait_event(start)
-        esz_q, esz_k = q.element_size(), k.element_size()
-        keys_in = [0] * b          # keys already copied, per sequence
-        pooled = [0] * b           # blocks already pooled, per sequence
-        for s0, s1, t0, t1 in bounds:
-            nseq, nq = s1 - s0, t1 - t0
-            # keys and blocks this piece needs beyond the earlier pieces
-            n_hi = int(min(L, max(1, nv_host[s0:s1, t0:t1].max())))
-            with torch.cuda.stream(s_in):
-                for sq in range(s0, s1):
-                    if n_hi > keys_in[sq]:
-                        kd[sq, keys_in[sq]:n_hi].copy_(k[sq, keys_in[sq]:n_hi], non_blocking=True)
-                        keys_in[sq] = n_hi
-                qd[s0:s1, t0:t1].copy_(q[s0:s1, t0:t1], non_blocking=True)
-                wd[s0:s1, t0:t1].copy_(w[s0:s1, t0:t1], non_blocking=True)
-                nvd[s0:s1, t0:t1].copy_(n_visible[s0:s1, t0:t1], non_blocking=True)
-                ready = torch.cuda.Event()
-                ready.record(s_in)
-            s_run.wait_event(ready)
-            with torch.cuda.stream(s_run):
-                st = s_run.cuda_stream
-                c_hi = (n_hi - 1) // B        # blocks below the last visible one are complete
-                for sq in range(s0, s1):
-                    if c_hi > pooled[sq]:
-                        shp = Shape(1, L, 1, 1, d, B, 1, 1, dt)
-                        _check(lib.hisa_pool_blocks_range(kd[sq].data_ptr(), None, kpool[sq].data_ptr(), None,
-                                                          ctypes.byref(shp), pooled[sq], c_hi - pooled[sq], st),
-                               "hisa_pool_blocks_range")
-                        pooled[sq] = c_hi
-                shp = Shape(nseq, L, nq, H, d, B, m, kk, dt)
-                if b == 1:
-                    qp = qd[0, t0].data_ptr(); wp = wd[0, t0].data_ptr(); nvp = nvd[0, t0:].data_ptr()
-                    bp = blocks[0, t0].data_ptr(); ip = idx[0, t0].data_ptr()
-                    kp, kpp = kd.data_ptr(), kpool.data_ptr()
-                else:
-                    qp, wp, nvp = qd[s0].data_ptr(), wd[s0].data_ptr(), nvd[s0].data_ptr()
-                    bp, ip = blocks[s0].data_ptr(), idx[s0].data_ptr()
-                    kp, kpp = kd[s0].data_ptr(), kpool[s0].data_ptr()
-                _check(lib.hisa_block_score_topm(qp, None, wp, kpp, None, nvp, ctypes.byref(shp), bp,
-                                                 ws.data_ptr(), ws.numel(), st), "hisa_block_score_topm")
-                _check(lib.hisa_token_score_topk(qp, None, wp, kp, None, nvp, bp, ctypes.byref(shp), ip, None,
-                                                 None, 0, st), "hisa_token_score_topk")
-                fin = torch.cuda.Event()
-                fin.record(s_run)
-            s_out.wait_event(fin)
-            with torch.cuda.stream(s_out):
-                out[s0:s1, t0:t1].copy_(idx[s0:s1, t0:t1], non_blocking=True)
-        last = torch.cuda.Event()
-        last.record(s_out)
-        # the device buffers were allocated on the current stream, which now
-        # waits for the last copy: freeing them on return is ordered after it
-        cur.wait_event(last)
+        shape = Shape(b, k.shape[1], Q, H, d, self.block_size, self.top_m, self.top_k, dtype_code(q))
+        need = workspace_size(OP_FROM_HOST, shape)
+        if self._host_ws is None or self._host_ws.numel() < need or self._host_ws.device != dev:
+            self._host_ws = _workspace(need, dev)
+        with torch.cuda.device(dev):
+            _check(load().hisa_indexer_from_host(q.data_ptr(), _ptr(q_scale), w.data_ptr(), k.data_ptr(),
+                                                 _ptr(k_scale), n_visible.data_ptr(), ctypes.byref(shape),
+                                                 out.data_ptr(), chunks, self._host_ws.data_ptr(),
+                                                 self._host_ws.numel(), torch.cuda.current_stream(dev).cuda_stream),
+                   "hisa_indexer_from_host")
         return out
 
 

@@ -20,7 +20,8 @@ Recipe (the pages print no data, so every real activation is replaced by):
 * q[t,h,:] i.i.d. N(0, sigma^2) across t, h and the feature dimension.
 * keys: an AR(1) chain along the sequence, independently per feature,
   k_0 = e_0, k_s = rho*k_{s-1} + sqrt(1-rho^2)*e_s with e ~ N(0,1), times sigma.
-* w[t,h] ~ U(0,1) * w_scale, kept in fp32.
+* w[t,h] ~ U(0,1) * w_scale, kept in fp32 (U(w_low,1) * w_scale for the test
+  cases with head weights of both signs).
 * needles: distinct uniform key positions s; for each, a query t is drawn
   uniformly among those that can see s, and k[s] := q[t, 0, :] (the stored,
   already-rounded value), so the key is an exact copy of a query head.
@@ -32,8 +33,10 @@ streams for q, keys, w and needles (and one set per sequence when batch > 1).
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 from typing import Optional
 
 import numpy as np
@@ -61,6 +64,7 @@ class Workload:
     compress_ratio: int = 1
     raw_keys: int = 0      # keys before compression (== num_keys when ratio is 1)
     description: str = ""
+    w_low: float = 0.0     # w ~ U(w_low, 1) * w_scale; below 0 the head weights take both signs
 
     @property
     def num_blocks(self) -> int:
@@ -161,12 +165,18 @@ def generate(workload: Workload | str, seed: int = 0, *, batch: Optional[int] = 
     needle_query = np.zeros((nb, wl.needles), np.int64)
     root = np.random.SeedSequence(seed)
     seq_streams = root.spawn(wl.batch)
-    for b in range(nb):
+
+    def draw(b):
+        # every value of sequence b comes from its own four streams, so the
+        # sequences can be drawn in any order, or at the same time
         sq, sk, sw, sn = (np.random.default_rng(s) for s in seq_streams[b].spawn(4))
         qb = sq.standard_normal((Q, H, d), dtype=np.float32) * np.float32(wl.sigma)
         q[b] = round_to_storage(qb, wl.dtype)
         keys[b] = round_to_storage(_ar1_keys(sk, raw, d, wl.rho, wl.sigma), wl.dtype)
-        w[b] = (sw.random((Q, H), dtype=np.float32) * np.float32(wl.w_scale)).astype(np.float32)
+        u = sw.random((Q, H), dtype=np.float32)
+        if wl.w_low:
+            u = u * np.float32(1.0 - wl.w_low) + np.float32(wl.w_low)
+        w[b] = (u * np.float32(wl.w_scale)).astype(np.float32)
         positions[b] = wl.first_query_pos + np.arange(Q, dtype=np.int64)
         if wl.needles:
             # a needle at raw position s is seen by queries whose prefix covers s
@@ -178,6 +188,13 @@ def generate(workload: Workload | str, seed: int = 0, *, batch: Optional[int] = 
                 keys[b, sj] = q[b, t, 0]
                 needle_pos[b, j] = sj
                 needle_query[b, j] = t
+
+    if nb > 1:
+        with concurrent.futures.ThreadPoolExecutor(min(nb, os.cpu_count() or 1, 16)) as ex:
+            list(ex.map(draw, range(nb)))
+    else:
+        for b in range(nb):
+            draw(b)
     n_visible = visible_keys(positions, wl.compress_ratio)
     return Inputs(wl, q, keys, w, positions, n_visible, needle_pos, needle_query)
 
@@ -185,7 +202,7 @@ def generate(workload: Workload | str, seed: int = 0, *, batch: Optional[int] = 
 def small_case(*, batch=1, num_keys=300, num_queries=None, heads=4, head_dim=64,
                block_size=64, top_m=3, top_k=40, dtype="f32", first_query_pos=0,
                needles=4, rho=0.9, sigma=1.0, w_scale=1.0, compress_ratio=1,
-               name="small") -> Workload:
+               name="small", w_low=0.0) -> Workload:
     """A custom workload for tests (ragged sizes, odd shapes)."""
     raw = num_keys * compress_ratio
     if num_queries is None:
@@ -194,4 +211,54 @@ def small_case(*, batch=1, num_keys=300, num_queries=None, heads=4, head_dim=64,
                     heads=heads, head_dim=head_dim, block_size=block_size, top_m=top_m,
                     top_k=top_k, dtype=dtype, rho=rho, sigma=sigma, w_scale=w_scale,
                     needles=needles, first_query_pos=first_query_pos,
-                    compress_ratio=compress_ratio, raw_keys=raw)
+                    compress_ratio=compress_ratio, raw_keys=raw, w_low=w_low)
+
+
+# ---------------------------------------------------------------- attention inputs
+#
+# The consumer of the indexer's output (attention over the selected keys) in
+# latent form: one row of ATTN_DQK features per key position shared by every
+# head (ATTN_DV latent features, which are also the value, then positional
+# ones), and ATTN_HEADS query heads.  The pages give no dimensions for it; these
+# are those of DeepSeek-V3.2's absorbed sparse MLA.  q and the rows are i.i.d.
+# N(0, 1) rounded to bf16; the softmax scale is ATTN_SCALE.
+
+ATTN_HEADS, ATTN_DQK, ATTN_DV = 128, 576, 512
+ATTN_SCALE = 1.0 / math.sqrt(192.0)
+
+
+def attention_inputs(batch: int, num_queries: int, num_keys: int, seed: int = 0, heads: int = ATTN_HEADS):
+    """(q [batch, Q, heads, ATTN_DQK], kv [batch, L, ATTN_DQK]) as float32 arrays
+    holding bf16 values, from two streams of SeedSequence(seed)."""
+    sq, sk = (np.random.default_rng(s) for s in np.random.SeedSequence(seed).spawn(2))
+    q = round_to_storage(sq.standard_normal((batch, num_queries, heads, ATTN_DQK), dtype=np.float32), "bf16")
+    kv = round_to_storage(sk.standard_normal((batch, num_keys, ATTN_DQK), dtype=np.float32), "bf16")
+    return q, kv
+
+
+def attention_inputs_cuda(batch: int, num_queries: int, num_keys: int, seed: int = 0, heads: int = ATTN_HEADS,
+                          device="cuda"):
+    """The same distribution drawn directly on the GPU with torch's generator
+    (a different draw from attention_inputs; for timing workloads too large to
+    draw on the host): (q, kv) bf16 device tensors."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    q = torch.randn((batch, num_queries, heads, ATTN_DQK), generator=g, device=device,
+                    dtype=torch.float32).to(torch.bfloat16)
+    kv = torch.randn((batch, num_keys, ATTN_DQK), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    return q, kv
+
+
+def random_index_rows(batch: int, num_queries: int, num_keys: int, top_k: int, n_visible: np.ndarray,
+                      seed: int = 0) -> np.ndarray:
+    """Index rows shaped like an indexer's output: for query (b, t) min(top_k,
+    n_visible[b, t]) distinct positions below n_visible[b, t] in random order,
+    then -1 padding.  [batch, Q, top_k] int32."""
+    rng = np.random.default_rng(np.random.SeedSequence(seed).spawn(3)[2])
+    out = np.full((batch, num_queries, top_k), -1, np.int32)
+    for b in range(batch):
+        for t in range(num_queries):
+            n = int(min(n_visible[b, t], num_keys))
+            c = min(top_k, n)
+            if c:
+                out[b, t, :c] = rng.choice(n, size=c, replace=False)
+    return out

@@ -61,3 +61,11 @@ def iou(a, b) -> float:
     if not a and not b:
         return 1.0
     return len(a & b) / len(a | b)
+
+
+def recall(hisa, flat) -> float:
+    """|HISA & flat| / |flat| of two index rows (-1 = none)."""
+    a, b = set(int(x) for x in hisa if x >= 0), set(int(x) for x in flat if x >= 0)
+    if not b:
+        return 1.0
+    return len(a & b) / len(b)

@@ -50,3 +50,12 @@ def test_failed_estimates_take_the_fallback(lib):
     wl = synthetic.small_case(num_keys=2048, num_queries=48, first_query_pos=2000, heads=64, head_dim=128,
                               block_size=128, top_m=4, top_k=256, dtype="bf16", needles=0, name="flat_fallback")
     _flat_vs_oracle(synthetic.generate(wl), stride_boost=8.0)
+
+
+def test_threshold_path_with_signed_weights(lib):
+    """Head weights of both signs: many scores are negative, so the sample's
+    threshold and the selected keys fall on the sign half of the ordering keys."""
+    wl = synthetic.small_case(batch=2, num_keys=4096, num_queries=64, first_query_pos=4032, heads=64, head_dim=128,
+                              block_size=128, top_m=4, top_k=128, dtype="bf16", needles=8, w_low=-1.0,
+                              name="flat_lite_signed")
+    _flat_vs_oracle(synthetic.generate(wl))

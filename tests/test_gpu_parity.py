@@ -44,6 +44,14 @@ SMALL = {
     "compressed": dict(num_keys=600, compress_ratio=4, num_queries=300, first_query_pos=2100, heads=64,
                        head_dim=128, block_size=64, top_m=4, top_k=96, dtype="bf16", needles=0,
                        name="compressed"),
+    # head weights of both signs: scores below zero, the sign half of the ordering keys
+    "signed_w_bf16": dict(num_keys=1500, heads=64, head_dim=128, block_size=64, top_m=6, top_k=200, dtype="bf16",
+                          needles=6, w_low=-1.0, name="signed_w_bf16"),
+    "signed_w_f32": dict(num_keys=700, heads=4, head_dim=64, block_size=64, top_m=3, top_k=50, dtype="f32",
+                         needles=4, w_low=-1.0, name="signed_w_f32"),
+    "signed_w_decode": dict(batch=6, num_keys=3000, num_queries=1, first_query_pos=2999, heads=64, head_dim=128,
+                            block_size=64, top_m=8, top_k=128, dtype="bf16", needles=4, w_low=-1.0,
+                            name="signed_w_decode"),
 }
 
 
@@ -94,7 +102,8 @@ def _check_workload(inp, fp8, queries_per_seq, seqs=None):
     rtol = parity.RTOL[dt]
     dev, out = _run_gpu(inp, fp8)
     seqs = range(wl.batch) if seqs is None else seqs
-    stats = dict(queries=0, swaps_block=0, swaps_tok=0, swaps_flat=0, block_mismatch=0, iou=[])
+    stats = dict(queries=0, swaps_block=0, swaps_tok=0, swaps_flat=0, block_mismatch=0, iou=[], recall=[],
+                 negative_scores=0)
     # token stage fed with the oracle's blocks for the sampled rows
     blocks_o = out["blocks"].clone()
     plan = {}
@@ -164,8 +173,11 @@ def _check_workload(inp, fp8, queries_per_seq, seqs=None):
             stats["swaps_flat"] += parity.check_selection(fi[fi >= 0], fcand, fs, wl.top_k, what + " flat")
             parity.check_scores(fi, g["flat_sc"][b, t], lambda ix: seq.scores(t, ix), rtol, what + " flat scores")
             stats["iou"].append(parity.iou(hi, fi))
+            stats["recall"].append(parity.recall(hi, fi))
+            stats["negative_scores"] += int(np.sum(g["flat_sc"][b, t][fi >= 0] < 0))
     stats["mean_iou"] = float(np.mean(stats["iou"])) if stats["iou"] else 1.0
-    del stats["iou"]
+    stats["mean_recall"] = float(np.mean(stats["recall"])) if stats["recall"] else 1.0
+    del stats["iou"], stats["recall"]
     print(f"\n[parity] {wl.name}{'/fp8' if fp8 else ''}: {stats}")
     return stats
 
@@ -173,7 +185,9 @@ def _check_workload(inp, fp8, queries_per_seq, seqs=None):
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_small_parity(lib, name):
     inp = _inputs((name, tuple(sorted(SMALL[name].items()))))
-    _check_workload(inp, fp8=False, queries_per_seq=120)
+    stats = _check_workload(inp, fp8=False, queries_per_seq=120)
+    if SMALL[name].get("w_low", 0.0) < 0:
+        assert stats["negative_scores"] > 0, "signed weights should give some negative selected scores"
 
 
 @pytest.mark.parametrize("name", ["ragged_bf16", "batch_tail"])
@@ -201,11 +215,17 @@ def test_tiny_workload_every_query(lib):
 FULL = ["prefill_32k", "chunk_64k", "decode_128k", "compressed_256k"]
 
 
+# sampled queries per sequence at full size: first, last, around block
+# boundaries and random ones (every sequence of the decode workload)
+FULL_SAMPLES = {"prefill_32k": 512, "chunk_64k": 96, "decode_128k": 1, "compressed_256k": 96}
+
+
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_sampled(lib, name):
     inp = _inputs((name, ()))
-    seqs = [0, 17, 63] if inp.workload.batch > 1 else None
-    _check_workload(inp, fp8=False, queries_per_seq=6 if inp.workload.batch == 1 else 1, seqs=seqs)
+    stats = _check_workload(inp, fp8=False, queries_per_seq=FULL_SAMPLES[name])
+    if inp.workload.batch > 1:
+        assert stats["queries"] == inp.workload.batch
 
 
 def test_full_size_fp8_chunk_64k(lib):
