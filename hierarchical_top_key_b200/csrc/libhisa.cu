@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 #include <vector>
 
 #include <cudaTypedefs.h>
@@ -19,6 +20,8 @@
 #include "score_tc.cuh"
 #include "token_tc.cuh"
 #include "flat_lite.cuh"
+#include "sort.cuh"
+#include "sparse_attn.cuh"
 
 using namespace hisa;
 
@@ -293,6 +296,7 @@ hisa_status token_simt_h(const hisa_shape* s, const void* q, const float* qsc, c
 }
 
 constexpr size_t kSmemBudget = 232448;   // 227 KB opt-in dynamic shared memory per CTA
+constexpr int kSmemBudgetRows = 200 * 1024;   // shared memory per SM given to resident sorting CTAs
 
 bool token_tc_ok(const hisa_shape* s) {
   const int rb = s->head_dim * elem_bytes(s->dtype);
@@ -378,6 +382,8 @@ int token_parts(const hisa_shape* s) {
 size_t token_split_bytes(const hisa_shape* s, int parts) {
   return parts > 1 ? static_cast<size_t>(rows_of(s)) * parts * s->top_k * 8 : 0;
 }
+
+size_t host_pipe_bytes(const hisa_shape* s);   // device workspace of hisa_indexer_from_host
 
 // ------------------------------------------------------------ flat top-k without score rows
 
@@ -498,12 +504,49 @@ hisa_status check_indexer_ptrs(const hisa_shape* s, const void* q, const float* 
   return HISA_OK;
 }
 
+// Scored outputs are returned sorted by (score desc, index asc); rows longer
+// than the on-chip sort are refused up front, before anything is launched.
+hisa_status check_scored_rows(const hisa_shape* s, const float* topk_score) {
+  if (topk_score && s->top_k > kSortMaxK)
+    return fail(HISA_ERR_UNSUPPORTED, "with topk_score, top_k must be <= %d (rows are sorted on chip)", kSortMaxK);
+  if (topk_score && !aligned4(topk_score)) return fail(HISA_ERR_INVALID_ARG, "topk_score must be 4-byte aligned");
+  return HISA_OK;
+}
+
+hisa_status sort_scored_rows(int32_t* idx, float* score, int64_t rows, int k, cudaStream_t st) {
+  if (!score || rows == 0) return HISA_OK;
+  const int n = sort_pow2(k);
+  const int smem = n * static_cast<int>(sizeof(uint64_t));
+  hisa_status e = cuda_check(cudaFuncSetAttribute(sort_scored_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  smem), "sort_scored_rows attribute");
+  if (e != HISA_OK) return e;
+  const int per_sm = std::max(1, std::min(8, static_cast<int>(kSmemBudgetRows / std::max(smem, 1))));
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(rows, static_cast<int64_t>(num_sms()) * per_sm));
+  sort_scored_rows_kernel<<<grid, kSortThreads, smem, st>>>(idx, score, rows, k, n);
+  return launch_check("sort_scored_rows_kernel");
+}
+
 // The refinement stage after argument checks: split queries with the merge,
 // the tensor-core kernel, or (contiguous keys only) the CUDA-core kernel.
+hisa_status token_score_topk_unsorted(const void* q, const float* q_scale, const float* w, const void* k,
+                                      const float* k_scale, const int32_t* n_visible, const int32_t* block_idx,
+                                      const hisa_shape* s, int32_t* topk_idx, float* topk_score, void* workspace,
+                                      size_t ws_bytes, hisa_stream stream, KeyPages pg);
+
 hisa_status token_score_topk_checked(const void* q, const float* q_scale, const float* w, const void* k,
                                      const float* k_scale, const int32_t* n_visible, const int32_t* block_idx,
                                      const hisa_shape* s, int32_t* topk_idx, float* topk_score, void* workspace,
                                      size_t ws_bytes, hisa_stream stream, KeyPages pg) {
+  hisa_status e = token_score_topk_unsorted(q, q_scale, w, k, k_scale, n_visible, block_idx, s, topk_idx, topk_score,
+                                            workspace, ws_bytes, stream, pg);
+  if (e != HISA_OK) return e;
+  return sort_scored_rows(topk_idx, topk_score, rows_of(s), s->top_k, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hisa_status token_score_topk_unsorted(const void* q, const float* q_scale, const float* w, const void* k,
+                                      const float* k_scale, const int32_t* n_visible, const int32_t* block_idx,
+                                      const hisa_shape* s, int32_t* topk_idx, float* topk_score, void* workspace,
+                                      size_t ws_bytes, hisa_stream stream, KeyPages pg) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int parts = token_parts(s);
   if (parts > 1 && workspace && aligned16(workspace) && ws_bytes >= token_split_bytes(s, parts)) {
@@ -606,6 +649,7 @@ hisa_status hisa_workspace_size(int32_t op, const hisa_shape* s, size_t* bytes) 
     case HISA_OP_BLOCK_REFINE_TOPM:
       *bytes = static_cast<size_t>(pad4(rows_of(s)) * 4 + rows_of(s) * std::max(s->top_m - 1, 1) * 4);
       return HISA_OK;
+    case HISA_OP_INDEXER_FROM_HOST: *bytes = host_pipe_bytes(s); return HISA_OK;
     case HISA_OP_FLAT_TOPK_SAMPLED: {
       LitePlan lp;
       if (!lite_plan(s, &lp)) return fail(HISA_ERR_UNSUPPORTED, "shape not supported by the sampled flat top-k");
@@ -774,6 +818,8 @@ hisa_status hisa_token_score_topk(const void* q, const float* q_scale, const flo
   if (s->top_m > kMaxTopM) return fail(HISA_ERR_UNSUPPORTED, "top_m must be <= %d", kMaxTopM);
   if (static_cast<int64_t>(s->top_m) * s->block_size > kMaxCandidates)
     return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size must be <= %d", kMaxCandidates);
+  e = check_scored_rows(s, topk_score);
+  if (e != HISA_OK) return e;
   return token_score_topk_checked(q, q_scale, w, k, k_scale, n_visible, block_idx, s, topk_idx, topk_score,
                                   workspace, ws_bytes, stream, KeyPages{});
 }
@@ -795,6 +841,8 @@ hisa_status hisa_token_score_topk_paged(const void* q, const float* q_scale, con
   if (s->top_m > kMaxTopM) return fail(HISA_ERR_UNSUPPORTED, "top_m must be <= %d", kMaxTopM);
   if (static_cast<int64_t>(s->top_m) * s->block_size > kMaxCandidates)
     return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size must be <= %d", kMaxCandidates);
+  e = check_scored_rows(s, topk_score);
+  if (e != HISA_OK) return e;
   return token_score_topk_checked(q, q_scale, w, k_pages, k_page_scale, n_visible, block_idx, s, topk_idx,
                                   topk_score, workspace, ws_bytes, stream, KeyPages{page_table, num_pages});
 }
@@ -895,6 +943,8 @@ hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale, const flo
   e = check_indexer_ptrs(s, q, q_scale, w, k, k_scale, n_visible);
   if (e != HISA_OK) return e;
   if (!topk_idx || !aligned4(topk_idx)) return fail(HISA_ERR_INVALID_ARG, "topk_idx must be non-NULL, 4-byte aligned");
+  e = check_scored_rows(s, topk_score);
+  if (e != HISA_OK) return e;
   const int64_t ld = pad4(s->num_keys);
   const int64_t rows = rows_of(s);
   if (!workspace || !aligned16(workspace)) return fail(HISA_ERR_WORKSPACE, "workspace must be non-NULL, 16-byte aligned");
@@ -927,7 +977,7 @@ hisa_status dsa_flat_indexer_topk(const void* q, const float* q_scale, const flo
     e = launch_check("flat_select_kernel");
     if (e != HISA_OK) return e;
   }
-  return HISA_OK;
+  return sort_scored_rows(topk_idx, topk_score, rows, s->top_k, st);
 }
 
 hisa_status dsa_flat_indexer_topk_sampled(const void* q, const float* q_scale, const float* w, const void* k,
@@ -940,6 +990,8 @@ hisa_status dsa_flat_indexer_topk_sampled(const void* q, const float* q_scale, c
   if (e != HISA_OK) return e;
   if (!topk_idx || !aligned4(topk_idx)) return fail(HISA_ERR_INVALID_ARG, "topk_idx must be non-NULL, 4-byte aligned");
   LitePlan lp;
+  e = check_scored_rows(s, topk_score);
+  if (e != HISA_OK) return e;
   if (!lite_plan(s, &lp))
     return fail(HISA_ERR_UNSUPPORTED, "sampled flat top-k needs a tensor-core shape, num_keys divisible by the "
                                       "sample stride and top_k small enough for the pair buffer");
@@ -947,8 +999,287 @@ hisa_status dsa_flat_indexer_topk_sampled(const void* q, const float* q_scale, c
   if (ws_bytes < lp.fixed + lp.per_row * dense_group(s))
     return fail(HISA_ERR_WORKSPACE, "workspace holds fewer than one query group (%zu bytes needed)",
                 lp.fixed + lp.per_row * dense_group(s));
-  return flat_lite(s, lp, q, q_scale, w, k, k_scale, n_visible, topk_idx, topk_score, workspace, ws_bytes,
-                   reinterpret_cast<cudaStream_t>(stream));
+  e = flat_lite(s, lp, q, q_scale, w, k, k_scale, n_visible, topk_idx, topk_score, workspace, ws_bytes,
+                reinterpret_cast<cudaStream_t>(stream));
+  if (e != HISA_OK) return e;
+  return sort_scored_rows(topk_idx, topk_score, rows_of(s), s->top_k, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+// =================================================================== sparse attention
+
+extern "C" {
+
+hisa_status hisa_sparse_attention(const void* q, const void* kv, const int32_t* idx, int32_t batch,
+                                  int32_t num_queries, int32_t num_keys, int32_t heads, int32_t d_qk,
+                                  int32_t d_v, int32_t top_k, float scale, void* o, float* lse,
+                                  hisa_stream stream) {
+  if (batch < 1 || num_queries < 1 || num_keys < 1)
+    return fail(HISA_ERR_INVALID_ARG, "batch, num_queries and num_keys must be >= 1");
+  if (heads < 1 || heads % kAttnHeads != 0)
+    return fail(HISA_ERR_UNSUPPORTED, "heads must be a multiple of %d", kAttnHeads);
+  if (d_qk != kAttnDqk || d_v != kAttnDv)
+    return fail(HISA_ERR_UNSUPPORTED, "d_qk must be %d and d_v %d", kAttnDqk, kAttnDv);
+  if (top_k < 1 || top_k > kAttnMaxK) return fail(HISA_ERR_UNSUPPORTED, "top_k must be in [1, %d]", kAttnMaxK);
+  if (!std::isfinite(scale)) return fail(HISA_ERR_INVALID_ARG, "scale must be finite");
+  if (!q || !kv || !idx || !o || !lse) return fail(HISA_ERR_INVALID_ARG, "q, kv, idx, o and lse must be non-NULL");
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(o) || !aligned4(idx) || !aligned4(lse))
+    return fail(HISA_ERR_INVALID_ARG, "q, kv and o must be 16-byte aligned, idx and lse 4-byte aligned");
+  const int64_t rows = static_cast<int64_t>(batch) * num_queries;
+  const int slices = heads / kAttnHeads;
+  if (rows * slices * 2 > INT32_MAX) return fail(HISA_ERR_UNSUPPORTED, "too many (query, head slice) pairs");
+  CUtensorMap qm;
+  hisa_status e = tensor_map_2d(&qm, q, HISA_BF16, static_cast<uint64_t>(rows) * heads, kAttnDqk, kAttnHeads);
+  if (e != HISA_OK) return e;
+  const size_t smem = attn_smem_bytes();
+  e = cuda_check(cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(smem)), "sparse_attn attribute");
+  if (e != HISA_OK) return e;
+  AttnParams p{};
+  p.rows = rows; p.Q = num_queries; p.L = num_keys; p.slices = slices; p.top_k = top_k;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.idx = idx; p.kv = static_cast<const uint16_t*>(kv); p.o = static_cast<uint16_t*>(o); p.lse = lse;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows * slices * 2));
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cuda_check(cudaLaunchKernelEx(&cfg, sparse_attn_kernel, qm, p), "launch sparse_attn_kernel");
+  if (e != HISA_OK) return e;
+  return launch_check("sparse_attn_kernel");
+}
+
+}  // extern "C"
+
+// =================================================================== host buffers
+//
+// hisa_indexer_from_host: the whole indexer (pool -> coarse top-m -> refine
+// top-k) on inputs in host memory, for callers whose q, keys and weights
+// arrive from the host.  The work is cut into pieces (query ranges of one
+// sequence, or ranges of whole sequences) run as a pipeline on three streams
+// of the library's: the copy of piece i+1 in, the kernels of piece i and the
+// copy of piece i-1 out overlap.  A piece copies only the keys its queries
+// see beyond those earlier pieces copied, and pools only the blocks those
+// keys complete (the coarse stage scores complete blocks only).
+
+namespace {
+
+struct HostPipe {
+  cudaStream_t in = nullptr, run = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, ready = nullptr, fin = nullptr, last = nullptr;
+};
+
+constexpr int kMaxPipeDevices = 64;
+std::mutex g_pipe_mu;
+HostPipe g_pipe[kMaxPipeDevices];
+
+// The pipeline's streams and events on the current device, created on the
+// first call there and kept until the process exits.
+hisa_status host_pipe(HostPipe** out) {
+  int dev = 0;
+  hisa_status e = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (e != HISA_OK) return e;
+  if (dev < 0 || dev >= kMaxPipeDevices) return fail(HISA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  HostPipe& p = g_pipe[dev];
+  if (!p.in) {
+    cudaStream_t* ss[3] = {&p.in, &p.run, &p.out};
+    for (cudaStream_t* x : ss) {
+      e = cuda_check(cudaStreamCreateWithFlags(x, cudaStreamNonBlocking), "create pipeline stream");
+      if (e != HISA_OK) return e;
+    }
+    cudaEvent_t* es[4] = {&p.start, &p.ready, &p.fin, &p.last};
+    for (cudaEvent_t* x : es) {
+      e = cuda_check(cudaEventCreateWithFlags(x, cudaEventDisableTiming), "create pipeline event");
+      if (e != HISA_OK) return e;
+    }
+  }
+  *out = &p;
+  return HISA_OK;
+}
+
+constexpr size_t kPipeAlign = 256;
+
+size_t pipe_round(size_t n) { return (n + kPipeAlign - 1) / kPipeAlign * kPipeAlign; }
+
+// Device buffers of the host pipeline, carved from the caller's workspace.
+struct PipeBuffers {
+  uint8_t *q, *k, *kpool;
+  float *w, *q_scale, *k_scale, *kpool_scale;
+  int32_t *nv, *blocks, *idx;
+  void* coarse;
+  size_t coarse_bytes;
+  void* split;
+  size_t split_bytes;
+  size_t total;
+};
+
+PipeBuffers pipe_layout(const hisa_shape* s, uint8_t* base) {
+  const size_t es = static_cast<size_t>(elem_bytes(s->dtype));
+  const size_t rows = static_cast<size_t>(rows_of(s));
+  const size_t keys = static_cast<size_t>(s->batch) * s->num_keys;
+  const size_t nb = static_cast<size_t>(num_blocks(s));
+  const bool e4 = s->dtype == HISA_E4M3;
+  PipeBuffers b{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base ? base + off : nullptr;
+    off += pipe_round(bytes);
+    return p;
+  };
+  b.q = take(rows * s->heads * s->head_dim * es);
+  b.w = reinterpret_cast<float*>(take(rows * s->heads * 4));
+  b.nv = reinterpret_cast<int32_t*>(take(rows * 4));
+  b.k = take(keys * s->head_dim * es);
+  b.kpool = take(static_cast<size_t>(s->batch) * nb * s->head_dim * es);
+  b.q_scale = e4 ? reinterpret_cast<float*>(take(rows * 4)) : nullptr;
+  b.k_scale = e4 ? reinterpret_cast<float*>(take(keys * 4)) : nullptr;
+  b.kpool_scale = e4 ? reinterpret_cast<float*>(take(static_cast<size_t>(s->batch) * nb * 4)) : nullptr;
+  b.blocks = reinterpret_cast<int32_t*>(take(rows * s->top_m * 4));
+  b.idx = reinterpret_cast<int32_t*>(take(rows * s->top_k * 4));
+  b.coarse_bytes = rows * static_cast<size_t>(pad4(static_cast<int64_t>(nb))) * 4;
+  b.coarse = take(b.coarse_bytes);
+  // split refinement of small pieces: rows * parts <= SM count
+  b.split_bytes = static_cast<size_t>(num_sms()) * s->top_k * 8;
+  b.split = take(b.split_bytes);
+  b.total = off;
+  return b;
+}
+
+struct Piece {
+  int s0, s1, t0, t1;
+};
+
+size_t host_pipe_bytes(const hisa_shape* s) { return pipe_layout(s, nullptr).total; }
+
+}  // namespace
+
+extern "C" {
+
+hisa_status hisa_indexer_from_host(const void* q, const float* q_scale, const float* w, const void* k,
+                                   const float* k_scale, const int32_t* n_visible, const hisa_shape* s,
+                                   int32_t* topk_idx, int32_t pieces, void* workspace, size_t ws_bytes,
+                                   hisa_stream stream) {
+  hisa_status e = check_shape(s, true);
+  if (e != HISA_OK) return e;
+  if (!q || !w || !k || !n_visible || !topk_idx)
+    return fail(HISA_ERR_INVALID_ARG, "q, w, keys, n_visible and topk_idx must be non-NULL host pointers");
+  if (s->dtype == HISA_E4M3 && (!q_scale || !k_scale))
+    return fail(HISA_ERR_INVALID_ARG, "E4M3 inputs need q_scale and k_scale");
+  if (pieces < 0 || pieces > 256) return fail(HISA_ERR_INVALID_ARG, "pieces must be in [0, 256]");
+  if (s->top_m > kMaxTopM) return fail(HISA_ERR_UNSUPPORTED, "top_m must be <= %d", kMaxTopM);
+  if (static_cast<int64_t>(s->top_m) * s->block_size > kMaxCandidates)
+    return fail(HISA_ERR_UNSUPPORTED, "top_m * block_size must be <= %d", kMaxCandidates);
+  const PipeBuffers need = pipe_layout(s, nullptr);
+  if (!workspace || !aligned16(workspace) || ws_bytes < need.total)
+    return fail(HISA_ERR_WORKSPACE, "workspace needs %zu bytes (16-byte aligned device memory)", need.total);
+  const PipeBuffers d = pipe_layout(s, static_cast<uint8_t*>(workspace));
+  const int B = s->block_size, L = s->num_keys, Q = s->num_queries, H = s->heads, hd = s->head_dim;
+  const int64_t nb = num_blocks(s);
+  const size_t es = static_cast<size_t>(elem_bytes(s->dtype));
+  const size_t q_row = static_cast<size_t>(H) * hd * es, k_row = static_cast<size_t>(hd) * es;
+  const int P = pieces == 0 ? 16 : pieces;
+  // pieces: query ranges of a single sequence, or ranges of whole sequences
+  std::vector<Piece> plan;
+  for (int i = 0; i < P; ++i) {
+    Piece pc = s->batch == 1 ? Piece{0, 1, static_cast<int>(static_cast<int64_t>(Q) * i / P),
+                                     static_cast<int>(static_cast<int64_t>(Q) * (i + 1) / P)}
+                             : Piece{static_cast<int>(static_cast<int64_t>(s->batch) * i / P),
+                                     static_cast<int>(static_cast<int64_t>(s->batch) * (i + 1) / P), 0, Q};
+    if (pc.s1 > pc.s0 && pc.t1 > pc.t0) plan.push_back(pc);
+  }
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe* hp = nullptr;
+  e = host_pipe(&hp);
+  if (e != HISA_OK) return e;
+  cudaStream_t cur = reinterpret_cast<cudaStream_t>(stream);
+  const uint8_t* hq = static_cast<const uint8_t*>(q);
+  const uint8_t* hk = static_cast<const uint8_t*>(k);
+  auto h2d = [&](void* dst, const void* src, size_t bytes) {
+    return bytes ? cuda_check(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, hp->in), "copy in") : HISA_OK;
+  };
+  e = cuda_check(cudaEventRecord(hp->start, cur), "record start");
+  if (e != HISA_OK) return e;
+  e = cuda_check(cudaStreamWaitEvent(hp->in, hp->start, 0), "wait start");
+  if (e != HISA_OK) return e;
+  std::vector<int> keys_in(s->batch, 0), pooled(s->batch, 0);
+  for (const Piece& pc : plan) {
+    const int nseq = pc.s1 - pc.s0, nq = pc.t1 - pc.t0;
+    // keys this piece sees beyond the earlier pieces (n_visible read on the host)
+    int n_hi = 1;
+    for (int b = pc.s0; b < pc.s1; ++b)
+      for (int t = pc.t0; t < pc.t1; ++t) n_hi = std::max(n_hi, n_visible[static_cast<int64_t>(b) * Q + t]);
+    n_hi = std::min(n_hi, L);
+    for (int b = pc.s0; b < pc.s1; ++b) {
+      if (n_hi > keys_in[b]) {
+        const size_t r0 = static_cast<size_t>(b) * L + keys_in[b];
+        const size_t nr = static_cast<size_t>(n_hi - keys_in[b]);
+        if ((e = h2d(d.k + r0 * k_row, hk + r0 * k_row, nr * k_row)) != HISA_OK) return e;
+        if (d.k_scale && (e = h2d(d.k_scale + r0, k_scale + r0, nr * 4)) != HISA_OK) return e;
+        keys_in[b] = n_hi;
+      }
+    }
+    // this piece's rows of q, w, n_visible (and q scales): contiguous in both layouts
+    for (int b = pc.s0; b < pc.s1; ++b) {
+      const size_t r0 = static_cast<size_t>(b) * Q + pc.t0;
+      if ((e = h2d(d.q + r0 * q_row, hq + r0 * q_row, static_cast<size_t>(nq) * q_row)) != HISA_OK) return e;
+      if ((e = h2d(d.w + r0 * H, w + r0 * H, static_cast<size_t>(nq) * H * 4)) != HISA_OK) return e;
+      if ((e = h2d(d.nv + r0, n_visible + r0, static_cast<size_t>(nq) * 4)) != HISA_OK) return e;
+      if (d.q_scale && (e = h2d(d.q_scale + r0, q_scale + r0, static_cast<size_t>(nq) * 4)) != HISA_OK) return e;
+    }
+    if ((e = cuda_check(cudaEventRecord(hp->ready, hp->in), "record ready")) != HISA_OK) return e;
+    if ((e = cuda_check(cudaStreamWaitEvent(hp->run, hp->ready, 0), "wait ready")) != HISA_OK) return e;
+    // pool the blocks the new keys complete (every block below the last visible one)
+    const int c_hi = (n_hi - 1) / B;
+    for (int b = pc.s0; b < pc.s1; ++b) {
+      if (c_hi > pooled[b]) {
+        hisa_shape one = *s;
+        one.batch = 1;
+        e = hisa_pool_blocks_range(d.k + static_cast<size_t>(b) * L * k_row,
+                                   d.k_scale ? d.k_scale + static_cast<size_t>(b) * L : nullptr,
+                                   d.kpool + static_cast<size_t>(b) * nb * k_row,
+                                   d.kpool_scale ? d.kpool_scale + static_cast<size_t>(b) * nb : nullptr, &one,
+                                   pooled[b], c_hi - pooled[b], reinterpret_cast<hisa_stream>(hp->run));
+        if (e != HISA_OK) return e;
+        pooled[b] = c_hi;
+      }
+    }
+    hisa_shape ps = *s;
+    ps.batch = nseq;
+    ps.num_queries = nq;
+    // a piece of one sequence is that sequence with only the piece's queries;
+    // a piece of whole sequences starts at its first sequence
+    const size_t r0 = static_cast<size_t>(pc.s0) * Q + pc.t0;
+    const size_t kb = s->batch == 1 ? 0 : static_cast<size_t>(pc.s0);
+    const hisa_stream rs = reinterpret_cast<hisa_stream>(hp->run);
+    e = hisa_block_score_topm(d.q + r0 * q_row, d.q_scale ? d.q_scale + r0 : nullptr, d.w + r0 * H,
+                              d.kpool + kb * nb * k_row, d.kpool_scale ? d.kpool_scale + kb * nb : nullptr,
+                              d.nv + r0, &ps, d.blocks + r0 * s->top_m, d.coarse, d.coarse_bytes, rs);
+    if (e != HISA_OK) return e;
+    e = hisa_token_score_topk(d.q + r0 * q_row, d.q_scale ? d.q_scale + r0 : nullptr, d.w + r0 * H,
+                              d.k + kb * L * k_row, d.k_scale ? d.k_scale + kb * L : nullptr, d.nv + r0,
+                              d.blocks + r0 * s->top_m, &ps, d.idx + r0 * s->top_k, nullptr, d.split,
+                              d.split_bytes, rs);
+    if (e != HISA_OK) return e;
+    if ((e = cuda_check(cudaEventRecord(hp->fin, hp->run), "record fin")) != HISA_OK) return e;
+    if ((e = cuda_check(cudaStreamWaitEvent(hp->out, hp->fin, 0), "wait fin")) != HISA_OK) return e;
+    for (int b = pc.s0; b < pc.s1; ++b) {
+      const size_t rr = static_cast<size_t>(b) * Q + pc.t0;
+      e = cuda_check(cudaMemcpyAsync(topk_idx + rr * s->top_k, d.idx + rr * s->top_k,
+                                     static_cast<size_t>(nq) * s->top_k * 4, cudaMemcpyDeviceToHost, hp->out),
+                     "copy out");
+      if (e != HISA_OK) return e;
+    }
+  }
+  if ((e = cuda_check(cudaEventRecord(hp->last, hp->out), "record last")) != HISA_OK) return e;
+  return cuda_check(cudaStreamWaitEvent(cur, hp->last, 0), "wait last");
 }
 
 }  // extern "C"

@@ -28,8 +28,12 @@
  *  - Kernels that wait on on-chip barriers do so with a bounded spin; if a
  *    wait gives up, the kernel records HISA_ERR_TIMEOUT in a device status
  *    word and exits cleanly.  hisa_get_status() reads (and clears) that word.
- *  - Index outputs are -1 padded.  Index sets are returned in an unspecified
- *    order; when a score output is given, score[i] belongs to index[i].
+ *  - Index outputs are -1 padded.  Without a score output each row's indices
+ *    are a set in unspecified order.  With a score output, score[i] belongs
+ *    to index[i] and each row is sorted by (score desc, index asc), the
+ *    order that defines the top-k, with the -1 / -inf padding last; scored
+ *    rows are sorted on chip, so top_k <= 16384 when scores are requested
+ *    (HISA_ERR_UNSUPPORTED otherwise).
  *  - dtype HISA_E4M3: q and keys are OFP8 E4M3 codes with one fp32 scale per
  *    query token (over all H*d values) and one per key; the value of a code
  *    is code * scale.  For the other dtypes the scale pointers are ignored
@@ -87,7 +91,8 @@ enum {
   HISA_OP_TOKEN_SCORE_TOPK = 2,
   HISA_OP_FLAT_TOPK = 3,
   HISA_OP_FLAT_TOPK_SAMPLED = 4,
-  HISA_OP_BLOCK_REFINE_TOPM = 5
+  HISA_OP_BLOCK_REFINE_TOPM = 5,
+  HISA_OP_INDEXER_FROM_HOST = 6
 };
 
 /*
@@ -335,6 +340,70 @@ HISA_API hisa_status hisa_block_score_topm_static(const void* q, const float* q_
                                   const int32_t* n_visible,
                                   const hisa_shape* shape, int32_t* block_idx,
                                   hisa_stream stream);
+
+/*
+ * The whole HISA indexer (block pooling, coarse top-m, refinement top-k; HISA
+ * abstract, stages 1 and 2) on inputs that live in HOST memory, for callers
+ * whose q, keys and weights arrive from the host.  Layouts as for the device
+ * entry points, all pointers below HOST pointers:
+ *   q          [batch, Q, H, d] in dtype;  q_scale [batch, Q] fp32 (E4M3)
+ *   w          [batch, Q, H] fp32
+ *   k          [batch, L, d] in dtype;     k_scale [batch, L] fp32 (E4M3)
+ *   n_visible  [batch, Q] int32, read by the host during the call
+ *   topk_idx   [batch, Q, top_k] int32 (output), -1 padded, any order
+ * Page-locked host memory lets the copies overlap the kernels; pageable
+ * memory works but serialises them.
+ * The work is cut into `pieces` (0 = 16; at most 256) query ranges of one
+ * sequence, or ranges of whole sequences, run as a pipeline on three streams
+ * of the library's: the host-to-device copy of one piece, the kernels of the
+ * previous one and the device-to-host copy of the one before overlap.  A
+ * piece copies only the keys its queries see beyond those already copied,
+ * and pools only the blocks those keys complete (the coarse stage scores
+ * complete blocks only), so the result equals hisa_pool_blocks +
+ * hisa_block_score_topm + hisa_token_score_topk on the whole inputs.
+ *   workspace  DEVICE memory, 16-byte aligned, of at least
+ *              hisa_workspace_size(HISA_OP_INDEXER_FROM_HOST) bytes: the
+ *              device copies of every input, the pooled keys, the block and
+ *              token indices and the stages' scratch.
+ * Ordering: the pipeline starts after the work already enqueued on `stream`,
+ * and `stream` waits for the last copy out, so topk_idx is complete once the
+ * caller synchronises `stream` (or an event recorded on it after the call).
+ * The first call on a device creates the three non-blocking streams and four
+ * events it keeps until the process exits (make it before any stream
+ * capture); calls are serialised on the host by a lock.  Two calls that share
+ * a workspace must be ordered through their streams.
+ */
+HISA_API hisa_status hisa_indexer_from_host(const void* q, const float* q_scale, const float* w,
+                                            const void* k, const float* k_scale,
+                                            const int32_t* n_visible, const hisa_shape* shape,
+                                            int32_t* topk_idx, int32_t pieces, void* workspace,
+                                            size_t ws_bytes, hisa_stream stream);
+
+/*
+ * Attention over each query's selected keys: the consumer of the indexer's
+ * token-level top-k (HISA abstract: HISA keeps the index interface that the
+ * downstream sparse MLA operator reads; the pages give that operator no
+ * formula).  Latent attention in absorbed form, one key row per position
+ * shared by every head, its first d_v features being the value:
+ *     logit[h, j] = scale * q[t, h, :] . kv[s_j, :]
+ *     o[t, h, :]  = sum_j softmax_j(logit[h, :]) * kv[s_j, 0 : d_v]
+ *     lse[t, h]   = log sum_j exp(logit[h, j])      (natural log)
+ * over S_t = the positions in idx[t, :] with -1, out-of-range entries and
+ * repeats dropped; an empty S_t gives o = 0 and lse = -inf.
+ *   q    [batch, Q, heads, d_qk] bf16 (device)
+ *   kv   [batch, L, d_qk] bf16 (device)
+ *   idx  [batch, Q, top_k] int32 (device): the indexer's topk_idx
+ *   o    [batch, Q, heads, d_v] bf16 (device, output)
+ *   lse  [batch, Q, heads] fp32 (device, output)
+ * This build takes d_qk = 576, d_v = 512 (512 latent + 64 positional
+ * features), heads a multiple of 128 and top_k <= 4096; other shapes return
+ * HISA_ERR_UNSUPPORTED.  Each (query, 128-head slice) runs on a cluster of
+ * two CTAs; the score tensor [Q, heads, top_k] never leaves the chip.
+ */
+HISA_API hisa_status hisa_sparse_attention(const void* q, const void* kv, const int32_t* idx,
+                                           int32_t batch, int32_t num_queries, int32_t num_keys,
+                                           int32_t heads, int32_t d_qk, int32_t d_v, int32_t top_k,
+                                           float scale, void* o, float* lse, hisa_stream stream);
 
 /* Workspace bytes that let `op` run on `shape` in one pass (0 if none). */
 HISA_API hisa_status hisa_workspace_size(int32_t op, const hisa_shape* shape,

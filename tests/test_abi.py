@@ -147,3 +147,54 @@ def test_static_scratch_refuses_oversized_shape(L):
     st = L.hisa_block_score_topm_static(0x1000, None, 0x2000, 0x3000, None, 0x4000, ctypes.byref(s), 0x5000, None)
     assert st == 3
     assert b"16777216" in L.hisa_last_error()
+
+
+def test_scored_rows_longer_than_the_on_chip_sort_are_refused(L):
+    """With a score output rows come back sorted on chip, up to 16384 per row;
+    longer rows are refused before anything is launched."""
+    s = _shape(top_k=16385)
+    assert L.dsa_flat_indexer_topk(0x1000, None, 0x2000, 0x3000, None, 0x4000, ctypes.byref(s), 0x5000, 0x6000,
+                                   0x7000, 1 << 30, None) == 2
+    assert b"16384" in L.hisa_last_error()
+    s = _shape(top_k=16385, top_m=4, block_size=128)
+    assert L.hisa_token_score_topk(0x1000, None, 0x2000, 0x3000, None, 0x4000, 0x5000, ctypes.byref(s), 0x6000,
+                                   0x7000, None, 0, None) == 2
+
+
+def test_host_buffer_entry_validates_on_the_host(L):
+    """hisa_indexer_from_host: argument checks and the workspace rule, before
+    any stream, event or copy is made."""
+    s = _shape(num_keys=4096, num_queries=4096, top_m=8)
+    n = ctypes.c_size_t(0)
+    assert L.hisa_workspace_size(6, ctypes.byref(s), ctypes.byref(n)) == 0
+    # device copies of q (4096*64*128*2), keys, w, n_visible, pooled keys, block and token indices and scratch
+    assert n.value > 4096 * 64 * 128 * 2 + 4096 * 128 * 2 + 4096 * 2048 * 4
+    args = (0x1000, None, 0x2000, 0x3000, None, 0x4000, ctypes.byref(s), 0x5000)
+    assert L.hisa_indexer_from_host(None, None, 0x2000, 0x3000, None, 0x4000, ctypes.byref(s), 0x5000, 0, 0x6000,
+                                    n.value, None) == 1
+    assert L.hisa_indexer_from_host(*args, -1, 0x6000, n.value, None) == 1            # pieces out of range
+    assert L.hisa_indexer_from_host(*args, 0, 0x6000, n.value - 1, None) == 3         # workspace too small
+    assert L.hisa_indexer_from_host(*args, 0, 0x6001, n.value, None) == 3             # misaligned workspace
+    s8 = _shape(num_keys=4096, num_queries=4096, top_m=8, dtype=hb.HISA_E4M3)
+    assert L.hisa_indexer_from_host(0x1000, None, 0x2000, 0x3000, None, 0x4000, ctypes.byref(s8), 0x5000, 0,
+                                    0x6000, 1 << 40, None) == 1                       # E4M3 without scales
+
+
+def test_sparse_attention_validates_on_the_host(L):
+    """hisa_sparse_attention: shapes this build has no kernel for and bad
+    pointers are refused before any CUDA call."""
+    f = ctypes.c_float
+    ok = dict(q=0x1000, kv=0x2000, idx=0x3000, batch=1, Q=4, L=100, H=128, dqk=576, dv=512, k=64, scale=f(0.07),
+              o=0x4000, lse=0x5000)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.hisa_sparse_attention(a["q"], a["kv"], a["idx"], a["batch"], a["Q"], a["L"], a["H"], a["dqk"],
+                                       a["dv"], a["k"], a["scale"], a["o"], a["lse"], None)
+    assert call(H=64) == 2 and call(H=192) == 2          # heads: whole 128-head slices
+    assert call(dqk=192) == 2 and call(dv=128) == 2      # latent 512 + positional 64 only
+    assert call(k=0) == 2 and call(k=4097) == 2
+    assert call(batch=0) == 1 and call(L=0) == 1
+    assert call(scale=f(float("inf"))) == 1
+    assert call(q=None) == 1 and call(lse=None) == 1
+    assert call(kv=0x2008) == 1 and call(idx=0x3002) == 1
