@@ -1,0 +1,522 @@
+// sparse_attn.cuh - attention over each query's selected keys, the consumer of
+// the indexer's token-level top-k (HISA abstract: the output keeps the index
+// interface that the downstream sparse MLA operator reads).
+//
+// Latent attention in its absorbed form: every key position holds one row of
+// D_QK = 576 features shared by all heads (512 latent + 64 positional), and
+// its value is the first D_V = 512 of them.  For a query t with selected set
+// S_t (the index row with -1 and repeats dropped),
+//     logit[h, j] = scale * q[t, h, :] . kv[s_j, :]
+//     o[t, h, :]  = sum_j softmax_j(logit[h, :]) * kv[s_j, :D_V]
+//     lse[t, h]   = log sum_j exp(logit[h, j])          (natural log)
+// and an empty set gives o = 0, lse = -inf.
+//
+// One query's 128 heads are the M = 128 rows of every MMA, on a pair of CTAs
+// (a cluster of two).  Neither the query (128 x 576 bf16 = 144 KB) nor the
+// 512 fp32 accumulator columns of the output fit one SM next to the key
+// tiles and the scores, so the pair splits the features:
+//   CTA 0  features   0..255: q and key columns for part of every logit,
+//          the value columns   0..255 of the output
+//   CTA 1  features 256..575: the rest of every logit (with the 64
+//          positional features), the value columns 256..511
+// Each CTA computes a partial logit tile S_c = q_c . k_c^T (M = 128 heads,
+// N = 64 keys, K = its features) on tcgen05 into TMEM, the two partial tiles
+// are exchanged through distributed shared memory and summed (the sum is the
+// same in both CTAs: fp32 addition commutes), and both run the same online
+// softmax, so each can accumulate its half of the output, O_c += P . V_c,
+// with V_c the value columns it already holds (B operand read MN-major from
+// the key tile).  Keys are gathered from their positions with 16-byte
+// cp.async copies written straight into the 128-byte-swizzled layout the MMA
+// reads.
+//
+// Warp roles (10 warps):
+//   warp 0      TMEM owner, single-thread MMA issuer (QK of tile i, then
+//               PV of tile i-1)
+//   warp 1      q tile by TMA (once per query)
+//   warps 2..5  key gather (cp.async), two stages
+//   warps 6..9  softmax: thread = head row; exchange, online softmax, O
+//               rescaling in TMEM, P (bf16) to shared memory, epilogue
+// Every wait is bounded; a timeout sets the CTA's abort flag and the status
+// word, and the peer CTA's waits on it then time out too.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace hisa {
+
+constexpr int kAttnHeads = 128;            // M of every MMA: one query's heads
+constexpr int kAttnDqk = 576;
+constexpr int kAttnDv = 512;
+constexpr int kAttnTileN = 64;             // keys per tile
+constexpr int kAttnMaxK = 4096;            // longest index row
+constexpr int kAttnThreads = 320;
+constexpr int kAttnGatherBase = 64;        // warps 2..5
+constexpr int kAttnSoftBase = 192;         // warps 6..9
+constexpr int kAttnPanels = 5;             // 64-feature panels of the larger half
+constexpr uint32_t kAttnPanelQ = kAttnHeads * 128;     // bytes of one q panel (128 rows x 128 B)
+constexpr uint32_t kAttnPanelK = kAttnTileN * 128;     // bytes of one key panel (64 rows x 128 B)
+constexpr uint32_t kAttnStage = kAttnPanels * kAttnPanelK;
+constexpr uint32_t kAttnTmemS = 0;         // two 64-column logit buffers
+constexpr uint32_t kAttnTmemO = 256;       // 256 output columns
+
+struct AttnParams {
+  int64_t rows;              // batch * Q
+  int Q, L, slices;          // slices: heads / 128
+  int top_k;
+  float scale_log2;          // softmax scale * log2(e)
+  const int32_t* idx;        // [rows, top_k]
+  const uint16_t* kv;        // [batch, L, 576] bf16
+  uint16_t* o;               // [rows, heads, 512] bf16
+  float* lse;                // [rows, heads]
+};
+
+namespace sm100 {
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+// Arrive on an mbarrier of another CTA of the cluster, ordering this
+// thread's earlier shared::cluster stores before it.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3; "
+      "selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on a barrier completed by the other CTA of the cluster.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      record_status(HISA_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (the tensor core reads its operands through it).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns from registers into TMEM.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Shared-memory descriptor of an MN-major operand stored with the 128-byte
+// swizzle: rows of 128 bytes hold 64 consecutive MN elements for one K index,
+// 8-row groups along K are `sbo` bytes apart and 64-element groups along MN
+// `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// Instruction descriptor with the B operand MN-major (bf16, fp32 accumulate).
+__host__ __device__ constexpr uint32_t instr_desc_bmn(int M, int N) {
+  return instr_desc(M, N, 1u) | (1u << 16);
+}
+
+}  // namespace sm100
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+struct AttnSmem {
+  uint64_t q_full;
+  uint64_t kv_full[2], kv_empty[2];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full, pv_done;
+  uint64_t x_full, x_free;       // exchange of partial logits with the peer CTA
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int n_valid;
+  int pad;
+  int scan[kAttnThreads / 32 + 1];
+};
+
+inline size_t attn_smem_bytes() {
+  return 1024 + kAttnPanels * kAttnPanelQ      // q
+         + 2 * kAttnStage                      // key tiles
+         + kAttnHeads * 128                    // P (bf16, one 64-key panel)
+         + kAttnHeads * kAttnTileN * 4         // partial logits from the peer
+         + kAttnMaxK * 4                       // the query's sorted, deduplicated positions
+         + sizeof(AttnSmem) + 16;
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                     const AttnParams p) {
+  using namespace sm100;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_buf = smem;
+  uint8_t* kv_buf = q_buf + kAttnPanels * kAttnPanelQ;
+  uint8_t* p_buf = kv_buf + 2 * kAttnStage;
+  float* x_buf = reinterpret_cast<float*>(p_buf + kAttnHeads * 128);
+  int32_t* sidx = reinterpret_cast<int32_t*>(x_buf + kAttnHeads * kAttnTileN);
+  AttnSmem* sm = reinterpret_cast<AttnSmem*>(sidx + kAttnMaxK);
+  volatile int* abort_flag = &sm->abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();               // 0: features 0..255, 1: features 256..575
+  const uint32_t peer = rank ^ 1u;
+  const int64_t item = cluster_id_x();                   // (row, head slice)
+  const int64_t row = item / p.slices;
+  const int slice = static_cast<int>(item % p.slices);
+  const int b = static_cast<int>(row / p.Q);
+  const int npanels = rank == 0 ? 4 : 5;
+  const int feat0 = rank == 0 ? 0 : 256;
+  const int chunks_per_key = npanels * 8;                // 16-byte pieces of this CTA's part of a key row
+
+  if (tid == 0) {
+    mbar_init(&sm->q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm->kv_full[i], 128);
+      mbar_init(&sm->kv_empty[i], 1);
+      mbar_init(&sm->s_full[i], 1);
+      mbar_init(&sm->s_empty[i], 128);
+    }
+    mbar_init(&sm->p_full, 128);
+    mbar_init(&sm->pv_done, 1);
+    mbar_init(&sm->x_full, 128);
+    mbar_init(&sm->x_free, 128);
+    mbar_init(&sm->drain, 1);
+    sm->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) tmem_alloc(&sm->tmem_base, 512);
+  if (warp == 1 && lane == 0) tma_prefetch_desc(&qmap);
+
+  // ---- the query's positions: sorted, -1 / out-of-range / repeats dropped, compacted
+  const int K = p.top_k;
+  int npow = 1;
+  while (npow < K) npow <<= 1;
+  const int32_t* irow = p.idx + row * K;
+  for (int i = tid; i < npow; i += kAttnThreads) {
+    int v = i < K ? __ldg(irow + i) : INT32_MAX;
+    if (v < 0 || v >= p.L) v = INT32_MAX;             // not a key: sorts last, dropped below
+    sidx[i] = v;
+  }
+  __syncthreads();
+  for (int size = 2; size <= npow; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int q2 = tid; q2 < (npow >> 1); q2 += kAttnThreads) {
+        const int i = 2 * q2 - (q2 & (stride - 1)), j = i + stride;
+        const bool up = (i & size) == 0;
+        const int a = sidx[i], c = sidx[j];
+        if ((a > c) == up) { sidx[i] = c; sidx[j] = a; }
+      }
+      __syncthreads();
+    }
+  }
+  {
+    // keep the first of each run of equal positions; compact in order
+    const int per = (npow + kAttnThreads - 1) / kAttnThreads;
+    const int lo = tid * per, hi = min(npow, lo + per);
+    int keep[16];
+    int cnt = 0;
+    for (int i = lo; i < hi; ++i) {
+      const int v = sidx[i];
+      const bool k = v != INT32_MAX && (i == 0 || sidx[i - 1] != v);
+      keep[i - lo] = k ? v : -1;
+      cnt += k;
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) sm->scan[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w2 = 0; w2 < warp; ++w2) base += sm->scan[w2];
+    if (tid == kAttnThreads - 1) sm->n_valid = base + incl;
+    __syncthreads();                                   // every thread has read sidx[lo-1] before any write
+    int pos = base + incl - cnt;
+    for (int i = lo; i < hi; ++i)
+      if (keep[i - lo] >= 0) sidx[pos++] = keep[i - lo];
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                      // the peer's barriers exist before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem_base;
+  const int n_valid = sm->n_valid;
+  const int T = (n_valid + kAttnTileN - 1) / kAttnTileN;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_qk = instr_desc(kAttnHeads, kAttnTileN, 1u);
+      constexpr uint32_t id_pv = instr_desc_bmn(kAttnHeads, 256);
+      bool ok = T == 0 || mbar_wait(&sm->q_full, 0, abort_flag);
+      if (ok) tc_fence_after();
+      const uint64_t q_desc = desc_k_sw128(smem_u32(q_buf));
+      const uint64_t p_desc = desc_k_sw128(smem_u32(p_buf));
+      for (int i = 0; ok && i <= T; ++i) {
+        if (i < T) {
+          const int st = i & 1;
+          const uint32_t ph = static_cast<uint32_t>((i >> 1) & 1);
+          if (!(ok = mbar_wait(&sm->kv_full[st], ph, abort_flag))) break;
+          if (!(ok = mbar_wait(&sm->s_empty[st], ph ^ 1u, abort_flag))) break;
+          tc_fence_after();
+          const uint64_t k_desc = desc_k_sw128(smem_u32(kv_buf + st * kAttnStage));
+          const uint32_t d = tmem + kAttnTmemS + st * kAttnTileN;
+          if (npanels == 4) mma_tile_sw128<DT_BF16, 16, kAttnHeads, kAttnTileN>(d, q_desc, k_desc, id_qk);
+          else mma_tile_sw128<DT_BF16, 20, kAttnHeads, kAttnTileN>(d, q_desc, k_desc, id_qk);
+          mma_commit(&sm->s_full[st]);
+        }
+        if (i >= 1) {
+          const int j = i - 1, sj = j & 1;
+          if (!(ok = mbar_wait(&sm->p_full, static_cast<uint32_t>(j & 1), abort_flag))) break;
+          tc_fence_after();
+          // V: the first four 64-feature panels of the key tile, MN-major
+          const uint32_t v0 = smem_u32(kv_buf + sj * kAttnStage);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t vd = desc_mn_sw128(v0 + ks * 16 * 128, kAttnPanelK, 1024);
+            mma<DT_BF16>(tmem + kAttnTmemO, p_desc + static_cast<uint64_t>(ks * 2), vd, id_pv,
+                         (j > 0 || ks > 0) ? 1u : 0u);
+          }
+          mma_commit(&sm->kv_empty[sj]);
+          mma_commit(&sm->pv_done);
+        }
+      }
+      mma_commit(&sm->drain);
+      mbar_drain(&sm->drain, 0);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ q by TMA
+    if (lane == 0 && T > 0) {
+      mbar_arrive_expect_tx(&sm->q_full, static_cast<uint32_t>(npanels) * kAttnPanelQ);
+      const int qrow = static_cast<int>((row * p.slices + slice) * kAttnHeads);
+      for (int pn = 0; pn < npanels; ++pn)
+        tma_load_2d(q_buf + pn * kAttnPanelQ, &qmap, &sm->q_full, feat0 + 64 * pn, qrow);
+      mbar_drain(&sm->q_full, 0);                       // never leave with the copy in flight
+    }
+  } else if (warp < kAttnSoftBase / 32) {
+    // ------------------------------------------------------------ key gather
+    const int g = tid - kAttnGatherBase;               // 0..127
+    const uint16_t* kvb = p.kv + static_cast<int64_t>(b) * p.L * kAttnDqk + feat0;
+    const int total = kAttnTileN * chunks_per_key;
+    bool ok = true;
+    for (int i = 0; i < T; ++i) {
+      const int st = i & 1;
+      if (!(ok = mbar_wait(&sm->kv_empty[st], static_cast<uint32_t>(((i >> 1) & 1) ^ 1), abort_flag))) break;
+      const uint32_t stage = smem_u32(kv_buf + st * kAttnStage);
+      for (int c = g; c < total; c += 128) {
+        const int r = c / chunks_per_key, ch = c - r * chunks_per_key;
+        const int e = i * kAttnTileN + r;
+        const int s = sidx[e < n_valid ? e : 0];        // past the last position: any valid row, masked later
+        const int pn = ch >> 3, j = ch & 7;
+        cp_async16(stage + pn * kAttnPanelK + r * 128 + ((j ^ (r & 7)) << 4),
+                   kvb + static_cast<int64_t>(s) * kAttnDqk + pn * 64 + j * 8);
+      }
+      cp_async_commit();
+      if (i >= 1) {
+        cp_async_wait<1>();
+        fence_proxy_async_smem();
+        mbar_arrive(&sm->kv_full[(i - 1) & 1]);
+      }
+    }
+    cp_async_wait<0>();
+    if (ok && T > 0) {
+      fence_proxy_async_smem();
+      mbar_arrive(&sm->kv_full[(T - 1) & 1]);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const int h = quarter * 32 + lane;                 // head row = TMEM lane
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    float* xrow = x_buf + h * kAttnTileN;
+    const uint32_t peer_x = peer_addr(xrow, peer);
+    const uint32_t peer_x_full = peer_addr(&sm->x_full, peer);
+    const uint32_t peer_x_free = peer_addr(&sm->x_free, peer);
+    uint8_t* prow = p_buf + h * 128;
+    float m = -__int_as_float(0x7f800000), l = 0.f;
+    bool ok = true;
+    for (int i = 0; ok && i < T; ++i) {
+      const int st = i & 1;
+      if (!(ok = mbar_wait(&sm->s_full[st], static_cast<uint32_t>((i >> 1) & 1), abort_flag))) break;
+      tc_fence_after();
+      float s[64];
+      {
+        uint32_t v[32];
+        tmem_ld32(t_lane + kAttnTmemS + st * kAttnTileN, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
+        tmem_ld32(t_lane + kAttnTmemS + st * kAttnTileN + 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s[32 + j] = __uint_as_float(v[j]);
+      }
+      tc_fence_before();
+      mbar_arrive(&sm->s_empty[st]);
+      // exchange the partial logits with the peer: it may write my buffer again
+      // once I have read it, and I may write its buffer once it has read its own
+      if (i >= 1 && !(ok = mbar_wait_cluster(&sm->x_free, static_cast<uint32_t>((i - 1) & 1), abort_flag))) break;
+#pragma unroll
+      for (int j = 0; j < 64; j += 4) st_cluster_v4(peer_x + j * 4, s[j], s[j + 1], s[j + 2], s[j + 3]);
+      mbar_arrive_remote(peer_x_full);
+      if (!(ok = mbar_wait_cluster(&sm->x_full, static_cast<uint32_t>(i & 1), abort_flag))) break;
+      const float4* x4 = reinterpret_cast<const float4*>(xrow);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float4 v = x4[j];
+        s[4 * j + 0] += v.x; s[4 * j + 1] += v.y; s[4 * j + 2] += v.z; s[4 * j + 3] += v.w;
+      }
+      mbar_arrive_remote(peer_x_free);
+      // online softmax in the log2 domain
+      const int nk = min(kAttnTileN, n_valid - i * kAttnTileN);
+      float mx = m;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        s[j] = j < nk ? s[j] * p.scale_log2 : -__int_as_float(0x7f800000);
+        mx = fmaxf(mx, s[j]);
+      }
+      const float corr = (i == 0) ? 0.f : exp2f(m - mx);
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        s[j] = j < nk ? exp2f(s[j] - mx) : 0.f;
+        sum += s[j];
+      }
+      l = l * corr + sum;
+      m = mx;
+      // P and O belong to the previous tile's PV until it completes
+      if (i >= 1) {
+        if (!(ok = mbar_wait(&sm->pv_done, static_cast<uint32_t>((i - 1) & 1), abort_flag))) break;
+        tc_fence_after();
+        if (corr != 1.f) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < 256; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(t_lane + kAttnTmemO + c0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * corr);
+            tmem_st32(t_lane + kAttnTmemO + c0, v);
+          }
+          tmem_wait_st();
+        }
+      }
+      // P row (64 keys, bf16) in the 128-byte-swizzled K-major layout
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 v;
+        v.x = pack_bf16x2(s[8 * c + 0], s[8 * c + 1]);
+        v.y = pack_bf16x2(s[8 * c + 2], s[8 * c + 3]);
+        v.z = pack_bf16x2(s[8 * c + 4], s[8 * c + 5]);
+        v.w = pack_bf16x2(s[8 * c + 6], s[8 * c + 7]);
+        *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sm->p_full);
+    }
+    // ---- epilogue: O / l in bf16, and lse
+    const int64_t orow = (row * p.slices + slice) * kAttnHeads + h;
+    uint16_t* od = p.o + orow * kAttnDv + rank * 256;
+    const bool have = ok && T > 0 && mbar_wait(&sm->pv_done, static_cast<uint32_t>((T - 1) & 1), abort_flag);
+    if (have) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(t_lane + kAttnTmemO + c0, v);
+        tmem_wait_ld();
+        uint4* dst = reinterpret_cast<uint4*>(od + c0);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(v[8 * q4 + 0]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv);
+          dst[q4] = w;
+        }
+      }
+    } else if (T == 0) {
+      uint4* dst = reinterpret_cast<uint4*>(od);
+      for (int q4 = 0; q4 < 32; ++q4) dst[q4] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (rank == 0 && (have || T == 0))
+      p.lse[orow] = T == 0 ? -__int_as_float(0x7f800000) : (m + log2f(l)) * 0.69314718055994531f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                      // no CTA leaves while its peer may still write to it
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace hisa
