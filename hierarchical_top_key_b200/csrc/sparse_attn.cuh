@@ -33,7 +33,8 @@
 //   warp 0      TMEM owner, single-thread MMA issuer (QK of tile i, then
 //               PV of tile i-1)
 //   warp 1      q tile by TMA (once per query)
-//   warps 2..5  key gather (cp.async), two stages
+//   warps 2..5  key gather (cp.async): two groups of 64 threads, one per
+//               stage, each signalling its tile as soon as it has landed
 //   warps 6..9  softmax: thread = head row; exchange, online softmax, O
 //               rescaling in TMEM, P (bf16) to shared memory, epilogue
 // Every wait is bounded; a timeout sets the CTA's abort flag and the status
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
   if (tid == 0) {
     mbar_init(&sm->q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm->kv_full[i], 128);
+      mbar_init(&sm->kv_full[i], 64);
       mbar_init(&sm->kv_empty[i], 1);
       mbar_init(&sm->s_full[i], 1);
       mbar_init(&sm->s_empty[i], 128);
@@ -360,15 +361,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     }
   } else if (warp < kAttnSoftBase / 32) {
     // ------------------------------------------------------------ key gather
+    // two groups of 64 threads, one per stage: group g gathers the tiles
+    // i = g, g+2, ... and signals each as soon as its own copies have landed,
+    // so a tile never waits for the issue of a later one
     const int g = tid - kAttnGatherBase;               // 0..127
+    const int grp = g >> 6, gt = g & 63;
     const uint16_t* kvb = p.kv + static_cast<int64_t>(b) * p.L * kAttnDqk + feat0;
     const int total = kAttnTileN * chunks_per_key;
-    bool ok = true;
-    for (int i = 0; i < T; ++i) {
-      const int st = i & 1;
-      if (!(ok = mbar_wait(&sm->kv_empty[st], static_cast<uint32_t>(((i >> 1) & 1) ^ 1), abort_flag))) break;
-      const uint32_t stage = smem_u32(kv_buf + st * kAttnStage);
-      for (int c = g; c < total; c += 128) {
+    const uint32_t stage = smem_u32(kv_buf + grp * kAttnStage);
+    for (int i = grp; i < T; i += 2) {
+      if (!mbar_wait(&sm->kv_empty[grp], static_cast<uint32_t>(((i >> 1) & 1) ^ 1), abort_flag)) break;
+      for (int c = gt; c < total; c += 64) {
         const int r = c / chunks_per_key, ch = c - r * chunks_per_key;
         const int e = i * kAttnTileN + r;
         const int s = sidx[e < n_valid ? e : 0];        // past the last position: any valid row, masked later
@@ -377,17 +380,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
                    kvb + static_cast<int64_t>(s) * kAttnDqk + pn * 64 + j * 8);
       }
       cp_async_commit();
-      if (i >= 1) {
-        cp_async_wait<1>();
-        fence_proxy_async_smem();
-        mbar_arrive(&sm->kv_full[(i - 1) & 1]);
-      }
+      cp_async_wait<0>();
+      fence_proxy_async_smem();                        // the copies are generic-proxy writes the MMA reads
+      mbar_arrive(&sm->kv_full[grp]);
     }
     cp_async_wait<0>();
-    if (ok && T > 0) {
-      fence_proxy_async_smem();
-      mbar_arrive(&sm->kv_full[(T - 1) & 1]);
-    }
   } else {
     // ------------------------------------------------------------ softmax
     const int quarter = warp & 3;
