@@ -59,6 +59,7 @@ constexpr uint32_t kAttnPanelK = kAttnTileN * 128;     // bytes of one key panel
 constexpr uint32_t kAttnStage = kAttnPanels * kAttnPanelK;
 constexpr uint32_t kAttnTmemS = 0;         // two 64-column logit buffers
 constexpr uint32_t kAttnTmemO = 256;       // 256 output columns
+constexpr unsigned kFull = 0xffffffffu;
 
 struct AttnParams {
   int64_t rows;              // batch * Q
@@ -399,7 +400,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     bool ok = true;
     for (int i = 0; ok && i < T; ++i) {
       const int st = i & 1;
-      if (!(ok = mbar_wait(&sm->s_full[st], static_cast<uint32_t>((i >> 1) & 1), abort_flag))) break;
+      // every wait below is taken by all lanes and its outcome made warp-uniform:
+      // the tcgen05 loads and stores that follow are .sync.aligned
+      if (!(ok = __all_sync(kFull, mbar_wait(&sm->s_full[st], static_cast<uint32_t>((i >> 1) & 1), abort_flag))))
+        break;
       tc_fence_after();
       float s[64];
       {
@@ -417,11 +421,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       mbar_arrive(&sm->s_empty[st]);
       // exchange the partial logits with the peer: it may write my buffer again
       // once I have read it, and I may write its buffer once it has read its own
-      if (i >= 1 && !(ok = mbar_wait_cluster(&sm->x_free, static_cast<uint32_t>((i - 1) & 1), abort_flag))) break;
+      if (i >= 1 &&
+          !(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_free, static_cast<uint32_t>((i - 1) & 1), abort_flag))))
+        break;
 #pragma unroll
       for (int j = 0; j < 64; j += 4) st_cluster_v4(peer_x + j * 4, s[j], s[j + 1], s[j + 2], s[j + 3]);
       mbar_arrive_remote(peer_x_full);
-      if (!(ok = mbar_wait_cluster(&sm->x_full, static_cast<uint32_t>(i & 1), abort_flag))) break;
+      if (!(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_full, static_cast<uint32_t>(i & 1), abort_flag)))) break;
       const float4* x4 = reinterpret_cast<const float4*>(xrow);
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -448,9 +454,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       m = mx;
       // P and O belong to the previous tile's PV until it completes
       if (i >= 1) {
-        if (!(ok = mbar_wait(&sm->pv_done, static_cast<uint32_t>((i - 1) & 1), abort_flag))) break;
+        if (!(ok = __all_sync(kFull, mbar_wait(&sm->pv_done, static_cast<uint32_t>((i - 1) & 1), abort_flag))))
+          break;
         tc_fence_after();
-        if (corr != 1.f) {
+        if (__any_sync(kFull, corr != 1.f)) {          // rows whose maximum did not grow scale by 1
 #pragma unroll 1
           for (int c0 = 0; c0 < 256; c0 += 32) {
             uint32_t v[32];
@@ -480,7 +487,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     // ---- epilogue: O / l in bf16, and lse
     const int64_t orow = (row * p.slices + slice) * kAttnHeads + h;
     uint16_t* od = p.o + orow * kAttnDv + rank * 256;
-    const bool have = ok && T > 0 && mbar_wait(&sm->pv_done, static_cast<uint32_t>((T - 1) & 1), abort_flag);
+    const bool have =
+        __all_sync(kFull, ok && T > 0 && mbar_wait(&sm->pv_done, static_cast<uint32_t>((T - 1) & 1), abort_flag));
     if (have) {
       tc_fence_after();
       const float inv = 1.f / l;
