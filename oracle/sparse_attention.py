@@ -20,19 +20,23 @@ one: softmax attention of each query head over the selected keys only,
 with one key and one value row per position shared by all heads (latent
 attention keeps one compressed KV row per token for every head; a value row
 may be a prefix of the key row).  The selected set is the index row with -1
-entries and repeats removed: the indexer returns a set.  An empty set gives
-o = 0 and lse = -inf.  Everything is float64.
+entries, entries that name no key (outside 0..L-1) and repeats removed: the
+indexer returns a set of key positions.  An empty set gives o = 0 and
+lse = -inf.  Everything is float64.
 """
 from __future__ import annotations
 
 import numpy as np
 
 
-def selected_positions(idx_row) -> np.ndarray:
-    """The set a row of indexer output denotes: -1 padding dropped, repeats
-    counted once, ascending."""
+def selected_positions(idx_row, num_keys=None) -> np.ndarray:
+    """The set a row of indexer output denotes: -1 padding (and, given the key
+    count, entries at or past it) dropped, repeats counted once, ascending."""
     r = np.asarray(idx_row, np.int64)
-    return np.unique(r[r >= 0])
+    keep = r >= 0
+    if num_keys is not None:
+        keep &= r < num_keys
+    return np.unique(r[keep])
 
 
 def sparse_attention_query(q_t: np.ndarray, keys: np.ndarray, values: np.ndarray, idx_row,
@@ -40,7 +44,7 @@ def sparse_attention_query(q_t: np.ndarray, keys: np.ndarray, values: np.ndarray
     """One query: q_t [H, dk], keys [L, dk], values [L, dv], idx_row [k] int.
     Returns (o [H, dv], lse [H])."""
     q_t = np.asarray(q_t, np.float64)
-    s = selected_positions(idx_row)
+    s = selected_positions(idx_row, np.asarray(keys).shape[0])
     H = q_t.shape[0]
     dv = values.shape[1]
     if s.size == 0:

@@ -466,9 +466,9 @@ def pin_sparse_attention_brute_force():
     """Tiny inputs by explicit loops over a Python set of positions."""
     import math
     q, k, v, scale = _attn_case()
-    for row in ([4], [0, 3, 8], [8, -1, 2, 2, -1, 5], [-1, -1], list(range(9))):
+    for row in ([4], [0, 3, 8], [8, -1, 2, 2, -1, 5], [-1, -1], list(range(9)), [9, 2, 40, -1, 8, 9]):
         o, lse = sa.sparse_attention_query(q, k, v, row, scale)
-        sel = sorted({i for i in row if i >= 0})
+        sel = sorted({i for i in row if 0 <= i < k.shape[0]})
         for h in range(q.shape[0]):
             if not sel:
                 assert lse[h] == -math.inf and not np.any(o[h])

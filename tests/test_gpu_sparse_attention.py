@@ -23,7 +23,7 @@ def _check(q, kv, idx, o, lse, rows, what):
     """q [Q, H, dqk], kv [L, dqk] (float32 holding bf16), idx [Q, k]; o, lse from the GPU."""
     for t in rows:
         ro, rl = sa.sparse_attention_query(q[t], kv, kv[:, :synthetic.ATTN_DV], idx[t], synthetic.ATTN_SCALE)
-        sel = sa.selected_positions(idx[t])
+        sel = sa.selected_positions(idx[t], kv.shape[0])
         if sel.size == 0:
             assert np.all(o[t] == 0) and np.all(np.isneginf(lse[t])), f"{what} query {t}: empty set"
             continue

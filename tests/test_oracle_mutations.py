@@ -83,13 +83,18 @@ def _second_level_unforced(q_t, w_t, kpool, cands, c_t, top_m):
     return np.sort(cands[ho.top_by_score(s, top_m)]).astype(np.int64)
 
 
-def _padding_as_position(idx_row):
+def _padding_as_position(idx_row, num_keys=None):
     return np.unique(np.asarray(idx_row, np.int64))          # -1 reads the last key
 
 
-def _repeats_counted(idx_row):
+def _out_of_range_kept(idx_row, num_keys=None):
     r = np.asarray(idx_row, np.int64)
-    return np.sort(r[r >= 0])                                 # a repeated index weighs twice
+    return np.unique(r[r >= 0])                               # entries past the keys are not dropped
+
+
+def _repeats_counted(idx_row, num_keys=None):
+    r = np.asarray(idx_row, np.int64)
+    return np.sort(r[(r >= 0) & (r < (num_keys if num_keys is not None else np.iinfo(np.int64).max))])                                 # a repeated index weighs twice
 
 
 _orig_attn = sa.sparse_attention_query
@@ -173,6 +178,7 @@ MUTATIONS = {
     "e4m3_q_scale_per_head": [(ho, "quantize_q_tokens", _q_scale_per_head)],
     "attention_padding_as_position": [(sa, "selected_positions", _padding_as_position)],
     "attention_repeats_counted": [(sa, "selected_positions", _repeats_counted)],
+    "attention_out_of_range_kept": [(sa, "selected_positions", _out_of_range_kept)],
     "attention_softmax_over_heads": [(sa, "sparse_attention_query", _softmax_over_heads)],
     "attention_scale_dropped": [(sa, "sparse_attention_query", _scale_dropped)],
     "attention_lse_without_max": [(sa, "sparse_attention_query", _lse_without_max)],
