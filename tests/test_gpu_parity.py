@@ -186,7 +186,8 @@ def _check_workload(inp, fp8, queries_per_seq, seqs=None):
 def test_small_parity(lib, name):
     inp = _inputs((name, tuple(sorted(SMALL[name].items()))))
     stats = _check_workload(inp, fp8=False, queries_per_seq=120)
-    if SMALL[name].get("w_low", 0.0) < 0:
+    if SMALL[name].get("w_low", 0.0) < 0 and SMALL[name].get("first_query_pos", 0) == 0:
+        # early causal queries see fewer keys than k, so some selected scores are negative
         assert stats["negative_scores"] > 0, "signed weights should give some negative selected scores"
 
 
