@@ -1029,8 +1029,12 @@ hisa_status hisa_sparse_attention(const void* q, const void* kv, const int32_t* 
   const int64_t rows = static_cast<int64_t>(batch) * num_queries;
   const int slices = heads / kAttnHeads;
   if (rows * slices * 2 > INT32_MAX) return fail(HISA_ERR_UNSUPPORTED, "too many (query, head slice) pairs");
-  CUtensorMap qm;
+  if (static_cast<int64_t>(batch) * num_keys > INT32_MAX)
+    return fail(HISA_ERR_UNSUPPORTED, "batch * num_keys must fit in int32 (key row coordinates)");
+  CUtensorMap qm, kvm;
   hisa_status e = tensor_map_2d(&qm, q, HISA_BF16, static_cast<uint64_t>(rows) * heads, kAttnDqk, kAttnHeads);
+  if (e != HISA_OK) return e;
+  e = tensor_map_2d(&kvm, kv, HISA_BF16, static_cast<uint64_t>(batch) * num_keys, kAttnDqk, 1);
   if (e != HISA_OK) return e;
   const size_t smem = attn_smem_bytes();
   e = cuda_check(cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1052,7 +1056,7 @@ hisa_status hisa_sparse_attention(const void* q, const void* kv, const int32_t* 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cuda_check(cudaLaunchKernelEx(&cfg, sparse_attn_kernel, qm, p), "launch sparse_attn_kernel");
+  e = cuda_check(cudaLaunchKernelEx(&cfg, sparse_attn_kernel, qm, kvm, p), "launch sparse_attn_kernel");
   if (e != HISA_OK) return e;
   return launch_check("sparse_attn_kernel");
 }

@@ -25,17 +25,17 @@
 // same in both CTAs: fp32 addition commutes), and both run the same online
 // softmax, so each can accumulate its half of the output, O_c += P . V_c,
 // with V_c the value columns it already holds (B operand read MN-major from
-// the key tile).  Keys are gathered from their positions with 16-byte
-// cp.async copies written straight into the 128-byte-swizzled layout the MMA
-// reads.
+// the key tile).  Keys are gathered from their positions by the TMA engine,
+// four rows per instruction (tile::gather4 over a one-row box), straight into
+// the 128-byte-swizzled layout the MMA reads.
 //
-// Warp roles (10 warps):
+// Warp roles (8 warps):
 //   warp 0      TMEM owner, single-thread MMA issuer (QK of tile i, then
 //               PV of tile i-1)
 //   warp 1      q tile by TMA (once per query)
-//   warps 2..5  key gather (cp.async): two groups of 64 threads, one per
-//               stage, each signalling its tile as soon as it has landed
-//   warps 6..9  softmax: thread = head row; exchange, online softmax, O
+//   warps 2, 3  key gather by TMA, one warp per key stage (tiles i = 2,
+//               4, ... and 1, 3, ...), each tile completing on its barrier
+//   warps 4..7  softmax: thread = head row; exchange, online softmax, O
 //               rescaling in TMEM, P (bf16) to shared memory, epilogue
 // Every wait is bounded; a timeout sets the CTA's abort flag and the status
 // word, and the peer CTA's waits on it then time out too.
@@ -50,9 +50,9 @@ constexpr int kAttnDqk = 576;
 constexpr int kAttnDv = 512;
 constexpr int kAttnTileN = 64;             // keys per tile
 constexpr int kAttnMaxK = 4096;            // longest index row
-constexpr int kAttnThreads = 320;
-constexpr int kAttnGatherBase = 64;        // warps 2..5
-constexpr int kAttnSoftBase = 192;         // warps 6..9
+constexpr int kAttnThreads = 256;
+constexpr int kAttnGatherBase = 64;        // warps 2, 3
+constexpr int kAttnSoftBase = 128;         // warps 4..7
 constexpr int kAttnPanels = 5;             // 64-feature panels of the larger half
 constexpr uint32_t kAttnPanelQ = kAttnHeads * 128;     // bytes of one q panel (128 rows x 128 B)
 constexpr uint32_t kAttnPanelK = kAttnTileN * 128;     // bytes of one key panel (64 rows x 128 B)
@@ -134,12 +134,16 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// Four rows (y0..y3) of a tensor map whose box is one row high, placed in
+// shared memory as four consecutive box rows; completion counted on `bar`.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int x, int y0,
+                                            int y1, int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
+      : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (the tensor core reads its operands through it).
@@ -210,6 +214,7 @@ inline size_t attn_smem_bytes() {
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                     const __grid_constant__ CUtensorMap kvmap,
                                                                      const AttnParams p) {
   using namespace sm100;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -236,7 +241,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
   if (tid == 0) {
     mbar_init(&sm->q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm->kv_full[i], 64);
+      mbar_init(&sm->kv_full[i], 1);
       mbar_init(&sm->kv_empty[i], 1);
       mbar_init(&sm->s_full[i], 1);
       mbar_init(&sm->s_empty[i], 128);
@@ -250,7 +255,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     fence_barrier_init();
   }
   if (warp == 0) tmem_alloc(&sm->tmem_base, 512);
-  if (warp == 1 && lane == 0) tma_prefetch_desc(&qmap);
+  if (warp == 1 && lane == 0) { tma_prefetch_desc(&qmap); tma_prefetch_desc(&kvmap); }
 
   // ---- the query's positions: sorted, -1 / out-of-range / repeats dropped, compacted
   const int K = p.top_k;
@@ -362,30 +367,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     }
   } else if (warp < kAttnSoftBase / 32) {
     // ------------------------------------------------------------ key gather
-    // two groups of 64 threads, one per stage: group g gathers the tiles
-    // i = g, g+2, ... and signals each as soon as its own copies have landed,
-    // so a tile never waits for the issue of a later one
-    const int g = tid - kAttnGatherBase;               // 0..127
-    const int grp = g >> 6, gt = g & 63;
-    const uint16_t* kvb = p.kv + static_cast<int64_t>(b) * p.L * kAttnDqk + feat0;
-    const int total = kAttnTileN * chunks_per_key;
-    const uint32_t stage = smem_u32(kv_buf + grp * kAttnStage);
+    // warp 2 fills stage 0 with tiles 0, 2, ..., warp 3 stage 1 with tiles
+    // 1, 3, ...: per tile, 16 groups of four key rows x this CTA's panels,
+    // one gather4 each, spread over the lanes
+    const int grp = warp - kAttnGatherBase / 32;
+    const int kbase = b * p.L;
+    uint8_t* stage = kv_buf + grp * kAttnStage;
+    const uint32_t tile_bytes = static_cast<uint32_t>(npanels) * kAttnPanelK;
+    bool ok = true;
+    int issued = 0;
     for (int i = grp; i < T; i += 2) {
-      if (!mbar_wait(&sm->kv_empty[grp], static_cast<uint32_t>(((i >> 1) & 1) ^ 1), abort_flag)) break;
-      for (int c = gt; c < total; c += 64) {
-        const int r = c / chunks_per_key, ch = c - r * chunks_per_key;
-        const int e = i * kAttnTileN + r;
-        const int s = sidx[e < n_valid ? e : 0];        // past the last position: any valid row, masked later
-        const int pn = ch >> 3, j = ch & 7;
-        cp_async16(stage + pn * kAttnPanelK + r * 128 + ((j ^ (r & 7)) << 4),
-                   kvb + static_cast<int64_t>(s) * kAttnDqk + pn * 64 + j * 8);
+      int okl = 1;
+      if (lane == 0) okl = mbar_wait(&sm->kv_empty[grp], static_cast<uint32_t>(((i >> 1) & 1) ^ 1), abort_flag);
+      if (!(ok = __shfl_sync(kFull, okl, 0) != 0)) break;
+      if (lane == 0) mbar_arrive_expect_tx(&sm->kv_full[grp], tile_bytes);
+      __syncwarp();
+      for (int x = lane; x < 16 * npanels; x += 32) {
+        const int g4 = x & 15, pn = x >> 4;
+        int y[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = i * kAttnTileN + 4 * g4 + u;
+          y[u] = kbase + sidx[e < n_valid ? e : 0];       // past the last position: any valid row, masked later
+        }
+        tma_gather4(smem_u32(stage + pn * kAttnPanelK + g4 * 4 * 128), &kvmap, &sm->kv_full[grp],
+                    feat0 + 64 * pn, y[0], y[1], y[2], y[3]);
       }
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async_smem();                        // the copies are generic-proxy writes the MMA reads
-      mbar_arrive(&sm->kv_full[grp]);
+      ++issued;
     }
-    cp_async_wait<0>();
+    if (lane == 0 && issued > 0) {
+      // leave only once this warp's last tile has landed
+      const int last = grp + 2 * (issued - 1);
+      mbar_drain(&sm->kv_full[grp], static_cast<uint32_t>((last >> 1) & 1));
+    }
   } else {
     // ------------------------------------------------------------ softmax
     const int quarter = warp & 3;
