@@ -97,11 +97,6 @@ __device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
   return r;
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
 // Arrive on an mbarrier of another CTA of the cluster, ordering this
 // thread's earlier shared::cluster stores before it.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t addr) {
@@ -143,6 +138,14 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
       : "memory");
+}
+
+// 16 bytes into another CTA's shared memory, counted as complete_tx bytes on
+// that CTA's mbarrier `remote_bar` when they land (both cluster addresses).
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+               : "memory");
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
@@ -196,6 +199,7 @@ struct AttnSmem {
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full, pv_done;
   uint64_t x_full, x_free;       // exchange of partial logits with the peer CTA
+  uint64_t x_read;               // every softmax thread has read its row of the peer's logits
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -248,8 +252,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     }
     mbar_init(&sm->p_full, 128);
     mbar_init(&sm->pv_done, 1);
-    mbar_init(&sm->x_full, 128);
-    mbar_init(&sm->x_free, 128);
+    mbar_init(&sm->x_full, 1);      // local arrive with the tile's byte count + the peer's st.async bytes
+    mbar_init(&sm->x_free, 1);      // one remote arrive from the peer
+    mbar_init(&sm->x_read, 128);
     mbar_init(&sm->drain, 1);
     sm->abort_flag = 0;
     fence_barrier_init();
@@ -433,22 +438,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       }
       tc_fence_before();
       mbar_arrive(&sm->s_empty[st]);
-      // exchange the partial logits with the peer: it may write my buffer again
-      // once I have read it, and I may write its buffer once it has read its own
+      // exchange the partial logits with the peer.  Each thread's 64 values go
+      // to its row of the peer's buffer as 16-byte st.async pieces that count
+      // themselves on the peer's x_full (which expects one tile of bytes from
+      // a local arrive); the peer may write my buffer again once all my
+      // threads have read it (one remote arrive on its x_free).  Rows are
+      // swizzled by 16-byte piece (piece c at c ^ (h & 7)), so a warp's
+      // accesses to 32 rows spread over every bank.
+      if (h == 0) mbar_arrive_expect_tx(&sm->x_full, kAttnHeads * kAttnTileN * 4);
       if (i >= 1 &&
           !(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_free, static_cast<uint32_t>((i - 1) & 1), abort_flag))))
         break;
 #pragma unroll
-      for (int j = 0; j < 64; j += 4) st_cluster_v4(peer_x + j * 4, s[j], s[j + 1], s[j + 2], s[j + 3]);
-      mbar_arrive_remote(peer_x_full);
+      for (int c = 0; c < 16; ++c)
+        st_async_v4(peer_x + ((c ^ (h & 7)) << 4), s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3], peer_x_full);
       if (!(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_full, static_cast<uint32_t>(i & 1), abort_flag)))) break;
       const float4* x4 = reinterpret_cast<const float4*>(xrow);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float4 v = x4[j];
-        s[4 * j + 0] += v.x; s[4 * j + 1] += v.y; s[4 * j + 2] += v.z; s[4 * j + 3] += v.w;
+      for (int c = 0; c < 16; ++c) {
+        const float4 v = x4[c ^ (h & 7)];
+        s[4 * c + 0] += v.x; s[4 * c + 1] += v.y; s[4 * c + 2] += v.z; s[4 * c + 3] += v.w;
       }
-      mbar_arrive_remote(peer_x_free);
+      mbar_arrive(&sm->x_read);                        // this row of my buffer has been read
+      if (h == 0) {
+        if (!mbar_wait(&sm->x_read, static_cast<uint32_t>(i & 1), abort_flag)) ok = false;
+        else mbar_arrive_remote(peer_x_free);
+      }
+      if (!(ok = __all_sync(kFull, ok))) break;
       // online softmax in the log2 domain
       const int nk = min(kAttnTileN, n_valid - i * kAttnTileN);
       float mx = m;
