@@ -29,13 +29,14 @@
 // four rows per instruction (tile::gather4 over a one-row box), straight into
 // the 128-byte-swizzled layout the MMA reads.
 //
-// Warp roles (8 warps):
+// Warp roles (10 warps):
 //   warp 0      TMEM owner, single-thread MMA issuer (QK of tile i, then
 //               PV of tile i-1)
 //   warp 1      q tile by TMA (once per query)
-//   warps 2, 3  key gather by TMA, one warp per key stage (tiles i = 2,
-//               4, ... and 1, 3, ...), each tile completing on its barrier
-//   warps 4..7  softmax: thread = head row; exchange, online softmax, O
+//   warps 2..5  key gather by TMA, two warps per key stage (stage 0: tiles
+//               0, 2, ...; stage 1: tiles 1, 3, ...), each tile completing on
+//               its stage's barrier
+//   warps 6..9  softmax: thread = head row; exchange, online softmax, O
 //               rescaling in TMEM, P (bf16) to shared memory, epilogue
 // Every wait is bounded; a timeout sets the CTA's abort flag and the status
 // word, and the peer CTA's waits on it then time out too.
@@ -50,9 +51,9 @@ constexpr int kAttnDqk = 576;
 constexpr int kAttnDv = 512;
 constexpr int kAttnTileN = 64;             // keys per tile
 constexpr int kAttnMaxK = 4096;            // longest index row
-constexpr int kAttnThreads = 256;
-constexpr int kAttnGatherBase = 64;        // warps 2, 3
-constexpr int kAttnSoftBase = 128;         // warps 4..7
+constexpr int kAttnThreads = 320;
+constexpr int kAttnGatherBase = 64;        // warps 2..5
+constexpr int kAttnSoftBase = 192;         // warps 6..9
 constexpr int kAttnPanels = 5;             // 64-feature panels of the larger half
 constexpr uint32_t kAttnPanelQ = kAttnHeads * 128;     // bytes of one q panel (128 rows x 128 B)
 constexpr uint32_t kAttnPanelK = kAttnTileN * 128;     // bytes of one key panel (64 rows x 128 B)
@@ -188,6 +189,15 @@ __host__ __device__ constexpr uint32_t instr_desc_bmn(int M, int N) {
 
 }  // namespace sm100
 
+// 2^x by the SFU's approximate base-2 exponential (ex2.approx, a hardware
+// instruction: relative error of a few ulp, 2^-inf = 0); the softmax weights
+// it produces are rounded to bf16 before they are used.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -199,7 +209,6 @@ struct AttnSmem {
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full, pv_done;
   uint64_t x_full, x_free;       // exchange of partial logits with the peer CTA
-  uint64_t x_read;               // every softmax thread has read its row of the peer's logits
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -253,8 +262,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     mbar_init(&sm->p_full, 128);
     mbar_init(&sm->pv_done, 1);
     mbar_init(&sm->x_full, 1);      // local arrive with the tile's byte count + the peer's st.async bytes
-    mbar_init(&sm->x_free, 1);      // one remote arrive from the peer
-    mbar_init(&sm->x_read, 128);
+    mbar_init(&sm->x_free, 4);      // one remote arrive from each of the peer's softmax warps
     mbar_init(&sm->drain, 1);
     sm->abort_flag = 0;
     fence_barrier_init();
@@ -372,10 +380,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     }
   } else if (warp < kAttnSoftBase / 32) {
     // ------------------------------------------------------------ key gather
-    // warp 2 fills stage 0 with tiles 0, 2, ..., warp 3 stage 1 with tiles
-    // 1, 3, ...: per tile, 16 groups of four key rows x this CTA's panels,
-    // one gather4 each, spread over the lanes
-    const int grp = warp - kAttnGatherBase / 32;
+    // warps 2, 3 fill stage 0 with tiles 0, 2, ..., warps 4, 5 stage 1 with
+    // tiles 1, 3, ...: per tile, 16 groups of four key rows x this CTA's
+    // panels, one gather4 each, split between the stage's two warps
+    const int gw = warp - kAttnGatherBase / 32;        // 0..3
+    const int grp = gw >> 1, half = gw & 1;
     const int kbase = b * p.L;
     uint8_t* stage = kv_buf + grp * kAttnStage;
     const uint32_t tile_bytes = static_cast<uint32_t>(npanels) * kAttnPanelK;
@@ -385,9 +394,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       int okl = 1;
       if (lane == 0) okl = mbar_wait(&sm->kv_empty[grp], static_cast<uint32_t>(((i >> 1) & 1) ^ 1), abort_flag);
       if (!(ok = __shfl_sync(kFull, okl, 0) != 0)) break;
-      if (lane == 0) mbar_arrive_expect_tx(&sm->kv_full[grp], tile_bytes);
-      __syncwarp();
-      for (int x = lane; x < 16 * npanels; x += 32) {
+      // one arrive per tile carries the tile's byte count; both warps' copies count against it
+      if (half == 0 && lane == 0) mbar_arrive_expect_tx(&sm->kv_full[grp], tile_bytes);
+      for (int x = half * 32 + lane; x < 16 * npanels; x += 64) {
         const int g4 = x & 15, pn = x >> 4;
         int y[4];
 #pragma unroll
@@ -401,7 +410,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       ++issued;
     }
     if (lane == 0 && issued > 0) {
-      // leave only once this warp's last tile has landed
+      // leave only once the last tile this warp took part in has landed
       const int last = grp + 2 * (issued - 1);
       mbar_drain(&sm->kv_full[grp], static_cast<uint32_t>((last >> 1) & 1));
     }
@@ -459,33 +468,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
         const float4 v = x4[c ^ (h & 7)];
         s[4 * c + 0] += v.x; s[4 * c + 1] += v.y; s[4 * c + 2] += v.z; s[4 * c + 3] += v.w;
       }
-      mbar_arrive(&sm->x_read);                        // this row of my buffer has been read
-      if (h == 0) {
-        if (!mbar_wait(&sm->x_read, static_cast<uint32_t>(i & 1), abort_flag)) ok = false;
-        else mbar_arrive_remote(peer_x_free);
-      }
-      if (!(ok = __all_sync(kFull, ok))) break;
-      // online softmax in the log2 domain
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(peer_x_free);  // this warp's rows of my buffer have been read
+      // online softmax in the log2 domain: logits past the last key are -inf,
+      // whose exp2 is 0; maxima and sums in four independent chains
       const int nk = min(kAttnTileN, n_valid - i * kAttnTileN);
-      float mx = m;
+      float mx4[4] = {m, m, m, m};
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
         s[j] = j < nk ? s[j] * p.scale_log2 : -__int_as_float(0x7f800000);
-        mx = fmaxf(mx, s[j]);
+        mx4[j & 3] = fmaxf(mx4[j & 3], s[j]);
       }
-      const float corr = (i == 0) ? 0.f : exp2f(m - mx);
-      float sum = 0.f;
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      const float corr = (i == 0) ? 0.f : fast_exp2(m - mx);
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
-        s[j] = j < nk ? exp2f(s[j] - mx) : 0.f;
-        sum += s[j];
+        s[j] = fast_exp2(s[j] - mx);
+        sum4[j & 3] += s[j];
       }
+      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l = l * corr + sum;
       m = mx;
       // P and O belong to the previous tile's PV until it completes
+      if (i >= 1 &&
+          !(ok = __all_sync(kFull, mbar_wait(&sm->pv_done, static_cast<uint32_t>((i - 1) & 1), abort_flag))))
+        break;
+      // P row (64 keys, bf16) in the 128-byte-swizzled K-major layout
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 v;
+        v.x = pack_bf16x2(s[8 * c + 0], s[8 * c + 1]);
+        v.y = pack_bf16x2(s[8 * c + 2], s[8 * c + 3]);
+        v.z = pack_bf16x2(s[8 * c + 4], s[8 * c + 5]);
+        v.w = pack_bf16x2(s[8 * c + 6], s[8 * c + 7]);
+        *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) = v;
+      }
       if (i >= 1) {
-        if (!(ok = __all_sync(kFull, mbar_wait(&sm->pv_done, static_cast<uint32_t>((i - 1) & 1), abort_flag))))
-          break;
         tc_fence_after();
         if (__any_sync(kFull, corr != 1.f)) {          // rows whose maximum did not grow scale by 1
 #pragma unroll 1
@@ -499,16 +518,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
           }
           tmem_wait_st();
         }
-      }
-      // P row (64 keys, bf16) in the 128-byte-swizzled K-major layout
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 v;
-        v.x = pack_bf16x2(s[8 * c + 0], s[8 * c + 1]);
-        v.y = pack_bf16x2(s[8 * c + 2], s[8 * c + 3]);
-        v.z = pack_bf16x2(s[8 * c + 4], s[8 * c + 5]);
-        v.w = pack_bf16x2(s[8 * c + 6], s[8 * c + 7]);
-        *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) = v;
       }
       fence_proxy_async_smem();
       tc_fence_before();
