@@ -581,19 +581,13 @@ __device__ bool two_pass_topk_rows(const float* __restrict__ row, int n, uint32_
   for (int i = tid; i < nbins; i += nt) sm.hist[i] = 0;
   if (tid == 0) { *buf_count = 0; sm.n_slots = 0; }
   Grp::sync();
-  // two steps' loads issued before either step's histogram updates: 64
-  // bytes in flight per thread on the DRAM pass
-  for (int p0 = 8 * tid; p0 < n; p0 += 16 * nt) {
-    float v[8], v2[8];
-    uint32_t valid, valid2;
+  for (int p0 = 8 * tid; p0 < n; p0 += 8 * nt) {
+    float v[8];
+    uint32_t valid;
     load8(p0, v, valid);
-    load8(p0 + 8 * nt, v2, valid2);
 #pragma unroll
     for (int u = 0; u < 8; ++u)
       if ((valid >> u) & 1u) atomicAdd(&sm.hist[bin_of(v[u])], 1u);
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if ((valid2 >> u) & 1u) atomicAdd(&sm.hist[bin_of(v2[u])], 1u);
   }
   Grp::sync();
   uint32_t remaining = k;
