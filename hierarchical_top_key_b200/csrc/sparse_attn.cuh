@@ -473,14 +473,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       // online softmax in the log2 domain: logits past the last key are -inf,
       // whose exp2 is 0; maxima and sums in four independent chains
       const int nk = min(kAttnTileN, n_valid - i * kAttnTileN);
-      float mx4[4] = {m, m, m, m};
+      float mx4[4] = {-__int_as_float(0x7f800000), -__int_as_float(0x7f800000), -__int_as_float(0x7f800000),
+                      -__int_as_float(0x7f800000)};
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
         s[j] = j < nk ? s[j] * p.scale_log2 : -__int_as_float(0x7f800000);
         mx4[j & 3] = fmaxf(mx4[j & 3], s[j]);
       }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      const float corr = (i == 0) ? 0.f : fast_exp2(m - mx);
+      // the reference maximum moves only when the tile's maximum exceeds it by
+      // more than 8 (a factor 256): the weights stay below 2^8, the output rows
+      // are rescaled rarely, and o = sum p v / sum p is the same for any
+      // reference (the natural-log lse adds back the reference that was used)
+      const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      const bool move = i == 0 || mt > m + 8.f;
+      const float mx = move ? mt : m;
+      const float corr = (i == 0) ? 0.f : (move ? fast_exp2(m - mx) : 1.f);
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
