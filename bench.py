@@ -57,7 +57,12 @@ EXTRA_WORKLOADS = (("chunk_64k", False), ("chunk_64k", True), ("decode_128k", Fa
 # the same command and workload; see profiles/.  `src` is the hash of the
 # kernel sources it was taken on: when the sources change the figure no longer
 # describes the kernel and the bench reports null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum --clock-control none
+    #     -k regex:token_tc -c 1 python bench.py --steps 1 --warmup 1 --no-flat --no-e2e --no-extra
+    #     --no-cpu-baseline --no-attention   (559,312,640 B read + 241,551,104 B written)
+    "prefill_32k": {"bytes": 800863744, "src": "8e241947f82b6434"},
+}
 KERNEL_SOURCES = ("token_tc.cuh", "sm100.cuh", "select.cuh", "common.cuh")
 
 
