@@ -83,6 +83,9 @@ def parse(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-attention", action="store_true", help="skip the attention over the selected keys")
+    ap.add_argument("--attention-only", type=int, default=0, metavar="Q",
+                    help="time only the attention over the selected keys on Q queries x top_k random positions of "
+                         "the workload's keys (a small case for profilers), print one line and exit")
     ap.add_argument("--superblock-group", type=int, default=0,
                     help="also time the three-level indexer with super-blocks of this many blocks")
     ap.add_argument("--top-m2", type=int, default=8, help="super-blocks kept by the three-level indexer")
@@ -712,10 +715,38 @@ def end_to_end(hb, run, steps, stream, world, dev):
 # ------------------------------------------------------------------ our arm
 
 
+def attention_only(args):
+    """The attention over the selected keys alone: Q queries of 128 heads, top_k
+    distinct random positions per query among the workload's keys (seeded),
+    latent rows drawn on the GPU."""
+    import torch
+    from hierarchical_top_key_b200 import binding as hb
+    wl = synthetic.WORKLOADS[args.workload]
+    Q, L, K = args.attention_only, wl.num_keys, wl.top_k
+    q, kv = synthetic.attention_inputs_cuda(1, Q, L, seed=args.seed)
+    g = torch.Generator(device="cuda").manual_seed(args.seed + 1)
+    idx = torch.argsort(torch.rand((Q, L), generator=g, device="cuda"), dim=1)[:, :K].to(torch.int32)
+    idx = idx.view(1, Q, K).contiguous()
+    fn = lambda: hb.hisa_sparse_attention(q, kv, idx, scale=synthetic.ATTN_SCALE)  # noqa: E731
+    for _ in range(max(1, args.warmup)):
+        fn()
+    torch.cuda.synchronize()
+    hb.get_status()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    ms = timed(fn, max(1, args.steps), flush, torch.cuda.current_stream())
+    hb.get_status()
+    flops = 2.0 * Q * K * q.shape[2] * (synthetic.ATTN_DQK + synthetic.ATTN_DV)
+    print(json.dumps({"attention_only": {"queries": Q, "keys": L, "top_k": K, "ms": ms,
+                                         "tflops": flops / (ms / 1000.0) / 1e12}}))
+    return 0
+
+
 def main(argv=None):
     args = parse(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.attention_only:
+        return attention_only(args)
     import torch
     import torch.distributed as dist
     from hierarchical_top_key_b200 import binding as hb
