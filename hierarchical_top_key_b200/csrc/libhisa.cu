@@ -1031,10 +1031,8 @@ hisa_status hisa_sparse_attention(const void* q, const void* kv, const int32_t* 
   if (rows * slices * 2 > INT32_MAX) return fail(HISA_ERR_UNSUPPORTED, "too many (query, head slice) pairs");
   if (static_cast<int64_t>(batch) * num_keys > INT32_MAX)
     return fail(HISA_ERR_UNSUPPORTED, "batch * num_keys must fit in int32 (key row coordinates)");
-  CUtensorMap qm, kvm;
-  hisa_status e = tensor_map_2d(&qm, q, HISA_BF16, static_cast<uint64_t>(rows) * heads, kAttnDqk, kAttnHeads);
-  if (e != HISA_OK) return e;
-  e = tensor_map_2d(&kvm, kv, HISA_BF16, static_cast<uint64_t>(batch) * num_keys, kAttnDqk, 1);
+  CUtensorMap kvm;
+  hisa_status e = tensor_map_2d(&kvm, kv, HISA_BF16, static_cast<uint64_t>(batch) * num_keys, kAttnDqk, 1);
   if (e != HISA_OK) return e;
   const size_t smem = attn_smem_bytes();
   e = cuda_check(cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1043,7 +1041,7 @@ hisa_status hisa_sparse_attention(const void* q, const void* kv, const int32_t* 
   AttnParams p{};
   p.rows = rows; p.Q = num_queries; p.L = num_keys; p.slices = slices; p.top_k = top_k;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.idx = idx; p.kv = static_cast<const uint16_t*>(kv); p.o = static_cast<uint16_t*>(o); p.lse = lse;
+  p.idx = idx; p.q = static_cast<const uint16_t*>(q); p.kv = static_cast<const uint16_t*>(kv); p.o = static_cast<uint16_t*>(o); p.lse = lse;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(rows * slices * 2));
   cfg.blockDim = dim3(kAttnThreads);
@@ -1056,7 +1054,7 @@ hisa_status hisa_sparse_attention(const void* q, const void* kv, const int32_t* 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cuda_check(cudaLaunchKernelEx(&cfg, sparse_attn_kernel, qm, kvm, p), "launch sparse_attn_kernel");
+  e = cuda_check(cudaLaunchKernelEx(&cfg, sparse_attn_kernel, kvm, p), "launch sparse_attn_kernel");
   if (e != HISA_OK) return e;
   return launch_check("sparse_attn_kernel");
 }

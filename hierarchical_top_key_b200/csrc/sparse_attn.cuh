@@ -19,7 +19,9 @@
 //          the value columns   0..255 of the output
 //   CTA 1  features 256..575: the rest of every logit (with the 64
 //          positional features), the value columns 256..511
-// Each CTA computes a partial logit tile S_c = q_c . k_c^T (M = 128 heads,
+// Each CTA keeps its part of the query in TMEM (the A operand of the logit
+// MMA, loaded once per query), so that shared memory holds four key stages;
+// it computes a partial logit tile S_c = q_c . k_c^T (M = 128 heads,
 // N = 64 keys, K = its features) on tcgen05 into TMEM, the two partial tiles
 // are exchanged through distributed shared memory and summed (the sum is the
 // same in both CTAs: fp32 addition commutes), and both run the same online
@@ -29,15 +31,14 @@
 // four rows per instruction (tile::gather4 over a one-row box), straight into
 // the 128-byte-swizzled layout the MMA reads.
 //
-// Warp roles (10 warps):
+// Warp roles (9 warps):
 //   warp 0      TMEM owner, single-thread MMA issuer (QK of tile i, then
 //               PV of tile i-1)
-//   warp 1      q tile by TMA (once per query)
-//   warps 2..5  key gather by TMA, two warps per key stage (stage 0: tiles
-//               0, 2, ...; stage 1: tiles 1, 3, ...), each tile completing on
-//               its stage's barrier
-//   warps 6..9  softmax: thread = head row; exchange, online softmax, O
-//               rescaling in TMEM, P (bf16) to shared memory, epilogue
+//   warps 1..4  key gather by TMA, one warp per key stage (stage s: tiles
+//               s, s+4, ...), each tile completing on its stage's barrier
+//   warps 5..8  softmax: thread = head row; q into TMEM, exchange, online
+//               softmax, O rescaling in TMEM, P (bf16) to shared memory,
+//               epilogue
 // Every wait is bounded; a timeout sets the CTA's abort flag and the status
 // word, and the peer CTA's waits on it then time out too.
 #pragma once
@@ -51,14 +52,15 @@ constexpr int kAttnDqk = 576;
 constexpr int kAttnDv = 512;
 constexpr int kAttnTileN = 64;             // keys per tile
 constexpr int kAttnMaxK = 4096;            // longest index row
-constexpr int kAttnThreads = 320;
-constexpr int kAttnGatherBase = 64;        // warps 2..5
-constexpr int kAttnSoftBase = 192;         // warps 6..9
+constexpr int kAttnThreads = 288;
+constexpr int kAttnGatherBase = 32;        // warps 1..4
+constexpr int kAttnSoftBase = 160;         // warps 5..8
+constexpr int kAttnStages = 4;             // key stages
 constexpr int kAttnPanels = 5;             // 64-feature panels of the larger half
-constexpr uint32_t kAttnPanelQ = kAttnHeads * 128;     // bytes of one q panel (128 rows x 128 B)
 constexpr uint32_t kAttnPanelK = kAttnTileN * 128;     // bytes of one key panel (64 rows x 128 B)
 constexpr uint32_t kAttnStage = kAttnPanels * kAttnPanelK;
-constexpr uint32_t kAttnTmemS = 0;         // two 64-column logit buffers
+constexpr uint32_t kAttnTmemS = 0;         // one 64-column logit buffer
+constexpr uint32_t kAttnTmemQ = 64;        // the query part: 2 bf16 per column, up to 160 columns
 constexpr uint32_t kAttnTmemO = 256;       // 256 output columns
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -68,6 +70,7 @@ struct AttnParams {
   int top_k;
   float scale_log2;          // softmax scale * log2(e)
   const int32_t* idx;        // [rows, top_k]
+  const uint16_t* q;         // [rows, heads, 576] bf16
   const uint16_t* kv;        // [batch, L, 576] bf16
   uint16_t* o;               // [rows, heads, 512] bf16
   float* lse;                // [rows, heads]
@@ -182,6 +185,17 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr, uint32_t l
   return d;
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T (bf16), issued by one thread: A is M = 128
+// rows in 128 lanes, two consecutive K elements per 32-bit column.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Instruction descriptor with the B operand MN-major (bf16, fp32 accumulate).
 __host__ __device__ constexpr uint32_t instr_desc_bmn(int M, int N) {
   return instr_desc(M, N, 1u) | (1u << 16);
@@ -205,8 +219,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 struct AttnSmem {
   uint64_t q_full;
-  uint64_t kv_full[2], kv_empty[2];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t kv_full[kAttnStages], kv_empty[kAttnStages];
+  uint64_t s_full, s_empty;
   uint64_t p_full, pv_done;
   uint64_t x_full, x_free;       // exchange of partial logits with the peer CTA
   uint64_t drain;
@@ -218,23 +232,20 @@ struct AttnSmem {
 };
 
 inline size_t attn_smem_bytes() {
-  return 1024 + kAttnPanels * kAttnPanelQ      // q
-         + 2 * kAttnStage                      // key tiles
+  return 1024 + kAttnStages * kAttnStage       // key tiles
          + kAttnHeads * 128                    // P (bf16, one 64-key panel)
          + kAttnHeads * kAttnTileN * 4         // partial logits from the peer
          + kAttnMaxK * 4                       // the query's sorted, deduplicated positions
          + sizeof(AttnSmem) + 16;
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __grid_constant__ CUtensorMap qmap,
-                                                                     const __grid_constant__ CUtensorMap kvmap,
+__global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __grid_constant__ CUtensorMap kvmap,
                                                                      const AttnParams p) {
   using namespace sm100;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_buf = smem;
-  uint8_t* kv_buf = q_buf + kAttnPanels * kAttnPanelQ;
-  uint8_t* p_buf = kv_buf + 2 * kAttnStage;
+  uint8_t* kv_buf = smem;
+  uint8_t* p_buf = kv_buf + kAttnStages * kAttnStage;
   float* x_buf = reinterpret_cast<float*>(p_buf + kAttnHeads * 128);
   int32_t* sidx = reinterpret_cast<int32_t*>(x_buf + kAttnHeads * kAttnTileN);
   AttnSmem* sm = reinterpret_cast<AttnSmem*>(sidx + kAttnMaxK);
@@ -252,13 +263,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
   const int chunks_per_key = npanels * 8;                // 16-byte pieces of this CTA's part of a key row
 
   if (tid == 0) {
-    mbar_init(&sm->q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(&sm->q_full, 128);
+    for (int i = 0; i < kAttnStages; ++i) {
       mbar_init(&sm->kv_full[i], 1);
       mbar_init(&sm->kv_empty[i], 1);
-      mbar_init(&sm->s_full[i], 1);
-      mbar_init(&sm->s_empty[i], 128);
     }
+    mbar_init(&sm->s_full, 1);
+    mbar_init(&sm->s_empty, 128);
     mbar_init(&sm->p_full, 128);
     mbar_init(&sm->pv_done, 1);
     mbar_init(&sm->x_full, 1);      // local arrive with the tile's byte count + the peer's st.async bytes
@@ -268,7 +279,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     fence_barrier_init();
   }
   if (warp == 0) tmem_alloc(&sm->tmem_base, 512);
-  if (warp == 1 && lane == 0) { tma_prefetch_desc(&qmap); tma_prefetch_desc(&kvmap); }
+  if (warp == 1 && lane == 0) tma_prefetch_desc(&kvmap);
 
   // ---- the query's positions: sorted, -1 / out-of-range / repeats dropped, compacted
   const int K = p.top_k;
@@ -335,23 +346,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       constexpr uint32_t id_pv = instr_desc_bmn(kAttnHeads, 256);
       bool ok = T == 0 || mbar_wait(&sm->q_full, 0, abort_flag);
       if (ok) tc_fence_after();
-      const uint64_t q_desc = desc_k_sw128(smem_u32(q_buf));
       const uint64_t p_desc = desc_k_sw128(smem_u32(p_buf));
+      const int ksteps = npanels * 4;
       for (int i = 0; ok && i <= T; ++i) {
         if (i < T) {
-          const int st = i & 1;
-          const uint32_t ph = static_cast<uint32_t>((i >> 1) & 1);
-          if (!(ok = mbar_wait(&sm->kv_full[st], ph, abort_flag))) break;
-          if (!(ok = mbar_wait(&sm->s_empty[st], ph ^ 1u, abort_flag))) break;
+          const int st = i % kAttnStages;
+          if (!(ok = mbar_wait(&sm->kv_full[st], static_cast<uint32_t>((i / kAttnStages) & 1), abort_flag))) break;
+          // the single logit buffer is free once the softmax has read tile i-1
+          if (i >= 1 && !(ok = mbar_wait(&sm->s_empty, static_cast<uint32_t>((i - 1) & 1), abort_flag))) break;
           tc_fence_after();
           const uint64_t k_desc = desc_k_sw128(smem_u32(kv_buf + st * kAttnStage));
-          const uint32_t d = tmem + kAttnTmemS + st * kAttnTileN;
-          if (npanels == 4) mma_tile_sw128<DT_BF16, 16, kAttnHeads, kAttnTileN>(d, q_desc, k_desc, id_qk);
-          else mma_tile_sw128<DT_BF16, 20, kAttnHeads, kAttnTileN>(d, q_desc, k_desc, id_qk);
-          mma_commit(&sm->s_full[st]);
+#pragma unroll 4
+          for (int ks = 0; ks < ksteps; ++ks)
+            mma_ts(tmem + kAttnTmemS, tmem + kAttnTmemQ + ks * 8,
+                   k_desc + static_cast<uint64_t>((ks >> 2) * (kAttnTileN * 128 / 16) + (ks & 3) * 2), id_qk,
+                   ks > 0 ? 1u : 0u);
+          mma_commit(&sm->s_full);
         }
         if (i >= 1) {
-          const int j = i - 1, sj = j & 1;
+          const int j = i - 1, sj = j % kAttnStages;
           if (!(ok = mbar_wait(&sm->p_full, static_cast<uint32_t>(j & 1), abort_flag))) break;
           tc_fence_after();
           // V: the first four 64-feature panels of the key tile, MN-major
@@ -369,34 +382,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       mma_commit(&sm->drain);
       mbar_drain(&sm->drain, 0);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ q by TMA
-    if (lane == 0 && T > 0) {
-      mbar_arrive_expect_tx(&sm->q_full, static_cast<uint32_t>(npanels) * kAttnPanelQ);
-      const int qrow = static_cast<int>((row * p.slices + slice) * kAttnHeads);
-      for (int pn = 0; pn < npanels; ++pn)
-        tma_load_2d(q_buf + pn * kAttnPanelQ, &qmap, &sm->q_full, feat0 + 64 * pn, qrow);
-      mbar_drain(&sm->q_full, 0);                       // never leave with the copy in flight
-    }
   } else if (warp < kAttnSoftBase / 32) {
     // ------------------------------------------------------------ key gather
-    // warps 2, 3 fill stage 0 with tiles 0, 2, ..., warps 4, 5 stage 1 with
-    // tiles 1, 3, ...: per tile, 16 groups of four key rows x this CTA's
-    // panels, one gather4 each, split between the stage's two warps
-    const int gw = warp - kAttnGatherBase / 32;        // 0..3
-    const int grp = gw >> 1, half = gw & 1;
+    // warp 1 + s fills stage s with tiles s, s + 4, ...: per tile, 16 groups of
+    // four key rows x this CTA's panels, one gather4 each, spread over the lanes
+    const int grp = warp - kAttnGatherBase / 32;       // stage 0..3
     const int kbase = b * p.L;
     uint8_t* stage = kv_buf + grp * kAttnStage;
     const uint32_t tile_bytes = static_cast<uint32_t>(npanels) * kAttnPanelK;
     bool ok = true;
     int issued = 0;
-    for (int i = grp; i < T; i += 2) {
+    for (int i = grp; i < T; i += kAttnStages) {
       int okl = 1;
-      if (lane == 0) okl = mbar_wait(&sm->kv_empty[grp], static_cast<uint32_t>(((i >> 1) & 1) ^ 1), abort_flag);
+      if (lane == 0)
+        okl = mbar_wait(&sm->kv_empty[grp], static_cast<uint32_t>(((i / kAttnStages) & 1) ^ 1), abort_flag);
       if (!(ok = __shfl_sync(kFull, okl, 0) != 0)) break;
-      // one arrive per tile carries the tile's byte count; both warps' copies count against it
-      if (half == 0 && lane == 0) mbar_arrive_expect_tx(&sm->kv_full[grp], tile_bytes);
-      for (int x = half * 32 + lane; x < 16 * npanels; x += 64) {
+      if (lane == 0) mbar_arrive_expect_tx(&sm->kv_full[grp], tile_bytes);
+      __syncwarp();
+      for (int x = lane; x < 16 * npanels; x += 32) {
         const int g4 = x & 15, pn = x >> 4;
         int y[4];
 #pragma unroll
@@ -410,9 +413,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       ++issued;
     }
     if (lane == 0 && issued > 0) {
-      // leave only once the last tile this warp took part in has landed
-      const int last = grp + 2 * (issued - 1);
-      mbar_drain(&sm->kv_full[grp], static_cast<uint32_t>((last >> 1) & 1));
+      // leave only once this warp's last tile has landed
+      const int last = grp + kAttnStages * (issued - 1);
+      mbar_drain(&sm->kv_full[grp], static_cast<uint32_t>((last / kAttnStages) & 1));
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -426,27 +429,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     uint8_t* prow = p_buf + h * 128;
     float m = -__int_as_float(0x7f800000), l = 0.f;
     bool ok = true;
+    {
+      // this head's part of the query into TMEM, 64 features (32 columns) at a time
+      const uint4* qg = reinterpret_cast<const uint4*>(
+          p.q + ((row * p.slices + slice) * kAttnHeads + h) * static_cast<int64_t>(kAttnDqk) + feat0);
+#pragma unroll 1
+      for (int pn = 0; pn < npanels; ++pn) {
+        uint32_t v[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 x = __ldg(qg + pn * 8 + u);
+          v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
+        }
+        tmem_st32(t_lane + kAttnTmemQ + pn * 32, v);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm->q_full);
+    }
     for (int i = 0; ok && i < T; ++i) {
-      const int st = i & 1;
       // every wait below is taken by all lanes and its outcome made warp-uniform:
       // the tcgen05 loads and stores that follow are .sync.aligned
-      if (!(ok = __all_sync(kFull, mbar_wait(&sm->s_full[st], static_cast<uint32_t>((i >> 1) & 1), abort_flag))))
-        break;
+      if (!(ok = __all_sync(kFull, mbar_wait(&sm->s_full, static_cast<uint32_t>(i & 1), abort_flag)))) break;
       tc_fence_after();
       float s[64];
       {
         uint32_t v[32];
-        tmem_ld32(t_lane + kAttnTmemS + st * kAttnTileN, v);
+        tmem_ld32(t_lane + kAttnTmemS, v);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
-        tmem_ld32(t_lane + kAttnTmemS + st * kAttnTileN + 32, v);
+        tmem_ld32(t_lane + kAttnTmemS + 32, v);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 32; ++j) s[32 + j] = __uint_as_float(v[j]);
       }
       tc_fence_before();
-      mbar_arrive(&sm->s_empty[st]);
+      mbar_arrive(&sm->s_empty);
       // exchange the partial logits with the peer.  Each thread's 64 values go
       // to its row of the peer's buffer as 16-byte st.async pieces that count
       // themselves on the peer's x_full (which expects one tile of bytes from
