@@ -20,10 +20,13 @@
 //   CTA 1  features 256..575: the rest of every logit (with the 64
 //          positional features), the value columns 256..511
 // Each CTA keeps its part of the query in TMEM (the A operand of the logit
-// MMA, loaded once per query), so that shared memory holds four key stages;
+// MMA, loaded once per query) and the softmax weights P there too (the A
+// operand of the output MMA), so that shared memory holds three key stages
+// and two exchange buffers;
 // it computes a partial logit tile S_c = q_c . k_c^T (M = 128 heads,
 // N = 64 keys, K = its features) on tcgen05 into TMEM, the two partial tiles
-// are exchanged through distributed shared memory and summed (the sum is the
+// are exchanged through distributed shared memory (one buffer per tile
+// parity, so no "buffer free" handshake is needed) and summed (the sum is the
 // same in both CTAs: fp32 addition commutes), and both run the same online
 // softmax, so each can accumulate its half of the output, O_c += P . V_c,
 // with V_c the value columns it already holds (B operand read MN-major from
@@ -31,14 +34,13 @@
 // four rows per instruction (tile::gather4 over a one-row box), straight into
 // the 128-byte-swizzled layout the MMA reads.
 //
-// Warp roles (9 warps):
+// Warp roles (8 warps):
 //   warp 0      TMEM owner, single-thread MMA issuer (QK of tile i, then
 //               PV of tile i-1)
-//   warps 1..4  key gather by TMA, one warp per key stage (stage s: tiles
-//               s, s+4, ...), each tile completing on its stage's barrier
-//   warps 5..8  softmax: thread = head row; q into TMEM, exchange, online
-//               softmax, O rescaling in TMEM, P (bf16) to shared memory,
-//               epilogue
+//   warps 1..3  key gather by TMA, one warp per key stage (stage s: tiles
+//               s, s+3, ...), each tile completing on its stage's barrier
+//   warps 4..7  softmax: thread = head row; q into TMEM, exchange, online
+//               softmax, O rescaling and P (bf16) in TMEM, epilogue
 // Every wait is bounded; a timeout sets the CTA's abort flag and the status
 // word, and the peer CTA's waits on it then time out too.
 #pragma once
@@ -52,15 +54,16 @@ constexpr int kAttnDqk = 576;
 constexpr int kAttnDv = 512;
 constexpr int kAttnTileN = 64;             // keys per tile
 constexpr int kAttnMaxK = 4096;            // longest index row
-constexpr int kAttnThreads = 288;
-constexpr int kAttnGatherBase = 32;        // warps 1..4
-constexpr int kAttnSoftBase = 160;         // warps 5..8
-constexpr int kAttnStages = 4;             // key stages
+constexpr int kAttnThreads = 256;
+constexpr int kAttnGatherBase = 32;        // warps 1..3
+constexpr int kAttnSoftBase = 128;         // warps 4..7
+constexpr int kAttnStages = 3;             // key stages
 constexpr int kAttnPanels = 5;             // 64-feature panels of the larger half
 constexpr uint32_t kAttnPanelK = kAttnTileN * 128;     // bytes of one key panel (64 rows x 128 B)
 constexpr uint32_t kAttnStage = kAttnPanels * kAttnPanelK;
 constexpr uint32_t kAttnTmemS = 0;         // one 64-column logit buffer
 constexpr uint32_t kAttnTmemQ = 64;        // the query part: 2 bf16 per column, up to 160 columns
+constexpr uint32_t kAttnTmemP = 224;       // softmax weights of one tile: 64 bf16 = 32 columns
 constexpr uint32_t kAttnTmemO = 256;       // 256 output columns
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -99,12 +102,6 @@ __device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
   return r;
-}
-
-// Arrive on an mbarrier of another CTA of the cluster, ordering this
-// thread's earlier shared::cluster stores before it.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
@@ -150,12 +147,6 @@ __device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, flo
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
                "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
                : "memory");
-}
-
-// Make this thread's generic-proxy shared-memory writes visible to the async
-// proxy (the tensor core reads its operands through it).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // 32 lanes x 32 consecutive 32-bit columns from registers into TMEM.
@@ -222,7 +213,7 @@ struct AttnSmem {
   uint64_t kv_full[kAttnStages], kv_empty[kAttnStages];
   uint64_t s_full, s_empty;
   uint64_t p_full, pv_done;
-  uint64_t x_full, x_free;       // exchange of partial logits with the peer CTA
+  uint64_t x_full[2];            // partial logits of the peer CTA, one buffer per tile parity
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -233,8 +224,7 @@ struct AttnSmem {
 
 inline size_t attn_smem_bytes() {
   return 1024 + kAttnStages * kAttnStage       // key tiles
-         + kAttnHeads * 128                    // P (bf16, one 64-key panel)
-         + kAttnHeads * kAttnTileN * 4         // partial logits from the peer
+         + 2 * kAttnHeads * kAttnTileN * 4     // partial logits from the peer, two buffers
          + kAttnMaxK * 4                       // the query's sorted, deduplicated positions
          + sizeof(AttnSmem) + 16;
 }
@@ -245,9 +235,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* kv_buf = smem;
-  uint8_t* p_buf = kv_buf + kAttnStages * kAttnStage;
-  float* x_buf = reinterpret_cast<float*>(p_buf + kAttnHeads * 128);
-  int32_t* sidx = reinterpret_cast<int32_t*>(x_buf + kAttnHeads * kAttnTileN);
+  float* x_buf = reinterpret_cast<float*>(kv_buf + kAttnStages * kAttnStage);   // [2][128][64]
+  int32_t* sidx = reinterpret_cast<int32_t*>(x_buf + 2 * kAttnHeads * kAttnTileN);
   AttnSmem* sm = reinterpret_cast<AttnSmem*>(sidx + kAttnMaxK);
   volatile int* abort_flag = &sm->abort_flag;
 
@@ -272,8 +261,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     mbar_init(&sm->s_empty, 128);
     mbar_init(&sm->p_full, 128);
     mbar_init(&sm->pv_done, 1);
-    mbar_init(&sm->x_full, 1);      // local arrive with the tile's byte count + the peer's st.async bytes
-    mbar_init(&sm->x_free, 4);      // one remote arrive from each of the peer's softmax warps
+    for (int i = 0; i < 2; ++i)
+      mbar_init(&sm->x_full[i], 1);   // local arrive with the tile's byte count + the peer's st.async bytes
     mbar_init(&sm->drain, 1);
     sm->abort_flag = 0;
     fence_barrier_init();
@@ -346,7 +335,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       constexpr uint32_t id_pv = instr_desc_bmn(kAttnHeads, 256);
       bool ok = T == 0 || mbar_wait(&sm->q_full, 0, abort_flag);
       if (ok) tc_fence_after();
-      const uint64_t p_desc = desc_k_sw128(smem_u32(p_buf));
       const int ksteps = npanels * 4;
       for (int i = 0; ok && i <= T; ++i) {
         if (i < T) {
@@ -372,8 +360,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) {
             const uint64_t vd = desc_mn_sw128(v0 + ks * 16 * 128, kAttnPanelK, 1024);
-            mma<DT_BF16>(tmem + kAttnTmemO, p_desc + static_cast<uint64_t>(ks * 2), vd, id_pv,
-                         (j > 0 || ks > 0) ? 1u : 0u);
+            mma_ts(tmem + kAttnTmemO, tmem + kAttnTmemP + ks * 8, vd, id_pv, (j > 0 || ks > 0) ? 1u : 0u);
           }
           mma_commit(&sm->kv_empty[sj]);
           mma_commit(&sm->pv_done);
@@ -422,11 +409,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     const int quarter = warp & 3;
     const int h = quarter * 32 + lane;                 // head row = TMEM lane
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    float* xrow = x_buf + h * kAttnTileN;
-    const uint32_t peer_x = peer_addr(xrow, peer);
-    const uint32_t peer_x_full = peer_addr(&sm->x_full, peer);
-    const uint32_t peer_x_free = peer_addr(&sm->x_free, peer);
-    uint8_t* prow = p_buf + h * 128;
+    constexpr uint32_t kXBytes = kAttnHeads * kAttnTileN * 4;           // one exchange buffer
+    const uint32_t peer_x = peer_addr(x_buf + h * kAttnTileN, peer);   // + buffer * kXBytes
+    const uint32_t peer_x_full = peer_addr(&sm->x_full[0], peer);      // + buffer * 8
     float m = -__int_as_float(0x7f800000), l = 0.f;
     bool ok = true;
     {
@@ -467,28 +452,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       tc_fence_before();
       mbar_arrive(&sm->s_empty);
       // exchange the partial logits with the peer.  Each thread's 64 values go
-      // to its row of the peer's buffer as 16-byte st.async pieces that count
-      // themselves on the peer's x_full (which expects one tile of bytes from
-      // a local arrive); the peer may write my buffer again once all my
-      // threads have read it (one remote arrive on its x_free).  Rows are
+      // to its row of the peer's buffer for this tile's parity as 16-byte
+      // st.async pieces that count themselves on the peer's x_full of that
+      // parity (which expects one tile of bytes from a local arrive).  The
+      // peer writes a buffer again two tiles later, after it has received my
+      // next tile's pieces, which I send after reading this one.  Rows are
       // swizzled by 16-byte piece (piece c at c ^ (h & 7)), so a warp's
       // accesses to 32 rows spread over every bank.
-      if (h == 0) mbar_arrive_expect_tx(&sm->x_full, kAttnHeads * kAttnTileN * 4);
-      if (i >= 1 &&
-          !(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_free, static_cast<uint32_t>((i - 1) & 1), abort_flag))))
-        break;
+      const int xb = i & 1;
+      if (h == 0) mbar_arrive_expect_tx(&sm->x_full[xb], kXBytes);
 #pragma unroll
       for (int c = 0; c < 16; ++c)
-        st_async_v4(peer_x + ((c ^ (h & 7)) << 4), s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3], peer_x_full);
-      if (!(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_full, static_cast<uint32_t>(i & 1), abort_flag)))) break;
-      const float4* x4 = reinterpret_cast<const float4*>(xrow);
+        st_async_v4(peer_x + xb * kXBytes + ((c ^ (h & 7)) << 4), s[4 * c], s[4 * c + 1], s[4 * c + 2],
+                    s[4 * c + 3], peer_x_full + xb * 8);
+      if (!(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_full[xb], static_cast<uint32_t>((i >> 1) & 1),
+                                                     abort_flag))))
+        break;
+      const float4* x4 = reinterpret_cast<const float4*>(x_buf + xb * (kAttnHeads * kAttnTileN) + h * kAttnTileN);
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const float4 v = x4[c ^ (h & 7)];
         s[4 * c + 0] += v.x; s[4 * c + 1] += v.y; s[4 * c + 2] += v.z; s[4 * c + 3] += v.w;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(peer_x_free);  // this warp's rows of my buffer have been read
       // online softmax in the log2 domain: logits past the last key are -inf,
       // whose exp2 is 0; maxima and sums in four independent chains
       const int nk = min(kAttnTileN, n_valid - i * kAttnTileN);
@@ -520,18 +505,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       if (i >= 1 &&
           !(ok = __all_sync(kFull, mbar_wait(&sm->pv_done, static_cast<uint32_t>((i - 1) & 1), abort_flag))))
         break;
-      // P row (64 keys, bf16) in the 128-byte-swizzled K-major layout
+      tc_fence_after();
+      // P row (64 keys, bf16 pairs) into TMEM: the A operand of this tile's PV
+      {
+        uint32_t v[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 v;
-        v.x = pack_bf16x2(s[8 * c + 0], s[8 * c + 1]);
-        v.y = pack_bf16x2(s[8 * c + 2], s[8 * c + 3]);
-        v.z = pack_bf16x2(s[8 * c + 4], s[8 * c + 5]);
-        v.w = pack_bf16x2(s[8 * c + 6], s[8 * c + 7]);
-        *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) = v;
+        for (int c = 0; c < 32; ++c) v[c] = pack_bf16x2(s[2 * c], s[2 * c + 1]);
+        tmem_st32(t_lane + kAttnTmemP, v);
       }
       if (i >= 1) {
-        tc_fence_after();
         if (__any_sync(kFull, corr != 1.f)) {          // rows whose maximum did not grow scale by 1
 #pragma unroll 1
           for (int c0 = 0; c0 < 256; c0 += 32) {
@@ -542,10 +524,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
             for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * corr);
             tmem_st32(t_lane + kAttnTmemO + c0, v);
           }
-          tmem_wait_st();
         }
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm->p_full);
     }
