@@ -37,8 +37,8 @@
 // Warp roles (8 warps):
 //   warp 0      TMEM owner, single-thread MMA issuer (QK of tile i, then
 //               PV of tile i-1)
-//   warps 1..3  key gather by TMA, one warp per key stage (stage s: tiles
-//               s, s+3, ...), each tile completing on its stage's barrier
+//   warps 1..3  key gather by TMA: every tile's gather4 operations dealt
+//               over the three warps, completing on the tile's stage barrier
 //   warps 4..7  softmax: thread = head row; q into TMEM, exchange, online
 //               softmax, O rescaling and P (bf16) in TMEM, epilogue
 // Every wait is bounded; a timeout sets the CTA's abort flag and the status
@@ -58,9 +58,14 @@ constexpr int kAttnThreads = 256;
 constexpr int kAttnGatherBase = 32;        // warps 1..3
 constexpr int kAttnSoftBase = 128;         // warps 4..7
 constexpr int kAttnStages = 3;             // key stages
+constexpr int kAttnPer = kAttnMaxK / kAttnThreads;     // index-row places per thread
+constexpr int kAttnHashBits = 13;
+constexpr int kAttnHash = 1 << kAttnHashBits;          // dedup slots (2 x kAttnMaxK), in the key stages
 constexpr int kAttnPanels = 5;             // 64-feature panels of the larger half
 constexpr uint32_t kAttnPanelK = kAttnTileN * 128;     // bytes of one key panel (64 rows x 128 B)
 constexpr uint32_t kAttnStage = kAttnPanels * kAttnPanelK;
+static_assert(kAttnMaxK % kAttnThreads == 0 && kAttnPer <= 32, "one keep bit per place of a thread's run");
+static_assert(kAttnHash >= 2 * kAttnMaxK && kAttnHash * 8 <= kAttnStages * kAttnStage, "dedup table fits the stages");
 constexpr uint32_t kAttnTmemS = 0;         // one 64-column logit buffer
 constexpr uint32_t kAttnTmemQ = 64;        // the query part: 2 bf16 per column, up to 160 columns
 constexpr uint32_t kAttnTmemP = 224;       // softmax weights of one tile: 64 bf16 = 32 columns
@@ -139,6 +144,17 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
       : "memory");
+}
+
+// A hint to bring the 128-byte line holding `ptr` into L2.
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(ptr)));
+}
+
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (TMA) accesses of the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // 16 bytes into another CTA's shared memory, counted as complete_tx bytes on
@@ -225,7 +241,7 @@ struct AttnSmem {
 inline size_t attn_smem_bytes() {
   return 1024 + kAttnStages * kAttnStage       // key tiles
          + 2 * kAttnHeads * kAttnTileN * 4     // partial logits from the peer, two buffers
-         + kAttnMaxK * 4                       // the query's sorted, deduplicated positions
+         + kAttnMaxK * 4                       // the query's deduplicated positions
          + sizeof(AttnSmem) + 16;
 }
 
@@ -249,12 +265,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
   const int b = static_cast<int>(row / p.Q);
   const int npanels = rank == 0 ? 4 : 5;
   const int feat0 = rank == 0 ? 0 : 256;
-  const int chunks_per_key = npanels * 8;                // 16-byte pieces of this CTA's part of a key row
 
   if (tid == 0) {
     mbar_init(&sm->q_full, 128);
     for (int i = 0; i < kAttnStages; ++i) {
-      mbar_init(&sm->kv_full[i], 1);
+      mbar_init(&sm->kv_full[i], 3);            // one byte-announcing arrive per gather warp
       mbar_init(&sm->kv_empty[i], 1);
     }
     mbar_init(&sm->s_full, 1);
@@ -270,44 +285,63 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
   if (warp == 0) tmem_alloc(&sm->tmem_base, 512);
   if (warp == 1 && lane == 0) tma_prefetch_desc(&kvmap);
 
-  // ---- the query's positions: sorted, -1 / out-of-range / repeats dropped, compacted
-  const int K = p.top_k;
-  int npow = 1;
-  while (npow < K) npow <<= 1;
-  const int32_t* irow = p.idx + row * K;
-  for (int i = tid; i < npow; i += kAttnThreads) {
-    int v = i < K ? __ldg(irow + i) : INT32_MAX;
-    if (v < 0 || v >= p.L) v = INT32_MAX;             // not a key: sorts last, dropped below
-    sidx[i] = v;
+  if (warp >= kAttnSoftBase / 32) {
+    // this head's part of the query towards L2 while the index row is read
+    const char* qg = reinterpret_cast<const char*>(
+        p.q + ((row * p.slices + slice) * kAttnHeads + (tid - kAttnSoftBase)) * static_cast<int64_t>(kAttnDqk) + feat0);
+    for (int c = 0; c < npanels; ++c) prefetch_l2(qg + c * 128);
   }
-  __syncthreads();
-  for (int size = 2; size <= npow; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int q2 = tid; q2 < (npow >> 1); q2 += kAttnThreads) {
-        const int i = 2 * q2 - (q2 & (stride - 1)), j = i + stride;
-        const bool up = (i & size) == 0;
-        const int a = sidx[i], c = sidx[j];
-        if ((a > c) == up) { sidx[i] = c; sidx[j] = a; }
-      }
-      __syncthreads();
-    }
-  }
+
+  // ---- the query's positions: -1, out-of-range entries and repeats dropped,
+  // compacted in row order.  Each thread takes a contiguous run of the row;
+  // a hash table in the (still unused) key stages maps a position to the
+  // first place of the row where it occurs, and a place is kept when it is
+  // that first place.  The result does not depend on the order of the
+  // atomics, so it is the same on every run.
   {
-    // keep the first of each run of equal positions; compact in order
-    const int per = (npow + kAttnThreads - 1) / kAttnThreads;
-    const int lo = tid * per, hi = min(npow, lo + per);
-    int keep[16];
-    int cnt = 0;
-    for (int i = lo; i < hi; ++i) {
-      const int v = sidx[i];
-      const bool k = v != INT32_MAX && (i == 0 || sidx[i - 1] != v);
-      keep[i - lo] = k ? v : -1;
-      cnt += k;
+    uint32_t* hkey = reinterpret_cast<uint32_t*>(kv_buf);
+    int32_t* hfirst = reinterpret_cast<int32_t*>(kv_buf + kAttnHash * 4);
+    const int K = p.top_k;
+    const int per = (K + kAttnThreads - 1) / kAttnThreads;   // at most kAttnMaxK / kAttnThreads
+    const int lo = min(K, tid * per), hi = min(K, lo + per);
+    const int32_t* irow = p.idx + row * K;
+    int v[kAttnPer];
+#pragma unroll
+    for (int u = 0; u < kAttnPer; ++u) {
+      int x = lo + u < hi ? __ldg(irow + lo + u) : -1;
+      v[u] = x < p.L ? x : -1;                         // negative: not a key
     }
+    for (int i = tid; i < kAttnHash / 4; i += kAttnThreads) {
+      reinterpret_cast<uint4*>(hkey)[i] = make_uint4(~0u, ~0u, ~0u, ~0u);
+      reinterpret_cast<int4*>(hfirst)[i] = make_int4(INT32_MAX, INT32_MAX, INT32_MAX, INT32_MAX);
+    }
+    __syncthreads();
+    int slot[kAttnPer];
+#pragma unroll
+    for (int u = 0; u < kAttnPer; ++u) {
+      slot[u] = -1;
+      if (v[u] >= 0) {
+        // open addressing; at most kAttnMaxK distinct keys in twice as many slots
+        uint32_t hs = (static_cast<uint32_t>(v[u]) * 0x9E3779B1u) >> (32 - kAttnHashBits);
+        for (int probe = 0; probe < kAttnHash; ++probe) {
+          const uint32_t prev = atomicCAS(&hkey[hs], ~0u, static_cast<uint32_t>(v[u]));
+          if (prev == ~0u || prev == static_cast<uint32_t>(v[u])) break;
+          hs = (hs + 1) & (kAttnHash - 1);
+        }
+        atomicMin(&hfirst[hs], lo + u);
+        slot[u] = static_cast<int>(hs);
+      }
+    }
+    __syncthreads();
+    uint32_t keep = 0;
+#pragma unroll
+    for (int u = 0; u < kAttnPer; ++u)
+      if (slot[u] >= 0 && hfirst[slot[u]] == lo + u) keep |= 1u << u;
+    const int cnt = __popc(keep);
     int incl = cnt;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      const int o = __shfl_up_sync(kFull, incl, off);
       if (lane >= off) incl += o;
     }
     if (lane == 31) sm->scan[warp] = incl;
@@ -315,11 +349,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     int base = 0;
     for (int w2 = 0; w2 < warp; ++w2) base += sm->scan[w2];
     if (tid == kAttnThreads - 1) sm->n_valid = base + incl;
-    __syncthreads();                                   // every thread has read sidx[lo-1] before any write
     int pos = base + incl - cnt;
-    for (int i = lo; i < hi; ++i)
-      if (keep[i - lo] >= 0) sidx[pos++] = keep[i - lo];
+#pragma unroll
+    for (int u = 0; u < kAttnPer; ++u)
+      if (keep & (1u << u)) sidx[pos++] = v[u];
   }
+  // the table's generic-proxy accesses are ordered before the key gathers
+  // (async proxy) that will overwrite it
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   cluster_sync();                                      // the peer's barriers exist before any remote arrive
@@ -371,22 +408,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     }
   } else if (warp < kAttnSoftBase / 32) {
     // ------------------------------------------------------------ key gather
-    // warp 1 + s fills stage s with tiles s, s + 4, ...: per tile, 16 groups of
-    // four key rows x this CTA's panels, one gather4 each, spread over the lanes
-    const int grp = warp - kAttnGatherBase / 32;       // stage 0..3
+    // warps 1..3 share every tile: its 16 x npanels gather4 operations (four
+    // key rows x one 64-feature panel each) are dealt round-robin over the
+    // three warps, one per lane, and each warp announces its own bytes on
+    // the stage's barrier
+    const int gw = warp - kAttnGatherBase / 32;        // 0..2
     const int kbase = b * p.L;
-    uint8_t* stage = kv_buf + grp * kAttnStage;
-    const uint32_t tile_bytes = static_cast<uint32_t>(npanels) * kAttnPanelK;
-    bool ok = true;
+    const int nops = 16 * npanels;
+    const uint32_t my_bytes = static_cast<uint32_t>((nops - gw + 2) / 3) * 4 * 128;
     int issued = 0;
-    for (int i = grp; i < T; i += kAttnStages) {
+    for (int i = 0; i < T; ++i) {
+      const int st = i % kAttnStages;
       int okl = 1;
       if (lane == 0)
-        okl = mbar_wait(&sm->kv_empty[grp], static_cast<uint32_t>(((i / kAttnStages) & 1) ^ 1), abort_flag);
-      if (!(ok = __shfl_sync(kFull, okl, 0) != 0)) break;
-      if (lane == 0) mbar_arrive_expect_tx(&sm->kv_full[grp], tile_bytes);
+        okl = mbar_wait(&sm->kv_empty[st], static_cast<uint32_t>(((i / kAttnStages) & 1) ^ 1), abort_flag);
+      if (__shfl_sync(kFull, okl, 0) == 0) break;
+      if (lane == 0) mbar_arrive_expect_tx(&sm->kv_full[st], my_bytes);
       __syncwarp();
-      for (int x = lane; x < 16 * npanels; x += 32) {
+      const int x = gw + 3 * lane;
+      if (x < nops) {
         const int g4 = x & 15, pn = x >> 4;
         int y[4];
 #pragma unroll
@@ -394,15 +434,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
           const int e = i * kAttnTileN + 4 * g4 + u;
           y[u] = kbase + sidx[e < n_valid ? e : 0];       // past the last position: any valid row, masked later
         }
-        tma_gather4(smem_u32(stage + pn * kAttnPanelK + g4 * 4 * 128), &kvmap, &sm->kv_full[grp],
-                    feat0 + 64 * pn, y[0], y[1], y[2], y[3]);
+        tma_gather4(smem_u32(kv_buf + st * kAttnStage + pn * kAttnPanelK + g4 * 4 * 128), &kvmap,
+                    &sm->kv_full[st], feat0 + 64 * pn, y[0], y[1], y[2], y[3]);
       }
       ++issued;
     }
-    if (lane == 0 && issued > 0) {
-      // leave only once this warp's last tile has landed
-      const int last = grp + kAttnStages * (issued - 1);
-      mbar_drain(&sm->kv_full[grp], static_cast<uint32_t>((last / kAttnStages) & 1));
+    if (lane == 0) {
+      // leave only once this warp's copies have landed: the last tile of each stage
+      for (int j = max(0, issued - kAttnStages); j < issued; ++j)
+        mbar_drain(&sm->kv_full[j % kAttnStages], static_cast<uint32_t>((j / kAttnStages) & 1));
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -415,18 +455,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     float m = -__int_as_float(0x7f800000), l = 0.f;
     bool ok = true;
     {
-      // this head's part of the query into TMEM, 64 features (32 columns) at a time
+      // this head's part of the query into TMEM, 64 features (32 columns) at a
+      // time, the next panel's loads in flight while one is stored
       const uint4* qg = reinterpret_cast<const uint4*>(
           p.q + ((row * p.slices + slice) * kAttnHeads + h) * static_cast<int64_t>(kAttnDqk) + feat0);
+      uint32_t v[32];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint4 x = __ldg(qg + u);
+        v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
+      }
 #pragma unroll 1
       for (int pn = 0; pn < npanels; ++pn) {
-        uint32_t v[32];
+        uint4 nx[8];
+        if (pn + 1 < npanels) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint4 x = __ldg(qg + pn * 8 + u);
-          v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
+          for (int u = 0; u < 8; ++u) nx[u] = __ldg(qg + (pn + 1) * 8 + u);
         }
         tmem_st32(t_lane + kAttnTmemQ + pn * 32, v);
+        if (pn + 1 < npanels) {
+          tmem_wait_st();                              // v is rewritten below
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            v[4 * u] = nx[u].x; v[4 * u + 1] = nx[u].y; v[4 * u + 2] = nx[u].z; v[4 * u + 3] = nx[u].w;
+          }
+        }
       }
       tmem_wait_st();
       tc_fence_before();
