@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* kv_buf = smem;
-  float* x_buf = reinterpret_cast<float*>(kv_buf + kAttnStages * kAttnStage);   // [2][128][64]
+  float* x_buf = reinterpret_cast<float*>(kv_buf + kAttnStages * kAttnStage);   // [2 parities][16 pieces][128 rows][4]
   int32_t* sidx = reinterpret_cast<int32_t*>(x_buf + 2 * kAttnHeads * kAttnTileN);
   AttnSmem* sm = reinterpret_cast<AttnSmem*>(sidx + kAttnMaxK);
   volatile int* abort_flag = &sm->abort_flag;
@@ -450,7 +450,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     const int h = quarter * 32 + lane;                 // head row = TMEM lane
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     constexpr uint32_t kXBytes = kAttnHeads * kAttnTileN * 4;           // one exchange buffer
-    const uint32_t peer_x = peer_addr(x_buf + h * kAttnTileN, peer);   // + buffer * kXBytes
+    const uint32_t peer_x = peer_addr(x_buf + h * 4, peer);            // + buffer * kXBytes + piece * 2 KB
     const uint32_t peer_x_full = peer_addr(&sm->x_full[0], peer);      // + buffer * 8
     float m = -__int_as_float(0x7f800000), l = 0.f;
     bool ok = true;
@@ -505,26 +505,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       tc_fence_before();
       mbar_arrive(&sm->s_empty);
       // exchange the partial logits with the peer.  Each thread's 64 values go
-      // to its row of the peer's buffer for this tile's parity as 16-byte
-      // st.async pieces that count themselves on the peer's x_full of that
-      // parity (which expects one tile of bytes from a local arrive).  The
-      // peer writes a buffer again two tiles later, after it has received my
-      // next tile's pieces, which I send after reading this one.  Rows are
-      // swizzled by 16-byte piece (piece c at c ^ (h & 7)), so a warp's
-      // accesses to 32 rows spread over every bank.
+      // to the peer's buffer for this tile's parity as 16 16-byte st.async
+      // pieces that count themselves on the peer's x_full of that parity
+      // (which expects one tile of bytes from a local arrive).  The peer
+      // writes a buffer again two tiles later, after it has received my next
+      // tile's pieces, which I send after reading this one.  The buffer is
+      // piece-major, [piece c][head row h][16 B]: the 32 pieces one warp
+      // instruction sends are 512 contiguous bytes (a scattered row-major
+      // layout moved about half as many bytes per cycle between the SMs),
+      // and the reads below are conflict-free.
       const int xb = i & 1;
       if (h == 0) mbar_arrive_expect_tx(&sm->x_full[xb], kXBytes);
 #pragma unroll
       for (int c = 0; c < 16; ++c)
-        st_async_v4(peer_x + xb * kXBytes + ((c ^ (h & 7)) << 4), s[4 * c], s[4 * c + 1], s[4 * c + 2],
+        st_async_v4(peer_x + xb * kXBytes + c * (kAttnHeads * 16), s[4 * c], s[4 * c + 1], s[4 * c + 2],
                     s[4 * c + 3], peer_x_full + xb * 8);
       if (!(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_full[xb], static_cast<uint32_t>((i >> 1) & 1),
                                                      abort_flag))))
         break;
-      const float4* x4 = reinterpret_cast<const float4*>(x_buf + xb * (kAttnHeads * kAttnTileN) + h * kAttnTileN);
+      const float4* x4 = reinterpret_cast<const float4*>(x_buf + xb * (kAttnHeads * kAttnTileN)) + h;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const float4 v = x4[c ^ (h & 7)];
+        const float4 v = x4[c * kAttnHeads];
         s[4 * c + 0] += v.x; s[4 * c + 1] += v.y; s[4 * c + 2] += v.z; s[4 * c + 3] += v.w;
       }
       // online softmax in the log2 domain: logits past the last key are -inf,
