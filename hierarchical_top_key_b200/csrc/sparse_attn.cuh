@@ -229,7 +229,7 @@ struct AttnSmem {
   uint64_t kv_full[kAttnStages], kv_empty[kAttnStages];
   uint64_t s_full, s_empty;
   uint64_t p_full, pv_done;
-  uint64_t x_full[2];            // partial logits of the peer CTA, one buffer per tile parity
+  uint64_t x_full[2][2];         // partial logits of the peer CTA: [tile parity][key half]
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -277,7 +277,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     mbar_init(&sm->p_full, 128);
     mbar_init(&sm->pv_done, 1);
     for (int i = 0; i < 2; ++i)
-      mbar_init(&sm->x_full[i], 1);   // local arrive with the tile's byte count + the peer's st.async bytes
+      for (int hf = 0; hf < 2; ++hf)
+        mbar_init(&sm->x_full[i][hf], 1);   // local arrive with a half tile's bytes + the peer's st.async bytes
     mbar_init(&sm->drain, 1);
     sm->abort_flag = 0;
     fence_barrier_init();
@@ -451,7 +452,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     constexpr uint32_t kXBytes = kAttnHeads * kAttnTileN * 4;           // one exchange buffer
     const uint32_t peer_x = peer_addr(x_buf + h * 4, peer);            // + buffer * kXBytes + piece * 2 KB
-    const uint32_t peer_x_full = peer_addr(&sm->x_full[0], peer);      // + buffer * 8
+    const uint32_t peer_x_full = peer_addr(&sm->x_full[0][0], peer);   // + (buffer * 2 + half) * 8
     float m = -__int_as_float(0x7f800000), l = 0.f;
     bool ok = true;
     {
@@ -506,56 +507,70 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       mbar_arrive(&sm->s_empty);
       // exchange the partial logits with the peer.  Each thread's 64 values go
       // to the peer's buffer for this tile's parity as 16 16-byte st.async
-      // pieces that count themselves on the peer's x_full of that parity
-      // (which expects one tile of bytes from a local arrive).  The peer
-      // writes a buffer again two tiles later, after it has received my next
-      // tile's pieces, which I send after reading this one.  The buffer is
-      // piece-major, [piece c][head row h][16 B]: the 32 pieces one warp
-      // instruction sends are 512 contiguous bytes (a scattered row-major
-      // layout moved about half as many bytes per cycle between the SMs),
-      // and the reads below are conflict-free.
+      // pieces that count themselves on the peer's x_full of that parity and
+      // key half (each expects half a tile of bytes from a local arrive).
+      // The peer writes a buffer again two tiles later, after it has received
+      // my next tile's pieces, which I send after reading this one.  The
+      // buffer is piece-major, [piece c][head row h][16 B]: the 32 pieces one
+      // warp instruction sends are 512 contiguous bytes (a scattered
+      // row-major layout moved about half as many bytes per cycle between the
+      // SMs), and the reads below are conflict-free.  Keys 0..31 (pieces
+      // 0..7) go first: their softmax runs while keys 32..63 are in flight.
       const int xb = i & 1;
-      if (h == 0) mbar_arrive_expect_tx(&sm->x_full[xb], kXBytes);
+      if (h == 0) {
+        mbar_arrive_expect_tx(&sm->x_full[xb][0], kXBytes / 2);
+        mbar_arrive_expect_tx(&sm->x_full[xb][1], kXBytes / 2);
+      }
 #pragma unroll
       for (int c = 0; c < 16; ++c)
         st_async_v4(peer_x + xb * kXBytes + c * (kAttnHeads * 16), s[4 * c], s[4 * c + 1], s[4 * c + 2],
-                    s[4 * c + 3], peer_x_full + xb * 8);
-      if (!(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_full[xb], static_cast<uint32_t>((i >> 1) & 1),
-                                                     abort_flag))))
-        break;
+                    s[4 * c + 3], peer_x_full + (xb * 2 + (c >> 3)) * 8);
       const float4* x4 = reinterpret_cast<const float4*>(x_buf + xb * (kAttnHeads * kAttnTileN)) + h;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float4 v = x4[c * kAttnHeads];
-        s[4 * c + 0] += v.x; s[4 * c + 1] += v.y; s[4 * c + 2] += v.z; s[4 * c + 3] += v.w;
-      }
-      // online softmax in the log2 domain: logits past the last key are -inf,
-      // whose exp2 is 0; maxima and sums in four independent chains
       const int nk = min(kAttnTileN, n_valid - i * kAttnTileN);
-      float mx4[4] = {-__int_as_float(0x7f800000), -__int_as_float(0x7f800000), -__int_as_float(0x7f800000),
-                      -__int_as_float(0x7f800000)};
-#pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        s[j] = j < nk ? s[j] * p.scale_log2 : -__int_as_float(0x7f800000);
-        mx4[j & 3] = fmaxf(mx4[j & 3], s[j]);
-      }
-      // the reference maximum moves only when the tile's maximum exceeds it by
-      // more than 8 (a factor 256): the weights stay below 2^8, the output rows
-      // are rescaled rarely, and o = sum p v / sum p is the same for any
+      // online softmax in the log2 domain over the two key halves in turn:
+      // logits past the last key are -inf, whose exp2 is 0.  The reference
+      // maximum moves only when a half's maximum exceeds it by more than 8 (a
+      // factor 256): the weights stay below 2^8, the output rows are
+      // rescaled rarely, and o = sum p v / sum p is the same for any
       // reference (the natural-log lse adds back the reference that was used)
-      const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      const bool move = i == 0 || mt > m + 8.f;
-      const float mx = move ? mt : m;
-      const float corr = (i == 0) ? 0.f : (move ? fast_exp2(m - mx) : 1.f);
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      float corr = 1.f;                                // this tile's factor on O
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        s[j] = fast_exp2(s[j] - mx);
-        sum4[j & 3] += s[j];
+      for (int hf = 0; hf < 2; ++hf) {
+        if (!(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_full[xb][hf], static_cast<uint32_t>((i >> 1) & 1),
+                                                       abort_flag))))
+          break;
+        float mx4[4] = {-__int_as_float(0x7f800000), -__int_as_float(0x7f800000), -__int_as_float(0x7f800000),
+                        -__int_as_float(0x7f800000)};
+#pragma unroll
+        for (int c = 8 * hf; c < 8 * hf + 8; ++c) {
+          const float4 v = x4[c * kAttnHeads];
+          s[4 * c + 0] += v.x; s[4 * c + 1] += v.y; s[4 * c + 2] += v.z; s[4 * c + 3] += v.w;
+        }
+#pragma unroll
+        for (int j = 32 * hf; j < 32 * hf + 32; ++j) {
+          s[j] = j < nk ? s[j] * p.scale_log2 : -__int_as_float(0x7f800000);
+          mx4[j & 3] = fmaxf(mx4[j & 3], s[j]);
+        }
+        const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const bool first = i == 0 && hf == 0;        // key 0 of tile 0 exists: mt is finite
+        const bool move = first || mt > m + 8.f;
+        const float mx = move ? mt : m;
+        const float c = first ? 0.f : (move ? fast_exp2(m - mx) : 1.f);
+        if (hf == 1 && move) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) s[j] *= c;     // the first half's weights, to the new reference
+        }
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 32 * hf; j < 32 * hf + 32; ++j) {
+          s[j] = fast_exp2(s[j] - mx);
+          sum4[j & 3] += s[j];
+        }
+        l = l * c + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+        m = mx;
+        corr *= c;
       }
-      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-      l = l * corr + sum;
-      m = mx;
+      if (!ok) break;
       // P and O belong to the previous tile's PV until it completes
       if (i >= 1 &&
           !(ok = __all_sync(kFull, mbar_wait(&sm->pv_done, static_cast<uint32_t>((i - 1) & 1), abort_flag))))
