@@ -116,8 +116,11 @@ int num_sms() {
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 
+// A 2D map over [rows, cols] with boxes of box_rows x (128 bytes of columns,
+// or box_cols columns), 128-byte swizzle unless another is given.
 hisa_status tensor_map_2d(CUtensorMap* map, const void* base, int dtype, uint64_t rows, uint64_t cols,
-                          uint32_t box_rows, uint64_t row_stride_elems = 0) {
+                          uint32_t box_rows, uint64_t row_stride_elems = 0, uint32_t box_cols = 0,
+                          CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   if (!g_encode_tiled) {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -130,10 +133,10 @@ hisa_status tensor_map_2d(CUtensorMap* map, const void* base, int dtype, uint64_
   const CUtensorMapDataType ty = dtype == HISA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {(row_stride_elems ? row_stride_elems : cols) * es};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), box_rows};
+  cuuint32_t box[2] = {box_cols ? box_cols : static_cast<cuuint32_t>(128 / es), box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode_tiled(map, ty, 2, const_cast<void*>(base), dims, strides, box, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(HISA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return HISA_OK;
@@ -1031,8 +1034,13 @@ hisa_status hisa_sparse_attention(const void* q, const void* kv, const int32_t* 
   if (rows * slices * 2 > INT32_MAX) return fail(HISA_ERR_UNSUPPORTED, "too many (query, head slice) pairs");
   if (static_cast<int64_t>(batch) * num_keys > INT32_MAX)
     return fail(HISA_ERR_UNSUPPORTED, "batch * num_keys must fit in int32 (key row coordinates)");
-  CUtensorMap kvm;
+  // one-row boxes for the gathers: 64 value features (128-byte swizzle) and
+  // 32 positional features (64-byte swizzle)
+  CUtensorMap kvm, ropem;
   hisa_status e = tensor_map_2d(&kvm, kv, HISA_BF16, static_cast<uint64_t>(batch) * num_keys, kAttnDqk, 1);
+  if (e != HISA_OK) return e;
+  e = tensor_map_2d(&ropem, kv, HISA_BF16, static_cast<uint64_t>(batch) * num_keys, kAttnDqk, 1, 0, 32,
+                    CU_TENSOR_MAP_SWIZZLE_64B);
   if (e != HISA_OK) return e;
   const size_t smem = attn_smem_bytes();
   e = cuda_check(cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1054,7 +1062,7 @@ hisa_status hisa_sparse_attention(const void* q, const void* kv, const int32_t* 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cuda_check(cudaLaunchKernelEx(&cfg, sparse_attn_kernel, kvm, p), "launch sparse_attn_kernel");
+  e = cuda_check(cudaLaunchKernelEx(&cfg, sparse_attn_kernel, kvm, ropem, p), "launch sparse_attn_kernel");
   if (e != HISA_OK) return e;
   return launch_check("sparse_attn_kernel");
 }

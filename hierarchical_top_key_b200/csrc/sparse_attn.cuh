@@ -54,22 +54,30 @@ constexpr int kAttnDqk = 576;
 constexpr int kAttnDv = 512;
 constexpr int kAttnTileN = 64;             // keys per tile
 constexpr int kAttnMaxK = 4096;            // longest index row
-constexpr int kAttnThreads = 256;
-constexpr int kAttnGatherBase = 32;        // warps 1..3
-constexpr int kAttnSoftBase = 128;         // warps 4..7
-constexpr int kAttnStages = 3;             // key stages
-constexpr int kAttnPer = kAttnMaxK / kAttnThreads;     // index-row places per thread
+constexpr int kAttnThreads = 320;
+constexpr int kAttnPvWarp = 1;             // warp 0 issues the logit MMAs, warp 1 the output MMAs
+constexpr int kAttnGatherBase = 64;        // warps 2..5
+constexpr int kAttnGatherWarps = 4;
+constexpr int kAttnSoftBase = 192;         // warps 6..9
+constexpr int kAttnStages = 4;             // key stages
+constexpr int kAttnPer = (kAttnMaxK + kAttnThreads - 1) / kAttnThreads;   // index-row places per thread
 constexpr int kAttnHashBits = 13;
 constexpr int kAttnHash = 1 << kAttnHashBits;          // dedup slots (2 x kAttnMaxK), in the key stages
-constexpr int kAttnPanels = 5;             // 64-feature panels of the larger half
-constexpr uint32_t kAttnPanelK = kAttnTileN * 128;     // bytes of one key panel (64 rows x 128 B)
-constexpr uint32_t kAttnStage = kAttnPanels * kAttnPanelK;
-static_assert(kAttnMaxK % kAttnThreads == 0 && kAttnPer <= 32, "one keep bit per place of a thread's run");
+constexpr int kAttnPanels = 4;             // 64-feature value panels per CTA
+constexpr uint32_t kAttnPanelK = kAttnTileN * 128;     // bytes of one value panel (64 rows x 128 B)
+constexpr uint32_t kAttnRopeK = kAttnTileN * 64;       // bytes of the positional half panel (64 rows x 64 B)
+constexpr uint32_t kAttnStage = kAttnPanels * kAttnPanelK + kAttnRopeK;
+constexpr int kAttnKsteps = kAttnPanels * 4 + 2;       // K = 288 features per CTA, 16 per MMA
+constexpr int kAttnGatherOps = 16 * kAttnPanels + 16;  // gather4 operations per tile: 4 key rows each
+static_assert(kAttnPer <= 32 && kAttnPer * kAttnThreads >= kAttnMaxK, "one keep bit per place of a thread's run");
 static_assert(kAttnHash >= 2 * kAttnMaxK && kAttnHash * 8 <= kAttnStages * kAttnStage, "dedup table fits the stages");
+static_assert(kAttnGatherOps % kAttnGatherWarps == 0 && 16 * kAttnPanels % kAttnGatherWarps == 0 &&
+                  kAttnGatherOps <= 32 * kAttnGatherWarps, "equal gather shares, one operation per lane");
 constexpr uint32_t kAttnTmemS = 0;         // one 64-column logit buffer
-constexpr uint32_t kAttnTmemQ = 64;        // the query part: 2 bf16 per column, up to 160 columns
-constexpr uint32_t kAttnTmemP = 224;       // softmax weights of one tile: 64 bf16 = 32 columns
+constexpr uint32_t kAttnTmemQ = 64;        // the query part: 2 bf16 per column, 144 columns
+constexpr uint32_t kAttnTmemP = 208;       // softmax weights of one tile: 64 bf16 = 32 columns
 constexpr uint32_t kAttnTmemO = 256;       // 256 output columns
+static_assert(kAttnTmemQ + kAttnKsteps * 8 <= kAttnTmemP && kAttnTmemP + 32 <= kAttnTmemO, "TMEM map");
 constexpr unsigned kFull = 0xffffffffu;
 
 struct AttnParams {
@@ -178,6 +186,29 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 32 lanes x 16 consecutive 32-bit columns from registers into TMEM.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Shared-memory descriptor of a K-major operand stored by TMA with the
+// 64-byte swizzle: rows of 64 bytes (32 bf16), 8-row atoms of 512 bytes
+// (stride byte offset 512), layout type 4; version 1 (sm_100).
+__device__ __forceinline__ uint64_t desc_k_sw64(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>(512 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(4) << 61;
+  return d;
+}
+
 // Shared-memory descriptor of an MN-major operand stored with the 128-byte
 // swizzle: rows of 128 bytes hold 64 consecutive MN elements for one K index,
 // 8-row groups along K are `sbo` bytes apart and 64-element groups along MN
@@ -230,7 +261,7 @@ struct AttnSmem {
   uint64_t s_full, s_empty;
   uint64_t p_full, pv_done;
   uint64_t x_full[2][2];         // partial logits of the peer CTA: [tile parity][key half]
-  uint64_t drain;
+  uint64_t drain[2];             // one per MMA issuer
   uint32_t tmem_base;
   int abort_flag;
   int n_valid;
@@ -238,14 +269,15 @@ struct AttnSmem {
   int scan[kAttnThreads / 32 + 1];
 };
 
-inline size_t attn_smem_bytes() {
-  return 1024 + kAttnStages * kAttnStage       // key tiles
-         + 2 * kAttnHeads * kAttnTileN * 4     // partial logits from the peer, two buffers
-         + kAttnMaxK * 4                       // the query's deduplicated positions
-         + sizeof(AttnSmem) + 16;
-}
+constexpr size_t kAttnSmemBytes = 1024 + kAttnStages * kAttnStage   // key tiles (1 KB for alignment)
+                                  + 2 * kAttnHeads * kAttnTileN * 4  // partial logits from the peer, two buffers
+                                  + kAttnMaxK * 4                    // the query's deduplicated positions
+                                  + sizeof(AttnSmem) + 16;
+static_assert(kAttnSmemBytes <= 232448, "dynamic shared memory of one CTA");
+inline size_t attn_smem_bytes() { return kAttnSmemBytes; }
 
 __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __grid_constant__ CUtensorMap kvmap,
+                                                                     const __grid_constant__ CUtensorMap ropemap,
                                                                      const AttnParams p) {
   using namespace sm100;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -257,19 +289,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
   volatile int* abort_flag = &sm->abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = cluster_ctarank();               // 0: features 0..255, 1: features 256..575
+  const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
   const int64_t item = cluster_id_x();                   // (row, head slice)
   const int64_t row = item / p.slices;
   const int slice = static_cast<int>(item % p.slices);
   const int b = static_cast<int>(row / p.Q);
-  const int npanels = rank == 0 ? 4 : 5;
-  const int feat0 = rank == 0 ? 0 : 256;
+  const int val0 = 256 * static_cast<int>(rank);          // this CTA's value features: val0 .. val0 + 255
+  const int rope0 = kAttnDv + 32 * static_cast<int>(rank); // and positional features rope0 .. rope0 + 31
 
   if (tid == 0) {
     mbar_init(&sm->q_full, 128);
     for (int i = 0; i < kAttnStages; ++i) {
-      mbar_init(&sm->kv_full[i], 3);            // one byte-announcing arrive per gather warp
+      mbar_init(&sm->kv_full[i], kAttnGatherWarps);   // one byte-announcing arrive per gather warp
       mbar_init(&sm->kv_empty[i], 1);
     }
     mbar_init(&sm->s_full, 1);
@@ -279,18 +311,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     for (int i = 0; i < 2; ++i)
       for (int hf = 0; hf < 2; ++hf)
         mbar_init(&sm->x_full[i][hf], 1);   // local arrive with a half tile's bytes + the peer's st.async bytes
-    mbar_init(&sm->drain, 1);
+    mbar_init(&sm->drain[0], 1);
+    mbar_init(&sm->drain[1], 1);
     sm->abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0) tmem_alloc(&sm->tmem_base, 512);
-  if (warp == 1 && lane == 0) tma_prefetch_desc(&kvmap);
+  if (warp == 2 && lane == 0) {
+    tma_prefetch_desc(&kvmap);
+    tma_prefetch_desc(&ropemap);
+  }
 
   if (warp >= kAttnSoftBase / 32) {
     // this head's part of the query towards L2 while the index row is read
-    const char* qg = reinterpret_cast<const char*>(
-        p.q + ((row * p.slices + slice) * kAttnHeads + (tid - kAttnSoftBase)) * static_cast<int64_t>(kAttnDqk) + feat0);
-    for (int c = 0; c < npanels; ++c) prefetch_l2(qg + c * 128);
+    const uint16_t* qh = p.q + ((row * p.slices + slice) * kAttnHeads + (tid - kAttnSoftBase)) *
+                                   static_cast<int64_t>(kAttnDqk);
+    for (int c = 0; c < kAttnPanels; ++c) prefetch_l2(qh + val0 + 64 * c);
+    prefetch_l2(qh + rope0);
   }
 
   // ---- the query's positions: -1, out-of-range entries and repeats dropped,
@@ -367,56 +404,69 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
   const int T = (n_valid + kAttnTileN - 1) / kAttnTileN;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ logit MMA issuer
+    // S = q_c . k_c^T for tile k as soon as its keys have landed and the
+    // softmax has read tile k-1 out of the single logit buffer; the output
+    // MMAs come from another thread, so these never queue behind them
     if (lane == 0) {
       constexpr uint32_t id_qk = instr_desc(kAttnHeads, kAttnTileN, 1u);
-      constexpr uint32_t id_pv = instr_desc_bmn(kAttnHeads, 256);
       bool ok = T == 0 || mbar_wait(&sm->q_full, 0, abort_flag);
       if (ok) tc_fence_after();
-      const int ksteps = npanels * 4;
-      for (int i = 0; ok && i <= T; ++i) {
-        if (i < T) {
-          const int st = i % kAttnStages;
-          if (!(ok = mbar_wait(&sm->kv_full[st], static_cast<uint32_t>((i / kAttnStages) & 1), abort_flag))) break;
-          // the single logit buffer is free once the softmax has read tile i-1
-          if (i >= 1 && !(ok = mbar_wait(&sm->s_empty, static_cast<uint32_t>((i - 1) & 1), abort_flag))) break;
-          tc_fence_after();
-          const uint64_t k_desc = desc_k_sw128(smem_u32(kv_buf + st * kAttnStage));
-#pragma unroll 4
-          for (int ks = 0; ks < ksteps; ++ks)
-            mma_ts(tmem + kAttnTmemS, tmem + kAttnTmemQ + ks * 8,
-                   k_desc + static_cast<uint64_t>((ks >> 2) * (kAttnTileN * 128 / 16) + (ks & 3) * 2), id_qk,
-                   ks > 0 ? 1u : 0u);
-          mma_commit(&sm->s_full);
-        }
-        if (i >= 1) {
-          const int j = i - 1, sj = j % kAttnStages;
-          if (!(ok = mbar_wait(&sm->p_full, static_cast<uint32_t>(j & 1), abort_flag))) break;
-          tc_fence_after();
-          // V: the first four 64-feature panels of the key tile, MN-major
-          const uint32_t v0 = smem_u32(kv_buf + sj * kAttnStage);
+      for (int k = 0; ok && k < T; ++k) {
+        const int st = k % kAttnStages;
+        if (!(ok = mbar_wait(&sm->kv_full[st], static_cast<uint32_t>((k / kAttnStages) & 1), abort_flag))) break;
+        if (k >= 1 && !(ok = mbar_wait(&sm->s_empty, static_cast<uint32_t>((k - 1) & 1), abort_flag))) break;
+        tc_fence_after();
+        const uint32_t base = smem_u32(kv_buf + st * kAttnStage);
+        const uint64_t k_desc = desc_k_sw128(base);
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t vd = desc_mn_sw128(v0 + ks * 16 * 128, kAttnPanelK, 1024);
-            mma_ts(tmem + kAttnTmemO, tmem + kAttnTmemP + ks * 8, vd, id_pv, (j > 0 || ks > 0) ? 1u : 0u);
-          }
-          mma_commit(&sm->kv_empty[sj]);
-          mma_commit(&sm->pv_done);
-        }
+        for (int ks = 0; ks < 4 * kAttnPanels; ++ks)
+          mma_ts(tmem + kAttnTmemS, tmem + kAttnTmemQ + ks * 8,
+                 k_desc + static_cast<uint64_t>((ks >> 2) * (kAttnPanelK / 16) + (ks & 3) * 2), id_qk, ks > 0 ? 1u : 0u);
+        const uint64_t r_desc = desc_k_sw64(base + kAttnPanels * kAttnPanelK);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          mma_ts(tmem + kAttnTmemS, tmem + kAttnTmemQ + (4 * kAttnPanels + ks) * 8, r_desc + static_cast<uint64_t>(ks * 2),
+                 id_qk, 1u);
+        mma_commit(&sm->s_full);
       }
-      mma_commit(&sm->drain);
-      mbar_drain(&sm->drain, 0);
+      mma_commit(&sm->drain[0]);
+      mbar_drain(&sm->drain[0], 0);
+    }
+  } else if (warp == kAttnPvWarp) {
+    // ------------------------------------------------------------ output MMA issuer
+    // O_c += P . V_c for tile j once the softmax has written P_j; the tile's
+    // key stage is free when this MMA completes
+    if (lane == 0) {
+      constexpr uint32_t id_pv = instr_desc_bmn(kAttnHeads, 256);
+      bool ok = true;
+      for (int j = 0; ok && j < T; ++j) {
+        const int sj = j % kAttnStages;
+        if (!(ok = mbar_wait(&sm->p_full, static_cast<uint32_t>(j & 1), abort_flag))) break;
+        tc_fence_after();
+        // V: the four 64-feature value panels of the key tile, MN-major
+        const uint32_t v0 = smem_u32(kv_buf + sj * kAttnStage);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t vd = desc_mn_sw128(v0 + ks * 16 * 128, kAttnPanelK, 1024);
+          mma_ts(tmem + kAttnTmemO, tmem + kAttnTmemP + ks * 8, vd, id_pv, (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(&sm->kv_empty[sj]);
+        mma_commit(&sm->pv_done);
+      }
+      mma_commit(&sm->drain[1]);
+      mbar_drain(&sm->drain[1], 0);
     }
   } else if (warp < kAttnSoftBase / 32) {
     // ------------------------------------------------------------ key gather
-    // warps 1..3 share every tile: its 16 x npanels gather4 operations (four
-    // key rows x one 64-feature panel each) are dealt round-robin over the
-    // three warps, one per lane, and each warp announces its own bytes on
-    // the stage's barrier
-    const int gw = warp - kAttnGatherBase / 32;        // 0..2
+    // warps 2..5 share every tile: its gather4 operations (four key rows of
+    // one 64-feature value panel, or of the 32 positional features) are dealt
+    // round-robin over the warps, one per lane, and each warp announces its
+    // own bytes on the stage's barrier
+    const int gw = warp - kAttnGatherBase / 32;        // 0..3
     const int kbase = b * p.L;
-    const int nops = 16 * npanels;
-    const uint32_t my_bytes = static_cast<uint32_t>((nops - gw + 2) / 3) * 4 * 128;
+    constexpr uint32_t my_bytes = (16 * kAttnPanels / kAttnGatherWarps) * 4 * 128 + (16 / kAttnGatherWarps) * 4 * 64;
+    static_assert(my_bytes * kAttnGatherWarps == kAttnStage, "gather shares cover the stage");
     int issued = 0;
     for (int i = 0; i < T; ++i) {
       const int st = i % kAttnStages;
@@ -426,17 +476,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       if (__shfl_sync(kFull, okl, 0) == 0) break;
       if (lane == 0) mbar_arrive_expect_tx(&sm->kv_full[st], my_bytes);
       __syncwarp();
-      const int x = gw + 3 * lane;
-      if (x < nops) {
-        const int g4 = x & 15, pn = x >> 4;
+      const int x = gw + kAttnGatherWarps * lane;
+      if (x < kAttnGatherOps) {
+        const bool rope = x >= 16 * kAttnPanels;
+        const int g4 = rope ? x - 16 * kAttnPanels : (x & 15);
         int y[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int e = i * kAttnTileN + 4 * g4 + u;
           y[u] = kbase + sidx[e < n_valid ? e : 0];       // past the last position: any valid row, masked later
         }
-        tma_gather4(smem_u32(kv_buf + st * kAttnStage + pn * kAttnPanelK + g4 * 4 * 128), &kvmap,
-                    &sm->kv_full[st], feat0 + 64 * pn, y[0], y[1], y[2], y[3]);
+        uint8_t* stage = kv_buf + st * kAttnStage;
+        const uint32_t dst = rope ? smem_u32(stage + kAttnPanels * kAttnPanelK + g4 * 4 * 64)
+                                  : smem_u32(stage + (x >> 4) * kAttnPanelK + g4 * 4 * 128);
+        tma_gather4(dst, rope ? &ropemap : &kvmap, &sm->kv_full[st], rope ? rope0 : val0 + 64 * (x >> 4), y[0],
+                    y[1], y[2], y[3]);
       }
       ++issued;
     }
@@ -456,10 +510,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
     float m = -__int_as_float(0x7f800000), l = 0.f;
     bool ok = true;
     {
-      // this head's part of the query into TMEM, 64 features (32 columns) at a
-      // time, the next panel's loads in flight while one is stored
-      const uint4* qg = reinterpret_cast<const uint4*>(
-          p.q + ((row * p.slices + slice) * kAttnHeads + h) * static_cast<int64_t>(kAttnDqk) + feat0);
+      // this head's part of the query into TMEM: the four value panels (32
+      // columns each, the next panel's loads in flight while one is stored),
+      // then the 32 positional features (16 columns)
+      const uint16_t* qh = p.q + ((row * p.slices + slice) * kAttnHeads + h) * static_cast<int64_t>(kAttnDqk);
+      const uint4* qg = reinterpret_cast<const uint4*>(qh + val0);
+      const uint4* qr = reinterpret_cast<const uint4*>(qh + rope0);
+      uint4 rq[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) rq[u] = __ldg(qr + u);
       uint32_t v[32];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -467,14 +526,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
         v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
       }
 #pragma unroll 1
-      for (int pn = 0; pn < npanels; ++pn) {
+      for (int pn = 0; pn < kAttnPanels; ++pn) {
         uint4 nx[8];
-        if (pn + 1 < npanels) {
+        if (pn + 1 < kAttnPanels) {
 #pragma unroll
           for (int u = 0; u < 8; ++u) nx[u] = __ldg(qg + (pn + 1) * 8 + u);
         }
         tmem_st32(t_lane + kAttnTmemQ + pn * 32, v);
-        if (pn + 1 < npanels) {
+        if (pn + 1 < kAttnPanels) {
           tmem_wait_st();                              // v is rewritten below
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -482,101 +541,107 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
           }
         }
       }
+      uint32_t r16[16];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        r16[4 * u] = rq[u].x; r16[4 * u + 1] = rq[u].y; r16[4 * u + 2] = rq[u].z; r16[4 * u + 3] = rq[u].w;
+      }
+      tmem_st16(t_lane + kAttnTmemQ + 32 * kAttnPanels, r16);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm->q_full);
     }
-    for (int i = 0; ok && i < T; ++i) {
-      // every wait below is taken by all lanes and its outcome made warp-uniform:
-      // the tcgen05 loads and stores that follow are .sync.aligned
-      if (!(ok = __all_sync(kFull, mbar_wait(&sm->s_full, static_cast<uint32_t>(i & 1), abort_flag)))) break;
+    // Every wait below is taken by all lanes and its outcome made
+    // warp-uniform: the tcgen05 loads and stores that follow are .sync.aligned.
+    //
+    // This CTA's partial logits of a tile go to the peer's exchange buffer
+    // for the tile's parity as 16 16-byte st.async pieces per thread, which
+    // count themselves on the peer's x_full of that parity and key half (each
+    // expects half a tile of bytes from a local arrive).  The buffer is
+    // piece-major, [piece c][head row h][16 B]: the 32 pieces one warp
+    // instruction sends are 512 contiguous bytes (a scattered row-major
+    // layout moved about half as many bytes per cycle between the SMs), and
+    // the reads are conflict-free.  The partial logits of tile i+1 leave
+    // before the softmax of tile i, so the exchange overlaps that work.  A
+    // buffer is written again two tiles later: the peer sends tile i+1 after
+    // it has received all of my tile i, which each of my threads sends after
+    // reading its rows of tile i-1 from the same buffer.
+    auto load_send = [&](float (&dst)[64], int tile) -> bool {
+      if (!__all_sync(kFull, mbar_wait(&sm->s_full, static_cast<uint32_t>(tile & 1), abort_flag))) return false;
       tc_fence_after();
-      float s[64];
-      {
-        uint32_t v[32];
-        tmem_ld32(t_lane + kAttnTmemS, v);
-        tmem_wait_ld();
+      uint32_t v[32];
+      tmem_ld32(t_lane + kAttnTmemS, v);
+      tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
-        tmem_ld32(t_lane + kAttnTmemS + 32, v);
-        tmem_wait_ld();
+      for (int j = 0; j < 32; ++j) dst[j] = __uint_as_float(v[j]);
+      tmem_ld32(t_lane + kAttnTmemS + 32, v);
+      tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) s[32 + j] = __uint_as_float(v[j]);
-      }
+      for (int j = 0; j < 32; ++j) dst[32 + j] = __uint_as_float(v[j]);
       tc_fence_before();
       mbar_arrive(&sm->s_empty);
-      // exchange the partial logits with the peer.  Each thread's 64 values go
-      // to the peer's buffer for this tile's parity as 16 16-byte st.async
-      // pieces that count themselves on the peer's x_full of that parity and
-      // key half (each expects half a tile of bytes from a local arrive).
-      // The peer writes a buffer again two tiles later, after it has received
-      // my next tile's pieces, which I send after reading this one.  The
-      // buffer is piece-major, [piece c][head row h][16 B]: the 32 pieces one
-      // warp instruction sends are 512 contiguous bytes (a scattered
-      // row-major layout moved about half as many bytes per cycle between the
-      // SMs), and the reads below are conflict-free.  Keys 0..31 (pieces
-      // 0..7) go first: their softmax runs while keys 32..63 are in flight.
-      const int xb = i & 1;
+      const int xb = tile & 1;
       if (h == 0) {
         mbar_arrive_expect_tx(&sm->x_full[xb][0], kXBytes / 2);
         mbar_arrive_expect_tx(&sm->x_full[xb][1], kXBytes / 2);
       }
 #pragma unroll
       for (int c = 0; c < 16; ++c)
-        st_async_v4(peer_x + xb * kXBytes + c * (kAttnHeads * 16), s[4 * c], s[4 * c + 1], s[4 * c + 2],
-                    s[4 * c + 3], peer_x_full + (xb * 2 + (c >> 3)) * 8);
+        st_async_v4(peer_x + xb * kXBytes + c * (kAttnHeads * 16), dst[4 * c], dst[4 * c + 1], dst[4 * c + 2],
+                    dst[4 * c + 3], peer_x_full + (xb * 2 + (c >> 3)) * 8);
+      return true;
+    };
+    float s[64], sn[64];
+    if (T > 0) ok = load_send(s, 0);
+    for (int i = 0; ok && i < T; ++i) {
+      // 1. the peer's part of tile i, sent one tile ago
+      const int xb = i & 1;
+      if (!(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_full[xb][0], static_cast<uint32_t>((i >> 1) & 1),
+                                                     abort_flag) &&
+                                       mbar_wait_cluster(&sm->x_full[xb][1], static_cast<uint32_t>((i >> 1) & 1),
+                                                         abort_flag))))
+        break;
       const float4* x4 = reinterpret_cast<const float4*>(x_buf + xb * (kAttnHeads * kAttnTileN)) + h;
-      const int nk = min(kAttnTileN, n_valid - i * kAttnTileN);
-      // online softmax in the log2 domain over the two key halves in turn:
-      // logits past the last key are -inf, whose exp2 is 0.  The reference
-      // maximum moves only when a half's maximum exceeds it by more than 8 (a
-      // factor 256): the weights stay below 2^8, the output rows are
-      // rescaled rarely, and o = sum p v / sum p is the same for any
-      // reference (the natural-log lse adds back the reference that was used)
-      float corr = 1.f;                                // this tile's factor on O
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        if (!(ok = __all_sync(kFull, mbar_wait_cluster(&sm->x_full[xb][hf], static_cast<uint32_t>((i >> 1) & 1),
-                                                       abort_flag))))
-          break;
-        float mx4[4] = {-__int_as_float(0x7f800000), -__int_as_float(0x7f800000), -__int_as_float(0x7f800000),
-                        -__int_as_float(0x7f800000)};
-#pragma unroll
-        for (int c = 8 * hf; c < 8 * hf + 8; ++c) {
-          const float4 v = x4[c * kAttnHeads];
-          s[4 * c + 0] += v.x; s[4 * c + 1] += v.y; s[4 * c + 2] += v.z; s[4 * c + 3] += v.w;
-        }
-#pragma unroll
-        for (int j = 32 * hf; j < 32 * hf + 32; ++j) {
-          s[j] = j < nk ? s[j] * p.scale_log2 : -__int_as_float(0x7f800000);
-          mx4[j & 3] = fmaxf(mx4[j & 3], s[j]);
-        }
-        const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-        const bool first = i == 0 && hf == 0;        // key 0 of tile 0 exists: mt is finite
-        const bool move = first || mt > m + 8.f;
-        const float mx = move ? mt : m;
-        const float c = first ? 0.f : (move ? fast_exp2(m - mx) : 1.f);
-        if (hf == 1 && move) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) s[j] *= c;     // the first half's weights, to the new reference
-        }
-        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 32 * hf; j < 32 * hf + 32; ++j) {
-          s[j] = fast_exp2(s[j] - mx);
-          sum4[j & 3] += s[j];
-        }
-        l = l * c + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
-        m = mx;
-        corr *= c;
+      for (int c = 0; c < 16; ++c) {
+        const float4 v = x4[c * kAttnHeads];
+        s[4 * c + 0] += v.x; s[4 * c + 1] += v.y; s[4 * c + 2] += v.z; s[4 * c + 3] += v.w;
       }
-      if (!ok) break;
-      // P and O belong to the previous tile's PV until it completes
+      // 2. my part of tile i+1 out to the peer
+      if (i + 1 < T && !(ok = load_send(sn, i + 1))) break;
+      // 3. online softmax of tile i in the log2 domain: logits past the last
+      // key are -inf, whose exp2 is 0; maxima and sums in four independent
+      // chains.  The reference maximum moves only when the tile's maximum
+      // exceeds it by more than 8 (a factor 256): the weights stay below 2^8,
+      // the output rows are rescaled rarely, and o = sum p v / sum p is the
+      // same for any reference (the natural-log lse adds back the reference
+      // that was used)
+      const int nk = min(kAttnTileN, n_valid - i * kAttnTileN);
+      float mx4[4] = {-__int_as_float(0x7f800000), -__int_as_float(0x7f800000), -__int_as_float(0x7f800000),
+                      -__int_as_float(0x7f800000)};
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        s[j] = j < nk ? s[j] * p.scale_log2 : -__int_as_float(0x7f800000);
+        mx4[j & 3] = fmaxf(mx4[j & 3], s[j]);
+      }
+      const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      const bool move = i == 0 || mt > m + 8.f;
+      const float mx = move ? mt : m;
+      const float corr = (i == 0) ? 0.f : (move ? fast_exp2(m - mx) : 1.f);
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        s[j] = fast_exp2(s[j] - mx);
+        sum4[j & 3] += s[j];
+      }
+      l = l * corr + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+      m = mx;
+      // P and O belong to the previous tile's output MMA until it completes
       if (i >= 1 &&
           !(ok = __all_sync(kFull, mbar_wait(&sm->pv_done, static_cast<uint32_t>((i - 1) & 1), abort_flag))))
         break;
       tc_fence_after();
-      // P row (64 keys, bf16 pairs) into TMEM: the A operand of this tile's PV
+      // P row (64 keys, bf16 pairs) into TMEM: the A operand of this tile's output MMA
       {
         uint32_t v[32];
 #pragma unroll
@@ -599,6 +664,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_kernel(const __gr
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm->p_full);
+#pragma unroll
+      for (int j = 0; j < 64; ++j) s[j] = sn[j];
     }
     // ---- epilogue: O / l in bf16, and lse
     const int64_t orow = (row * p.slices + slice) * kAttnHeads + h;
