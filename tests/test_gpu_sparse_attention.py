@@ -92,3 +92,44 @@ def test_consumes_the_indexer_output(lib):
     hidx = idx.cpu().numpy()
     o, lse = _run(q, kv, hidx)
     _check(q[0], kv[0], hidx[0], o[0], lse[0], range(wl.num_queries), "indexer -> attention")
+
+
+def _bf16(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def test_output_rescaled_when_the_maximum_jumps(lib):
+    """The online softmax moves its reference maximum only when a tile's
+    maximum exceeds it by more than 8 (log2 units), and then rescales the
+    output rows.  With i.i.d. N(0, 1) rows that never happens after the first
+    tile, so here keys aligned with each query's mean head direction are
+    planted at chosen places of its index row (tiles 2, 9 and 20), each
+    raising the maximum by some tens; a few heads are anti-aligned and keep
+    their reference, so rows of one warp rescale and others do not."""
+    Q, L, K = 6, 4096, 2048
+    q, kv = synthetic.attention_inputs(1, Q, L, seed=21)
+    idx = synthetic.random_index_rows(1, Q, L, K, np.full((1, Q), L), seed=21)
+    used = set()
+    for t in range(Q):
+        u = q[0, t].astype(np.float64).sum(axis=0)
+        u /= np.linalg.norm(u)
+        for place, c in ((2 * 64 + 7, 120.0), (9 * 64 + 33, 240.0), (20 * 64 + 63, 360.0)):
+            pos = int(idx[0, t, place])
+            if pos in used:
+                continue
+            used.add(pos)
+            kv[0, pos] = _bf16(c * u)
+    o, lse = _run(q, kv, idx)
+    _check(q[0], kv[0], idx[0], o[0], lse[0], range(Q), "planted maxima")
+    # the planted keys do dominate: lse far above what unplanted rows give
+    assert np.median(lse[0]) > 30.0
+
+
+def test_two_head_slices(lib):
+    """256 query heads: two 128-head slices, each its own pair of CTAs."""
+    Q, L, K = 5, 3000, 500
+    q, kv = synthetic.attention_inputs(1, Q, L, seed=8, heads=256)
+    idx = synthetic.random_index_rows(1, Q, L, K, np.full((1, Q), L), seed=8)
+    o, lse = _run(q, kv, idx)
+    assert o.shape == (1, Q, 256, synthetic.ATTN_DV) and lse.shape == (1, Q, 256)
+    _check(q[0], kv[0], idx[0], o[0], lse[0], range(Q), "256 heads")
