@@ -14,32 +14,33 @@
 // One query's 128 heads are the M = 128 rows of every MMA, on a pair of CTAs
 // (a cluster of two).  Neither the query (128 x 576 bf16 = 144 KB) nor the
 // 512 fp32 accumulator columns of the output fit one SM next to the key
-// tiles and the scores, so the pair splits the features:
-//   CTA 0  features   0..255: q and key columns for part of every logit,
-//          the value columns   0..255 of the output
-//   CTA 1  features 256..575: the rest of every logit (with the 64
-//          positional features), the value columns 256..511
+// tiles and the scores, so the pair splits the features 288/288:
+//   CTA r  value features 256r .. 256r+255 (four 64-feature panels) and
+//          positional features 512+32r .. 512+32r+31 (one 32-feature panel,
+//          64-byte swizzle): its part of every logit, and the value columns
+//          256r .. 256r+255 of the output
 // Each CTA keeps its part of the query in TMEM (the A operand of the logit
 // MMA, loaded once per query) and the softmax weights P there too (the A
-// operand of the output MMA), so that shared memory holds three key stages
-// and two exchange buffers;
-// it computes a partial logit tile S_c = q_c . k_c^T (M = 128 heads,
-// N = 64 keys, K = its features) on tcgen05 into TMEM, the two partial tiles
-// are exchanged through distributed shared memory (one buffer per tile
-// parity, so no "buffer free" handshake is needed) and summed (the sum is the
-// same in both CTAs: fp32 addition commutes), and both run the same online
-// softmax, so each can accumulate its half of the output, O_c += P . V_c,
-// with V_c the value columns it already holds (B operand read MN-major from
-// the key tile).  Keys are gathered from their positions by the TMA engine,
-// four rows per instruction (tile::gather4 over a one-row box), straight into
-// the 128-byte-swizzled layout the MMA reads.
+// operand of the output MMA), so that shared memory holds four key stages
+// and two exchange buffers.  Per 64-key tile it computes a partial logit
+// tile S_c = q_c . k_c^T (M = 128 heads, N = 64 keys, K = 288) on tcgen05
+// into TMEM; the two partial tiles are exchanged through distributed shared
+// memory (one buffer per tile parity, so no "buffer free" handshake is
+// needed; each tile's exchange is sent before the softmax of the previous
+// tile, so it overlaps that work) and summed (the same in both CTAs: fp32
+// addition commutes); both run the same online softmax, so each can
+// accumulate its half of the output, O_c += P . V_c, with V_c the value
+// columns it already holds (B operand read MN-major from the key tile).
+// Keys are gathered from their positions by the TMA engine, four rows per
+// instruction (tile::gather4 over a one-row box), straight into the swizzled
+// layouts the MMA reads.
 //
-// Warp roles (8 warps):
-//   warp 0      TMEM owner, single-thread MMA issuer (QK of tile i, then
-//               PV of tile i-1)
-//   warps 1..3  key gather by TMA: every tile's gather4 operations dealt
-//               over the three warps, completing on the tile's stage barrier
-//   warps 4..7  softmax: thread = head row; q into TMEM, exchange, online
+// Warp roles (10 warps):
+//   warp 0      TMEM owner, logit MMA issuer (one thread)
+//   warp 1      output MMA issuer (one thread)
+//   warps 2..5  key gather by TMA: every tile's gather4 operations dealt
+//               over the four warps, completing on the tile's stage barrier
+//   warps 6..9  softmax: thread = head row; q into TMEM, exchange, online
 //               softmax, O rescaling and P (bf16) in TMEM, epilogue
 // Every wait is bounded; a timeout sets the CTA's abort flag and the status
 // word, and the peer CTA's waits on it then time out too.
