@@ -142,6 +142,31 @@ hisa_status tensor_map_2d(CUtensorMap* map, const void* base, int dtype, uint64_
   return HISA_OK;
 }
 
+// A 3D map over [rows, 2 panels of 128 bytes] for 2-panel rows (256 bytes):
+// dims {elements per panel, rows, 2}, strides {row bytes, 128 bytes}, boxes of
+// box_rows rows x both panels, 128-byte swizzle.  One load of a box fills
+// [panel][row][128 B] in shared memory.
+hisa_status tensor_map_3d_panels(CUtensorMap* map, const void* base, int dtype, uint64_t rows, uint64_t cols,
+                                 uint32_t box_rows) {
+  if (!g_encode_tiled) {
+    CUtensorMap probe;
+    hisa_status e = tensor_map_2d(&probe, base, dtype, rows, cols, 1);   // resolves the entry point
+    if (e != HISA_OK) return e;
+  }
+  const int es = elem_bytes(dtype);
+  const uint64_t panel = 128 / es;
+  const CUtensorMapDataType ty = dtype == HISA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  cuuint64_t dims[3] = {panel, rows, cols / panel};
+  cuuint64_t strides[2] = {cols * es, 128};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(panel), box_rows, static_cast<cuuint32_t>(cols / panel)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode_tiled(map, ty, 3, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HISA_ERR_CUDA, "cuTensorMapEncodeTiled (3D panels) failed (%d)", static_cast<int>(r));
+  return HISA_OK;
+}
+
 // ------------------------------------------------------------ dense scoring plan
 
 // Tensor-core path: bf16 or E4M3 rows of 128/256 bytes, and H that divides 256
@@ -348,7 +373,10 @@ hisa_status launch_token_tc(const hisa_shape* s, const void* q, const float* qsc
   if (e != HISA_OK) return e;
   const uint64_t key_rows = pg.table ? static_cast<uint64_t>(pg.count) * s->block_size
                                     : static_cast<uint64_t>(s->batch) * s->num_keys;
-  e = tensor_map_2d(&km, k, s->dtype, key_rows, s->head_dim, s->block_size);
+  // a 128-key block of 256-byte rows is one load of both panels
+  p.k3d = s->block_size == kTokTileM && rb == 256;
+  e = p.k3d ? tensor_map_3d_panels(&km, k, s->dtype, key_rows, s->head_dim, s->block_size)
+            : tensor_map_2d(&km, k, s->dtype, key_rows, s->head_dim, s->block_size);
   if (e != HISA_OK) return e;
   auto kern = token_tc_kernel<DT, H>;
   e = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),

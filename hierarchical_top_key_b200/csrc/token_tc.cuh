@@ -60,6 +60,8 @@ struct TokenParams {
   int parts;                // > 1: each query's retained blocks split over `parts` jobs, each writing its own top-k
   const int32_t* pages;     // non-NULL: block j of sequence b is page pages[b * nb + j] of the keys ([num_pages, B, d])
   int num_pages;
+  int k3d;                  // 1: the key map is 3D (64 elements, rows, 2 panels of 128 bytes): a block of 128
+                            //    rows is one load; 0: one 2D load per block and panel
 };
 
 struct alignas(16) TokJob {
@@ -271,9 +273,15 @@ __global__ void __launch_bounds__(kTokThreads, 1) token_tc_kernel(
           mbar_arrive_expect_tx(kf, static_cast<uint32_t>(nblk_t * p.B * row_bytes));
           for (int q = 0; q < nblk_t; ++q) {
             const int krow = p.pages ? J.page[first + q] * p.B : kb + J.blk[first + q] * p.B;
-            for (int pn = 0; pn < panels; ++pn)
-              tma_load_2d(k_buf + st * k_bytes + pn * (kTokTileM * 128) + q * p.B * 128, &kmap, kf,
-                          pn * panel_elems, krow);
+            if (p.k3d) {
+              // both panels of the block in one instruction: the box is [panel][row][128 B],
+              // the layout the panel loads below produce
+              tma_load_3d(k_buf + st * k_bytes, &kmap, kf, 0, krow, 0);
+            } else {
+              for (int pn = 0; pn < panels; ++pn)
+                tma_load_2d(k_buf + st * k_bytes + pn * (kTokTileM * 128) + q * p.B * 128, &kmap, kf,
+                            pn * panel_elems, krow);
+            }
           }
           last_ph[st] = static_cast<int8_t>((fph >> kfi) & 1u);
           last_bar[st] = static_cast<int8_t>(kfi);
