@@ -14,6 +14,7 @@ import subprocess
 import sys
 
 import numpy as np
+import pytest
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -135,3 +136,50 @@ def test_reference_arm_runs_on_rank_zero_only():
                         "--workload", "tiny", "--steps", "1", "--warmup", "0", "--cpu-seconds", "1"],
                        env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def _leaving_rank_main(rank, world, port, out):
+    import datetime
+    import time
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    from hierarchical_top_key_b200 import partition, synthetic
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+    if rank == 1:
+        # this rank leaves between steps, before the shard all-gather
+        dist.destroy_process_group()
+        out[rank] = "left"
+        return
+    wl = synthetic.WORKLOADS["tiny"]
+    inp = synthetic.generate(wl, 0, batch=1)
+    shards = partition.shard_job(inp.n_visible, wl.block_size, wl.top_m, world)
+    mine = torch.full((1, shards[0].t1 - shards[0].t0, wl.top_k), -1, dtype=torch.int32)
+    t0 = time.monotonic()
+    try:
+        bench.gather_shards(mine, shards, wl.batch, wl.num_queries, wl.top_k, world)
+        out[rank] = ("gathered", time.monotonic() - t0)
+    except Exception as e:                              # the collective ends with an error, not a hang
+        out[rank] = ("error", time.monotonic() - t0, type(e).__name__)
+    finally:
+        try:
+            dist.destroy_process_group()
+        except Exception:
+            pass
+
+
+@pytest.mark.timeout(180)
+def test_a_rank_that_leaves_fails_the_gather_instead_of_hanging():
+    """Failure detection on the host: a rank that leaves before the shard
+    all-gather of a query split makes the remaining rank's collective end with
+    an error within the process group's timeout (10 s here), not wait for good."""
+    world = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_leaving_rank_main, args=(world, _free_port(), out), nprocs=world, start_method="spawn")
+        res = dict(out)
+    assert res[1] == "left"
+    assert res[0][0] == "error", res[0]
+    assert res[0][1] < 60.0
